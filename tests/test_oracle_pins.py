@@ -1,0 +1,341 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Closed forms, explicit-loop brute force, invariants, library routines
+(scipy softmax, torch's bf16 conversion) and the hand-worked commit example
+in tests/golden/.  No GPU needed.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import twotower_oracle as O
+import tt_inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rnd(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- bf16 format
+def test_round_bf16_ties_and_specials():
+    one = 1.0
+    ulp = 2.0 ** -7
+    assert O.round_bf16(np.array([one + ulp / 2]))[0] == one                # tie -> even (1.0)
+    assert O.round_bf16(np.array([one + 1.5 * ulp]))[0] == one + 2 * ulp    # tie -> even
+    assert O.round_bf16(np.array([one + 0.51 * ulp]))[0] == one + ulp
+    assert O.round_bf16(np.array([-3.0]))[0] == -3.0
+    assert O.round_bf16(np.array([0.0]))[0] == 0.0
+    assert O.round_bf16(np.array([1e39]))[0] == np.inf
+    assert O.round_bf16(np.array([2.0 ** -130]))[0] == 2.0 ** -130          # subnormal, exact
+
+
+def test_round_bf16_matches_torch_and_input_module():
+    x32 = (rnd(20000, 1) * np.exp(rnd(20000, 2) * 8)).astype(np.float32)
+    mine = O.round_bf16(x32.astype(np.float64))
+    ref_torch = torch.from_numpy(x32).to(torch.bfloat16).to(torch.float64).numpy()
+    ref_inputs = O.from_bf16(tt_inputs.bf16_bits(x32))
+    np.testing.assert_array_equal(mine, ref_torch)
+    np.testing.assert_array_equal(mine, ref_inputs)
+
+
+def test_from_bf16_exact():
+    bits = np.array([0x3F80, 0xBF80, 0x4000, 0x0000, 0x3F81, 0x7F80], dtype=np.uint16)
+    np.testing.assert_array_equal(O.from_bf16(bits), [1.0, -1.0, 2.0, 0.0, 1.0 + 2 ** -7, np.inf])
+
+
+# ------------------------------------------------------------------ attention
+def _attn_inputs(B, S, Hq, Hkv, dh, L, seed=0, scale=1.0):
+    q = rnd((B, S, Hq, dh), seed, scale)
+    kb = rnd((B, S, Hkv, dh), seed + 1, scale)
+    vb = rnd((B, S, Hkv, dh), seed + 2)
+    kc = rnd((B, Hkv, L, dh), seed + 3, scale)
+    vc = rnd((B, Hkv, L, dh), seed + 4)
+    return q, kb, vb, kc, vc
+
+
+def test_attention_matches_explicit_loops():
+    q, kb, vb, kc, vc = _attn_inputs(2, 3, 4, 2, 5, 6, seed=10)
+    ctx_len = np.array([4, 0])
+    a = O.block_attention(q, kb, vb, kc, vc, ctx_len)
+    b = O.block_attention_loops(q, kb, vb, kc, vc, ctx_len)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_hand_example_joint_softmax_and_scale():
+    # dh = 4: one context key with score 2*1/sqrt(4) = 1, one block key with
+    # score 0.  Joint softmax gives weights e/(e+1) and 1/(e+1).
+    q = np.zeros((1, 1, 1, 4)); q[0, 0, 0, 0] = 2.0
+    kc = np.zeros((1, 1, 1, 4)); kc[0, 0, 0, 0] = 1.0
+    kb = np.zeros((1, 1, 1, 4))
+    vc = np.zeros((1, 1, 1, 4)); vc[0, 0, 0, 0] = 1.0
+    vb = np.zeros((1, 1, 1, 4)); vb[0, 0, 0, 1] = 1.0
+    o = O.block_attention(q, kb, vb, kc, vc, np.array([1]))
+    e = math.e
+    np.testing.assert_allclose(o[0, 0, 0], [e / (e + 1), 1 / (e + 1), 0, 0], rtol=1e-14)
+
+
+def test_attention_closed_forms():
+    # no context, one block position: the only key is the block's own -> o = v
+    q, kb, vb, kc, vc = _attn_inputs(1, 1, 4, 2, 8, 3, seed=3)
+    o = O.block_attention(q, kb, vb, kc, vc, np.array([0]))
+    for h in range(4):
+        np.testing.assert_allclose(o[0, 0, h], vb[0, 0, h // 2], rtol=1e-14)
+    # all keys equal -> uniform weights -> mean of the values
+    q, kb, vb, kc, vc = _attn_inputs(1, 4, 2, 1, 8, 5, seed=4)
+    kb[:] = 0.3
+    kc[:] = 0.3
+    o = O.block_attention(q, kb, vb, kc, vc, np.array([5]))
+    allv = np.concatenate([vc[0, 0], vb[0, :, 0]])
+    np.testing.assert_allclose(o[0, 2, 1], allv.mean(axis=0), rtol=1e-12)
+
+
+def test_attention_block_permutation_equivariance():
+    q, kb, vb, kc, vc = _attn_inputs(2, 6, 4, 2, 8, 7, seed=5, scale=2.0)
+    ctx_len = np.array([7, 3])
+    o = O.block_attention(q, kb, vb, kc, vc, ctx_len)
+    perm = np.random.default_rng(0).permutation(6)
+    o2 = O.block_attention(q[:, perm], kb[:, perm], vb[:, perm], kc, vc, ctx_len)
+    np.testing.assert_allclose(o2, o[:, perm], rtol=1e-12, atol=1e-13)
+
+
+def test_attention_context_permutation_and_tail_ignored():
+    q, kb, vb, kc, vc = _attn_inputs(1, 4, 4, 2, 8, 9, seed=6, scale=2.0)
+    o = O.block_attention(q, kb, vb, kc, vc, np.array([6]))
+    perm = np.random.default_rng(1).permutation(6)
+    kc2, vc2 = kc.copy(), vc.copy()
+    kc2[:, :, :6] = kc[:, :, perm]
+    vc2[:, :, :6] = vc[:, :, perm]
+    kc2[:, :, 6:] = 1e3        # rows past ctx_len must not matter
+    vc2[:, :, 6:] = np.nan
+    o2 = O.block_attention(q, kb, vb, kc2, vc2, np.array([6]))
+    np.testing.assert_allclose(o2, o, rtol=1e-12, atol=1e-13)
+
+
+def test_attention_gqa_grouping_and_own_layer_only():
+    B, S, Hq, Hkv, dh, L = 1, 3, 8, 2, 4, 5
+    q, kb, vb, kc, vc = _attn_inputs(B, S, Hq, Hkv, dh, L, seed=7)
+    o = O.block_attention(q, kb, vb, kc, vc, np.array([L]))
+    kc2, vb2 = kc.copy(), vb.copy()
+    kc2[:, 1] += 1.0
+    vb2[:, :, 1] -= 0.5
+    o2 = O.block_attention(q, kb, vb2, kc2, vc, np.array([L]))
+    np.testing.assert_array_equal(o2[:, :, :4], o[:, :, :4])   # heads 0..3 read KV head 0
+    assert np.all(np.abs(o2[:, :, 4:] - o[:, :, 4:]).max(axis=-1) > 1e-6)
+    # two layers: layer 0's output depends on layer 0's K/V only
+    layers = [_attn_inputs(B, S, Hq, Hkv, dh, L, seed=s) for s in (20, 30)]
+    ref = O.block_attention(*layers[0], np.array([L]))
+    pert = [a.copy() for a in layers[1]]
+    pert[3] *= -1
+    _ = O.block_attention(*pert, np.array([L]))
+    np.testing.assert_array_equal(O.block_attention(*layers[0], np.array([L])), ref)
+
+
+# ----------------------------------------------------------------------- adaLN
+def test_timestep_embedding_closed_form():
+    H = 64
+    t = 0.37
+    phi = O.timestep_embedding(t, H)
+    assert phi.shape == (2 * H,)
+    assert phi[0] == pytest.approx(math.sin(t))
+    assert phi[H] == pytest.approx(math.cos(t))
+    assert phi[H // 2] == pytest.approx(math.sin(t * 0.01))          # 10000^(-1/2)
+    assert phi[H + H // 4] == pytest.approx(math.cos(t * 0.1))       # 10000^(-1/4)
+    z = O.timestep_embedding(0.0, H)
+    np.testing.assert_array_equal(z[:H], 0.0)
+    np.testing.assert_array_equal(z[H:], 1.0)
+
+
+def test_adaln_closed_forms():
+    H = 256
+    x = rnd((5, H), 11, 3.0) + 2.0
+    E = np.zeros((2, H))
+    y = O.adaln_modulate(x, E, np.zeros(5))       # t = 0: shift 0, scale 1 -> 2 LN(x)
+    ln = y / 2
+    np.testing.assert_allclose(ln.mean(axis=1), 0, atol=1e-12)
+    var = x.var(axis=1)
+    np.testing.assert_allclose((ln ** 2).mean(axis=1), var / (var + O.LN_EPS), rtol=1e-12)
+    # affine invariance of LN: a*x + c gives the same output (up to eps)
+    y2 = O.adaln_modulate(4.0 * x - 7.0, E, np.zeros(5))
+    np.testing.assert_allclose(y2, y, atol=1e-6)
+    # constant row: LN = 0 so y = shift = E0 + sin(t w)
+    E = rnd((2, H), 12)
+    t = np.array([0.25])
+    yc = O.adaln_modulate(np.full((1, H), 1.5), E, t)
+    phi = O.timestep_embedding(0.25, H)
+    np.testing.assert_allclose(yc[0], E[0] + phi[:H], rtol=1e-12, atol=1e-12)
+    # shift and scale rows are not swapped: scale multiplies, shift adds
+    x1 = rnd((1, H), 13)
+    y1 = O.adaln_modulate(x1, E, np.array([0.0]))
+    n = (x1 - x1.mean()) / np.sqrt(x1.var() + O.LN_EPS)
+    np.testing.assert_allclose(y1, n * (2.0 + E[1]) + E[0], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------ confidence/argmax
+def test_confidence_matches_scipy_and_ties():
+    lg = rnd((7, 300), 14, 3.0)
+    conf, tok = O.confidence(lg)
+    p = scipy.special.softmax(lg, axis=-1)
+    np.testing.assert_allclose(conf, p.max(axis=-1), rtol=1e-13)
+    np.testing.assert_array_equal(tok, p.argmax(axis=-1))
+    lg2 = np.zeros((1, 10)); lg2[0, [3, 7]] = 2.0
+    c2, t2 = O.confidence(lg2)
+    assert t2[0] == 3
+    np.testing.assert_allclose(c2[0], math.e ** 2 / (2 * math.e ** 2 + 8))
+    c3, _ = O.confidence(np.zeros((1, 1024)))
+    assert c3[0] == pytest.approx(1 / 1024)
+
+
+def test_logits_orientation_and_scale():
+    V, H = 50, 16
+    w = rnd((V, H), 15)
+    y = np.zeros((1, H)); y[0, 5] = 1.0
+    np.testing.assert_allclose(O.logits(y, w, 2.5)[0], 2.5 * w[:, 5])
+    wb = tt_inputs.bf16_bits(w.astype(np.float32))
+    yr = rnd((3, H), 16)
+    conf, tok, gl, gp = O.vocab_confidence(yr, wb, 3.0, rows_per_block=2)
+    p = scipy.special.softmax(3.0 * yr @ O.from_bf16(wb).T, axis=-1)
+    np.testing.assert_allclose(conf, p.max(axis=-1), rtol=1e-12)
+    ps = np.sort(p, axis=-1)
+    np.testing.assert_allclose(gp, ps[:, -1] - ps[:, -2], rtol=1e-9, atol=1e-15)
+
+
+# --------------------------------------------------------------------- commit
+def _golden():
+    with open(os.path.join(GOLDEN, "commit_example.json")) as f:
+        return json.load(f)
+
+
+def test_commit_golden_example():
+    g = _golden()
+    tokens = np.array([[-1, -1]])
+    masked = np.array([[1, 1]], dtype=bool)
+    for st in g["steps"]:
+        np.testing.assert_array_equal(masked[0].astype(int), st["masked_before"])
+        lg = np.array(st["logits"])
+        conf, tok = O.confidence(lg)
+        for s in range(2):
+            if st["probs"][s] is not None:
+                np.testing.assert_allclose(scipy.special.softmax(lg[s]), st["probs"][s], atol=1e-6)
+                assert conf[s] == pytest.approx(st["conf"][s], abs=1e-6)
+                assert tok[s] == st["tok"][s]
+        conf = np.where(masked[0], conf, np.nan)
+        tokens, masked, committed, fb = O.commit(conf[None], tok[None], tokens, masked, g["gamma"])
+        np.testing.assert_array_equal(committed[0].astype(int), st["committed"])
+        assert bool(fb[0]) == st["fallback"]
+    np.testing.assert_array_equal(tokens[0], g["final_tokens"])
+    assert not masked.any()
+
+
+def test_commit_golden_variants():
+    g = _golden()
+    lg = np.array(g["steps"][0]["logits"])
+    conf, tok = O.confidence(lg)
+    v = g["variant_gamma_0_7"]
+    t, m, c, _ = O.commit(conf[None], tok[None], np.array([[-1, -1]]), np.ones((1, 2), bool), v["gamma"])
+    np.testing.assert_array_equal(t[0], v["final_tokens_step1"])
+    np.testing.assert_array_equal(c[0].astype(int), v["committed_step1"])
+    v = g["variant_fallback"]
+    _, _, c, fb = O.commit(np.array([v["conf"]]), np.array([[0, 0]]), np.array([[-1, -1]]),
+                           np.ones((1, 2), bool), v["gamma"])
+    assert fb[0] and c[0, v["chosen"]] and c.sum() == 1
+    v = g["variant_tie"]
+    conf, tok = O.confidence(np.array([v["logits"]]))
+    assert tok[0] == v["tok"] and conf[0] == pytest.approx(v["p_top"], abs=1e-6)
+    _, gp = O.top2_margin(np.array([v["logits"]]))
+    assert gp[0] == pytest.approx(v["top2_prob_gap"], abs=1e-15)
+
+
+def test_commit_invariants_random():
+    rng = np.random.default_rng(17)
+    for trial in range(200):
+        B, S = 3, 8
+        masked = rng.random((B, S)) < 0.6
+        tokens = np.where(masked, -1, rng.integers(0, 100, (B, S)))
+        conf = rng.random((B, S))
+        if trial % 3 == 0:
+            conf[:, :4] = conf[:, :1]                     # planted ties
+        tok = rng.integers(0, 100, (B, S))
+        gamma = rng.choice([0.5, 0.8, 0.95])
+        t2, m2, c, fb = O.commit(conf, tok, tokens, masked, gamma)
+        assert not np.any(c & ~masked)                      # only masked positions commit
+        np.testing.assert_array_equal(t2[~masked], tokens[~masked])   # committed never change
+        for b in range(B):
+            if masked[b].any():
+                assert c[b].sum() >= 1                      # progress every step
+                if (conf[b][masked[b]] >= gamma).any():
+                    np.testing.assert_array_equal(c[b], masked[b] & (conf[b] >= gamma))
+                else:
+                    cand = np.where(masked[b])[0]
+                    best = cand[np.argmax(conf[b][cand])]   # first max = lowest position
+                    assert c[b].sum() == 1 and c[b, best]
+        np.testing.assert_array_equal(m2, masked & ~c)
+
+
+# ------------------------------------------------------------ embed / update
+def test_embed_and_linear_update_orientation():
+    B, S, Hq, Hkv, dh = 1, 3, 2, 1, 4
+    H = Hq * dh
+    n_qkv = H + 2 * Hkv * dh
+    emb = tt_inputs.bf16_bits(rnd((10, H), 18).astype(np.float32))
+    e_mask = tt_inputs.bf16_bits(rnd((H,), 19).astype(np.float32))
+    tokens = np.array([[4, -1, 7]])
+    masked = np.array([[0, 1, 0]], dtype=bool)
+    e = O.embed_block(tokens, masked, emb, e_mask)
+    np.testing.assert_array_equal(e[0, 0], O.from_bf16(emb[4]))
+    np.testing.assert_array_equal(e[0, 1], O.from_bf16(e_mask))
+    # u_t rows pick coordinates: output column j of [q|k|v] = e[:, j % H]
+    u_t = np.zeros((n_qkv, H))
+    for j in range(n_qkv):
+        u_t[j, j % H] = 1.0
+    q, k, v = O.linear_update(e, u_t, Hq, Hkv, dh)
+    np.testing.assert_array_equal(q.reshape(B, S, H), e)
+    np.testing.assert_array_equal(k.reshape(B, S, -1), e[..., :Hkv * dh])
+    np.testing.assert_array_equal(v.reshape(B, S, -1), e[..., Hkv * dh:2 * Hkv * dh])
+
+
+# ----------------------------------------------------------------------- loop
+def _tiny_loop_inputs(seed=0, **kw):
+    d = tt_inputs.workload("tiny", **kw)
+    return d, tt_inputs.generate(d, seed)
+
+
+def test_loop_invariants_canonical_scale():
+    d, inp = _tiny_loop_inputs(B=2)
+    r = O.denoise_block_loop(inp, gamma=0.8)
+    assert not r["masked"].any()
+    prev_tok, prev_m = inp["tokens"], inp["masked"].astype(bool)
+    for st in r["trace"]:
+        # at V = 1024 and unit logit scale no confidence gets near 0.8, so the
+        # fallback commits exactly one position per sequence per step
+        assert np.nanmax(st["conf"]) < 0.5
+        np.testing.assert_array_equal(st["committed"].sum(axis=1), prev_m.any(axis=1).astype(int))
+        np.testing.assert_array_equal(st["tokens"][~prev_m], prev_tok[~prev_m])
+        prev_tok, prev_m = st["tokens"], st["masked"]
+    np.testing.assert_array_equal(r["steps_taken"], [16, 16])
+    # with nothing to tell masked positions apart (no positional signal) they
+    # tie, and the lowest position commits first
+    np.testing.assert_array_equal(r["commit_step"], np.tile(np.arange(16), (2, 1)))
+
+
+def test_loop_multi_commit_and_resume():
+    d, inp = _tiny_loop_inputs(B=2, precommit=("uniform", 0.0, 0.75))
+    r = O.denoise_block_loop(inp, gamma=0.5, logit_scale=40.0)
+    n0 = inp["masked"].sum(axis=1)
+    assert np.all(r["steps_taken"] <= n0)
+    assert np.all(r["steps_taken"] >= 1)
+    assert any(st["committed"].sum() > 2 for st in r["trace"])  # several commits in one step
+    pre = ~inp["masked"].astype(bool)
+    np.testing.assert_array_equal(r["tokens"][pre], inp["tokens"][pre])
+    np.testing.assert_array_equal(r["commit_step"][pre], -1)
+    # resume: stop after 1 step, restart from that state, same final tokens
+    r1 = O.denoise_block_loop(inp, gamma=0.5, logit_scale=40.0, max_steps=1)
+    inp2 = dict(inp, tokens=r1["tokens"], masked=r1["masked"].astype(np.uint8))
+    r2 = O.denoise_block_loop(inp2, gamma=0.5, logit_scale=40.0)
+    np.testing.assert_array_equal(r2["tokens"], r["tokens"])
