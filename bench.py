@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Benchmark of the block-wise diffusion denoise loop on B200.
+
+One step = one tt_denoise_block_loop call: a block of S masked positions per
+sequence is refined (re-embed + linear update -> block-denoise attention ->
+adaLN -> vocab GEMM with fused confidence -> commit) until every position is
+committed.  Default workload: 8 sequences, 32 query / 2 KV heads (GQA 16),
+d_head 128, hidden 4096, context 4096, S = 16, V = 131072, gamma 0.8, unit
+logit scale; synthetic seeded inputs resident in HBM.
+
+Metric: committed tokens/s (whole job), with denoise steps/s alongside.
+Timing: CUDA events on the library's stream around each call, an L2 flush
+(256 MiB write) between calls outside the events, max over ranks.
+`--impl reference` times the float64 CPU oracle on a bounded sample instead.
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
+torch.distributed.run (one rank per GPU, independent replicas, weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import tt_inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+KERNEL_SOURCES = {
+    "gemm_vocab": ["tt_gemm.cu", "tt_ptx.cuh", "tt_internal.h"],
+    "gemm_qkv": ["tt_gemm.cu", "tt_ptx.cuh", "tt_internal.h"],
+    "attn": ["tt_attn.cu", "tt_ptx.cuh", "tt_internal.h"],
+}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="mid", choices=sorted(tt_inputs.WORKLOADS))
+    p.add_argument("--gamma", type=float, default=0.8)
+    p.add_argument("--logit-scale", type=float, default=1.0)
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    return a
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each replica draws its own batch (independent sequences)."""
+    return seed + 1000 * rank
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max of a host float over all ranks (identity for one rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def workload_config(d, args, world):
+    return {
+        "workload": (f"{args.workload}-block-loop: B={d.B} S={d.S} Hq={d.Hq} Hkv={d.Hkv} "
+                     f"dh={d.dh} H={d.H} V={d.V} ctx={d.ctx} gamma={args.gamma} "
+                     f"logit_scale={args.logit_scale}"),
+        "global_batch": d.B * world,
+        "seq_len": d.L_cap,
+        "block_size": d.S,
+        "l2": "flushed between timed steps (256 MiB write, outside the events)",
+        "parallelism": "replicas" if world == 1 else f"dp{world} independent replicas",
+    }
+
+
+# ------------------------------------------------------------------ peaks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {k: float(pk[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(kind: str) -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES.get(kind, []):
+        with open(os.path.join(ROOT, "block_wise_diffusion_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kind: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if still current."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        e = t[kind]
+        if e.get("src_sha") == source_sha(kind) and e.get("workload") == workload:
+            return float(e["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.out = None
+        if gpu_id is None:
+            return
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def gpu_uuid(torch, idx):
+    try:
+        u = str(torch.cuda.get_device_properties(idx).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+# -------------------------------------------------------- CPU oracle arm
+def oracle_sample(d, inp, gamma, logit_scale):
+    """Run the oracle's block loop on one sequence of the workload."""
+    from oracle import twotower_oracle as O
+    one = dict(inp)
+    for k in ("k_ctx", "v_ctx", "ctx_len", "tokens", "masked"):
+        one[k] = inp[k][:1]
+    t0 = time.perf_counter()
+    r = O.denoise_block_loop(one, gamma, logit_scale)
+    dt = time.perf_counter() - t0
+    committed = int(inp["masked"][:1].sum())
+    steps = len(r["trace"])
+    return dt, committed, steps
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    d = tt_inputs.workload(args.workload)
+    inp = tt_inputs.generate(d, seed=rank_seed(args.seed, 0))
+    times, tokens, steps = [], 0, 0
+    for i in range(args.warmup + args.steps):
+        dt, c, s = oracle_sample(d, inp, args.gamma, args.logit_scale)
+        if i >= args.warmup:
+            times.append(dt)
+            tokens += c
+            steps += s
+    total = sum(times)
+    value = tokens / total
+    sample = (f"1 of {d.B} sequences of the workload per step, full block loop "
+              f"({steps // max(1, args.steps)} denoise steps), float64 NumPy oracle")
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": "committed tokens/s", "value": value,
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": workload_config(d, args, 1),
+        "denoise_steps_per_s": steps / total,
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ GPU arm
+def algorithmic(kind, d, inp, m_rows_total, launches):
+    """(bound, algorithmic bytes or flops per launch, unit) of a kernel kind."""
+    n_vt = -(-d.V // 256)
+    if kind == "gemm_vocab":
+        m_avg = m_rows_total / max(1, launches)
+        return "hbm", d.V * d.H * 2 + m_avg * (d.H * 2 + n_vt * 12), "GB/s"
+    if kind == "attn":
+        kv = 2 * d.Hkv * d.dh * 2 * float(np.sum(inp["ctx_len"]))
+        blk = d.B * d.S * (d.Hq + 2 * d.Hkv) * d.dh * 2 + d.B * d.S * d.H * 2
+        return "hbm", kv + blk, "GB/s"
+    if kind == "gemm_qkv":
+        n_qkv = d.H + 2 * d.Hkv * d.dh
+        return "tensor", 2.0 * d.B * d.S * d.H * n_qkv, "TFLOP/s"
+    return None, None, None
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import block_wise_diffusion_b200 as tt
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    tt.lib()
+    d = tt_inputs.workload(args.workload)
+    D = tt.dims(d)
+    t0 = time.time()
+    inp = tt_inputs.generate(d, seed=rank_seed(args.seed, rank))
+    log(f"[rank {rank}] inputs generated in {time.time() - t0:.1f}s")
+
+    def bf(k):
+        return torch.from_numpy(inp[k].view(np.int16)).to(dev).view(torch.bfloat16)
+
+    names = ["k_ctx", "v_ctx", "emb", "e_mask", "u_t", "shift_scale", "w"]
+    X = {k: bf(k) for k in names}
+    ctx_len = torch.from_numpy(inp["ctx_len"]).to(dev)
+    tokens0 = torch.from_numpy(inp["tokens"]).to(dev)
+    masked0 = torch.from_numpy(inp["masked"]).to(dev)
+    tokens, masked = tokens0.clone(), masked0.clone()
+    steps_taken = torch.empty(d.B, dtype=torch.int32, device=dev)
+    commit_step = torch.empty((d.B, d.S), dtype=torch.int32, device=dev)
+    ws = tt.workspace(D, tt.TT_WS_LOOP, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n_masked0 = int(inp["masked"].sum())
+
+    def call(kc=None, vc=None, cl=None, tk=None, mk=None):
+        return tt.tt_denoise_block_loop(
+            D, kc if kc is not None else X["k_ctx"], vc if vc is not None else X["v_ctx"],
+            cl if cl is not None else ctx_len, X["emb"], X["e_mask"], X["u_t"],
+            X["shift_scale"], X["w"], args.gamma, args.logit_scale, d.S,
+            tk if tk is not None else tokens, mk if mk is not None else masked,
+            steps_taken, commit_step, ws, stream)
+
+    def reset():
+        tokens.copy_(tokens0)
+        masked.copy_(masked0)
+        flush.zero_()
+
+    # warm-up
+    for _ in range(args.warmup):
+        reset()
+        call()
+    torch.cuda.synchronize(dev)
+
+    # timed region
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(gpu_uuid(torch, local))
+    launches0 = tt.tt_launch_count()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    denoise_steps = 0
+    for i in range(args.steps):
+        reset()
+        ev[i][0].record(stream)
+        denoise_steps += call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    gpu_launches = tt.tt_launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    ms_local = sum(a.elapsed_time(b) for a, b in ev)
+    assert not masked.any().item(), "block not committed"
+    ms = reduce_max(ms_local, world, dev)
+    tokens_all = reduce_sum(float(n_masked0 * args.steps), world, dev)
+    steps_all = reduce_sum(float(denoise_steps), world, dev)
+    value = tokens_all / (ms / 1e3)
+
+    # end to end through the public API with host buffers: H2D of the block's
+    # inputs (context K/V, lengths, tokens, mask) from pinned memory, the loop,
+    # D2H of the results; weights stay resident.
+    h_in = {"k_ctx": X["k_ctx"].cpu().pin_memory(), "v_ctx": X["v_ctx"].cpu().pin_memory(),
+            "ctx_len": ctx_len.cpu().pin_memory(), "tokens": tokens0.cpu().pin_memory(),
+            "masked": masked0.cpu().pin_memory()}
+    h_out = {"tokens": torch.empty_like(tokens0, device="cpu").pin_memory(),
+             "masked": torch.empty_like(masked0, device="cpu").pin_memory(),
+             "steps_taken": torch.empty_like(steps_taken, device="cpu").pin_memory(),
+             "commit_step": torch.empty_like(commit_step, device="cpu").pin_memory()}
+    d_in = {k: torch.empty_like(v, device=dev) for k, v in h_in.items()}
+    h2d = sum(v.numel() * v.element_size() for v in h_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in h_out.values())
+    e2e_ms = 0.0
+    if world > 1:
+        torch.distributed.barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for k in h_in:
+            d_in[k].copy_(h_in[k], non_blocking=True)
+        call(d_in["k_ctx"], d_in["v_ctx"], d_in["ctx_len"], d_in["tokens"], d_in["masked"])
+        h_out["tokens"].copy_(d_in["tokens"], non_blocking=True)
+        h_out["masked"].copy_(d_in["masked"], non_blocking=True)
+        h_out["steps_taken"].copy_(steps_taken, non_blocking=True)
+        h_out["commit_step"].copy_(commit_step, non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        e2e_ms += a.elapsed_time(b)
+    assert not h_out["masked"].any().item()
+    e2e_ms = reduce_max(e2e_ms, world, dev)
+    e2e_value = tokens_all / (e2e_ms / 1e3)
+
+    # per-kernel profile (one extra call, outside the timed region)
+    reset()
+    tt.tt_profile_enable(True)
+    call()
+    table = tt.profile_table()
+    tt.tt_profile_enable(False)
+    cs = commit_step.cpu().numpy()
+    m_rows_total = float((cs[inp["masked"].astype(bool)] + 1).sum())
+    peaks, peak_src = load_peaks()
+    kernels = {}
+    for kind, (kms, n) in sorted(table.items(), key=lambda kv: -kv[1][0]):
+        e = {"launches": n, "total_ms": round(kms, 4), "avg_us": round(1e3 * kms / n, 2)}
+        bound, per, unit = algorithmic(kind, d, inp, m_rows_total, n)
+        if bound is not None:
+            ach = per / (kms / n / 1e3) / (1e9 if unit == "GB/s" else 1e12)
+            pk = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops_sustained"]
+            e.update(bound=bound, achieved=round(ach, 2), unit=unit, frac=round(ach / pk, 4))
+        kernels[kind] = e
+    dom = max(table, key=lambda k: table[k][0])
+    bound, per, unit = algorithmic(dom, d, inp, m_rows_total, table[dom][1])
+    roofline = None
+    if bound is not None:
+        avg_s = table[dom][0] / table[dom][1] / 1e3
+        ach = per / avg_s / (1e9 if unit == "GB/s" else 1e12)
+        pk = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops_sustained"]
+        roofline = {"kernel": dom, "bound": bound, "achieved": round(ach, 2), "peak": pk,
+                    "unit": unit, "frac": round(ach / pk, 4),
+                    "traffic": committed_traffic(dom, args.workload),
+                    "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
+                    "algorithmic_per_launch": per}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, c, s = oracle_sample(d, inp, args.gamma, args.logit_scale)
+        cpu = {"value": c / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"1 of {d.B} sequences of the workload, full block loop ({s} denoise "
+                         f"steps, {dt:.1f} s), float64 NumPy oracle"}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": "committed tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(fan-in), bf16)",
+        "config": workload_config(d, args, world),
+        "denoise_steps_per_s": steps_all / (ms / 1e3),
+        "gpu_launches": gpu_launches,
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "roofline": roofline,
+        "kernels": kernels,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.gpus != world and world != 1:
+        log(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

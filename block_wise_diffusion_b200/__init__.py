@@ -1,0 +1,214 @@
+"""Python binding of libtwotower (argument marshalling only).
+
+Every function with a ``tt_`` name calls the C entry point of the same name
+in ``libtwotower.so`` (built in-tree by ``block_wise_diffusion_b200.build``)
+with raw device pointers taken from torch tensors.  Nothing here computes:
+torch provides device memory and streams; all arithmetic runs in the
+library's sm_100a kernels.  There is no CPU path: if the library or a CUDA
+device is missing, the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "TTError", "Dims", "lib", "lib_path", "dims", "workspace", "tt_workspace_bytes",
+    "tt_block_denoise_attn", "tt_adaln_modulate", "tt_vocab_confidence_commit",
+    "tt_denoise_block_loop", "tt_device_status", "tt_launch_count", "tt_set_attn_splits",
+    "tt_status_string", "tt_last_error", "EXPORTS", "tt_profile_enable", "tt_profile_read",
+    "profile_table", "KERNEL_KINDS",
+    "TT_WS_ATTN", "TT_WS_ADALN", "TT_WS_VOCAB", "TT_WS_LOOP",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libtwotower.so")
+
+TT_WS_ATTN, TT_WS_ADALN, TT_WS_VOCAB, TT_WS_LOOP = 0, 1, 2, 3
+STATUS = {0: "TT_OK", 1: "TT_ERR_INVALID_ARG", 2: "TT_ERR_UNSUPPORTED", 3: "TT_ERR_WORKSPACE",
+          4: "TT_ERR_CUDA", 5: "TT_ERR_TIMEOUT", 6: "TT_ERR_INTERNAL"}
+
+# Every symbol the header declares.
+EXPORTS = (
+    "tt_status_string", "tt_last_error", "tt_workspace_bytes", "tt_device_status",
+    "tt_launch_count", "tt_set_attn_splits", "tt_block_denoise_attn", "tt_adaln_modulate",
+    "tt_vocab_confidence_commit", "tt_denoise_block_loop", "tt_profile_enable", "tt_profile_read",
+)
+KERNEL_KINDS = ("plan", "embed", "gemm_qkv", "attn", "merge", "adaln", "gemm_vocab", "commit",
+                "gather", "init")
+
+
+class TTError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}: {detail}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "S", "Hq", "Hkv", "dh", "H", "V", "L_cap")]
+
+
+_P = ctypes.c_void_p
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtwotower.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise RuntimeError(
+                f"{lib_path} is missing: build it with `python -m block_wise_diffusion_b200.build`")
+        L = ctypes.CDLL(lib_path)
+        L.tt_status_string.restype = ctypes.c_char_p
+        L.tt_status_string.argtypes = [ctypes.c_int]
+        L.tt_last_error.restype = ctypes.c_char_p
+        L.tt_last_error.argtypes = []
+        L.tt_workspace_bytes.restype = ctypes.c_size_t
+        L.tt_workspace_bytes.argtypes = [ctypes.POINTER(Dims), ctypes.c_int]
+        L.tt_device_status.restype = ctypes.c_int
+        L.tt_device_status.argtypes = [_P, _P]
+        L.tt_launch_count.restype = ctypes.c_uint64
+        L.tt_launch_count.argtypes = []
+        L.tt_set_attn_splits.restype = ctypes.c_int
+        L.tt_set_attn_splits.argtypes = [ctypes.c_int32]
+        L.tt_profile_enable.restype = ctypes.c_int
+        L.tt_profile_enable.argtypes = [ctypes.c_int32]
+        L.tt_profile_read.restype = ctypes.c_int
+        L.tt_profile_read.argtypes = [ctypes.c_int32, ctypes.POINTER(ctypes.c_double),
+                                      ctypes.POINTER(ctypes.c_int64)]
+        L.tt_block_denoise_attn.restype = ctypes.c_int
+        L.tt_block_denoise_attn.argtypes = [ctypes.POINTER(Dims)] + [_P] * 7 + [_P, ctypes.c_size_t, _P]
+        L.tt_adaln_modulate.restype = ctypes.c_int
+        L.tt_adaln_modulate.argtypes = [ctypes.POINTER(Dims), _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+        L.tt_vocab_confidence_commit.restype = ctypes.c_int
+        L.tt_vocab_confidence_commit.argtypes = (
+            [ctypes.POINTER(Dims), _P, _P, ctypes.c_float, ctypes.c_float] + [_P] * 5
+            + [_P, ctypes.c_size_t, _P])
+        L.tt_denoise_block_loop.restype = ctypes.c_int
+        L.tt_denoise_block_loop.argtypes = (
+            [ctypes.POINTER(Dims)] + [_P] * 8 + [ctypes.c_float, ctypes.c_float, ctypes.c_int32]
+            + [_P] * 5 + [_P, ctypes.c_size_t, _P])
+        _lib = L
+    return _lib
+
+
+def dims(d) -> Dims:
+    """tt_dims from any object with B, S, Hq, Hkv, dh, V, L_cap (and H) fields."""
+    H = getattr(d, "H", d.Hq * d.dh)
+    return Dims(d.B, d.S, d.Hq, d.Hkv, d.dh, H, d.V, d.L_cap)
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_cuda:
+        raise ValueError("libtwotower takes CUDA tensors only (no CPU path)")
+    if not x.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise TTError(code, where, lib().tt_last_error().decode())
+
+
+def tt_status_string(code: int) -> str:
+    return lib().tt_status_string(code).decode()
+
+
+def tt_last_error() -> str:
+    return lib().tt_last_error().decode()
+
+
+def tt_launch_count() -> int:
+    return int(lib().tt_launch_count())
+
+
+def tt_set_attn_splits(n: int) -> None:
+    _check(lib().tt_set_attn_splits(n), "tt_set_attn_splits")
+
+
+def tt_profile_enable(on: bool) -> None:
+    _check(lib().tt_profile_enable(1 if on else 0), "tt_profile_enable")
+
+
+def tt_profile_read(kind: int) -> tuple[float, int]:
+    """(total ms, launches) of one kernel kind since profiling was enabled."""
+    ms, n = ctypes.c_double(0), ctypes.c_int64(0)
+    _check(lib().tt_profile_read(kind, ctypes.byref(ms), ctypes.byref(n)), "tt_profile_read")
+    return ms.value, n.value
+
+
+def profile_table() -> dict:
+    """{kernel kind name: (total ms, launches)} for every kind that ran."""
+    out = {}
+    for k, name in enumerate(KERNEL_KINDS):
+        ms, n = tt_profile_read(k)
+        if n:
+            out[name] = (ms, n)
+    return out
+
+
+def tt_workspace_bytes(d: Dims, which: int) -> int:
+    n = lib().tt_workspace_bytes(ctypes.byref(d), which)
+    if n == 0:
+        raise TTError(1, "tt_workspace_bytes", tt_last_error())
+    return int(n)
+
+
+def workspace(d: Dims, which: int, device="cuda"):
+    """A torch uint8 device buffer of tt_workspace_bytes(d, which) bytes."""
+    import torch
+    return torch.empty(tt_workspace_bytes(d, which), dtype=torch.uint8, device=device)
+
+
+def tt_device_status(ws, stream=None) -> int:
+    """Synchronise and return (and clear) the device error code in `ws`."""
+    return int(lib().tt_device_status(_ptr(ws), _stream(stream)))
+
+
+def tt_block_denoise_attn(d: Dims, q_blk, k_blk, v_blk, k_ctx, v_ctx, ctx_len, out, ws,
+                          stream=None) -> None:
+    _check(lib().tt_block_denoise_attn(
+        ctypes.byref(d), _ptr(q_blk), _ptr(k_blk), _ptr(v_blk), _ptr(k_ctx), _ptr(v_ctx),
+        _ptr(ctx_len), _ptr(out), _ptr(ws), ws.numel() if hasattr(ws, "numel") else 0,
+        _stream(stream)), "tt_block_denoise_attn")
+
+
+def tt_adaln_modulate(d: Dims, x, shift_scale, t, y, ws, stream=None) -> None:
+    _check(lib().tt_adaln_modulate(
+        ctypes.byref(d), _ptr(x), _ptr(shift_scale), _ptr(t), _ptr(y), _ptr(ws), ws.numel(),
+        _stream(stream)), "tt_adaln_modulate")
+
+
+def tt_vocab_confidence_commit(d: Dims, y, w, gamma: float, logit_scale: float, tokens, masked,
+                               conf_out, argmax_out, n_committed, ws, stream=None) -> None:
+    _check(lib().tt_vocab_confidence_commit(
+        ctypes.byref(d), _ptr(y), _ptr(w), float(gamma), float(logit_scale), _ptr(tokens),
+        _ptr(masked), _ptr(conf_out), _ptr(argmax_out), _ptr(n_committed), _ptr(ws), ws.numel(),
+        _stream(stream)), "tt_vocab_confidence_commit")
+
+
+def tt_denoise_block_loop(d: Dims, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale, w,
+                          gamma: float, logit_scale: float, max_steps: int, tokens, masked,
+                          steps_taken, commit_step, ws, stream=None) -> int:
+    """Runs the loop; returns the number of steps that did work."""
+    steps_run = ctypes.c_int32(0)
+    _check(lib().tt_denoise_block_loop(
+        ctypes.byref(d), _ptr(k_ctx), _ptr(v_ctx), _ptr(ctx_len), _ptr(emb), _ptr(e_mask),
+        _ptr(u_t), _ptr(shift_scale), _ptr(w), float(gamma), float(logit_scale), int(max_steps),
+        _ptr(tokens), _ptr(masked), _ptr(steps_taken), _ptr(commit_step),
+        ctypes.addressof(steps_run), _ptr(ws), ws.numel(), _stream(stream)),
+        "tt_denoise_block_loop")
+    return int(steps_run.value)

@@ -1,0 +1,613 @@
+// C ABI of libtwotower: argument validation, workspace carving, tensor-map
+// construction and kernel sequencing.  All compute happens in the kernels of
+// tt_attn.cu, tt_gemm.cu and tt_small.cu.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "tt_internal.h"
+
+namespace tt {
+
+static thread_local char g_err[512];
+static std::atomic<uint64_t> g_launches{0};
+static std::atomic<int> g_forced_splits{0};
+
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// ----------------------------------------------------------------- profiler
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+static std::mutex g_prof_mu;
+static std::atomic<bool> g_prof_on{false};
+static std::vector<ProfRec> g_prof_pending;
+static std::vector<cudaEvent_t> g_prof_free;
+static double g_prof_ms[TT_K_COUNT];
+static int64_t g_prof_n[TT_K_COUNT];
+static thread_local cudaEvent_t g_prof_open = nullptr;
+
+static cudaEvent_t prof_event() {
+  if (!g_prof_free.empty()) {
+    cudaEvent_t e = g_prof_free.back();
+    g_prof_free.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+void prof_begin(int kind, cudaStream_t st) {
+  (void)kind;
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_open = prof_event();
+  if (g_prof_open) cudaEventRecord(g_prof_open, st);
+}
+
+void prof_end(int kind, cudaStream_t st) {
+  if (!g_prof_on.load(std::memory_order_relaxed) || g_prof_open == nullptr) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  cudaEvent_t e = prof_event();
+  if (e == nullptr) return;
+  cudaEventRecord(e, st);
+  g_prof_pending.push_back({kind, g_prof_open, e});
+  g_prof_open = nullptr;
+}
+
+static void prof_harvest() {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (const ProfRec& r : g_prof_pending) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+      g_prof_ms[r.kind] += ms;
+      g_prof_n[r.kind] += 1;
+    }
+    g_prof_free.push_back(r.a);
+    g_prof_free.push_back(r.b);
+  }
+  g_prof_pending.clear();
+}
+
+static tt_status fail(tt_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+#define TT_LAUNCH(kind, st, call) \
+  do {                             \
+    prof_begin((kind), (st));      \
+    TT_CUDA(call);                 \
+    prof_end((kind), (st));        \
+  } while (0)
+
+#define TT_CUDA(call)                                                                      \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess)                                                                 \
+      return fail(TT_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_),     \
+                  __FILE__, __LINE__);                                                     \
+  } while (0)
+
+// --------------------------------------------------------------- tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                  uint32_t b2) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ----------------------------------------------------------------- checks
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static tt_status check_dims(const tt_dims* d) {
+  if (d == nullptr) return fail(TT_ERR_INVALID_ARG, "dims is NULL");
+  if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->V < 2 || d->L_cap < 0)
+    return fail(TT_ERR_INVALID_ARG, "bad sizes: B=%d Hq=%d Hkv=%d V=%d L_cap=%d", d->B, d->Hq,
+                d->Hkv, d->V, d->L_cap);
+  if (d->S != 16 && d->S != 32) return fail(TT_ERR_UNSUPPORTED, "S=%d not in {16,32}", d->S);
+  if (d->dh != 64 && d->dh != 128)
+    return fail(TT_ERR_UNSUPPORTED, "dh=%d not in {64,128}", d->dh);
+  if (d->Hq % d->Hkv != 0)
+    return fail(TT_ERR_INVALID_ARG, "Hq=%d not a multiple of Hkv=%d", d->Hq, d->Hkv);
+  const int G = d->Hq / d->Hkv;
+  if (G > 128 || (G & (G - 1)) != 0)
+    return fail(TT_ERR_UNSUPPORTED, "G=Hq/Hkv=%d must be a power of two <= 128", G);
+  if (d->H != d->Hq * d->dh)
+    return fail(TT_ERR_INVALID_ARG, "H=%d != Hq*dh=%d", d->H, d->Hq * d->dh);
+  if (d->H % 64 != 0 || d->H > 8192)
+    return fail(TT_ERR_UNSUPPORTED, "H=%d must be a multiple of 64 and <= 8192", d->H);
+  if ((long long)d->B * d->Hkv * d->L_cap >= (1ll << 31) || (long long)d->B * d->S >= (1 << 24) ||
+      (long long)d->V * d->H >= (1ll << 40))
+    return fail(TT_ERR_UNSUPPORTED, "problem too large");
+  return TT_OK;
+}
+
+static tt_status check_ptr(const void* p, const char* name, bool need16) {
+  if (p == nullptr) return fail(TT_ERR_INVALID_ARG, "%s is NULL", name);
+  if (need16 && !aligned16(p)) return fail(TT_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return TT_OK;
+}
+#define TT_CHECK(x)               \
+  do {                            \
+    tt_status s_ = (x);           \
+    if (s_ != TT_OK) return s_;   \
+  } while (0)
+
+// ------------------------------------------------------------ geometry
+struct AttnGeom {
+  int G, s_per_half, rows_per_half, halves, n_qtiles, n_splits, chunk;
+  size_t part_o_bytes, part_ml_bytes;
+};
+
+static AttnGeom attn_geom(const tt_dims& d) {
+  AttnGeom g;
+  g.G = d.Hq / d.Hkv;
+  g.s_per_half = std::min(d.S, 128 / g.G);
+  g.rows_per_half = g.s_per_half * g.G;
+  g.halves = std::min(2, d.S / g.s_per_half);
+  g.n_qtiles = d.S / (g.halves * g.s_per_half);
+  const long long units = (long long)d.B * d.Hkv * g.n_qtiles;
+  const int max_tiles = std::max(1, (d.L_cap + kAttnBN - 1) / kAttnBN);
+  const int forced = g_forced_splits.load();
+  int n = forced > 0 ? forced : (int)std::max<long long>(1, kNumSMs / units);
+  n = std::min(std::min(n, max_tiles), 64);
+  int per = (d.L_cap + n - 1) / n;
+  g.chunk = std::max(kAttnBN, (per + kAttnBN - 1) / kAttnBN * kAttnBN);
+  g.n_splits = n;
+  const size_t rows = (size_t)units * n * 256;
+  g.part_o_bytes = n > 1 ? rows * d.dh * sizeof(float) : 0;
+  g.part_ml_bytes = n > 1 ? rows * 2 * sizeof(float) : 0;
+  return g;
+}
+
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  template <class T>
+  T* take(size_t bytes) {
+    off = (off + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+struct Ws {
+  int* ctrl = nullptr;
+  int* rowlist = nullptr;
+  float* tvec = nullptr;
+  uint16_t* egath = nullptr;
+  uint16_t* qkv = nullptr;
+  uint16_t* attn_out = nullptr;
+  uint16_t* y_c = nullptr;
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  float* part_v = nullptr;
+  float* part_z = nullptr;
+  int* part_a = nullptr;
+  size_t total = 0;
+};
+
+static Ws carve(const tt_dims& d, int which, void* ws) {
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  Ws w;
+  const size_t rows = (size_t)d.B * d.S;
+  const size_t n_vt = (size_t)(d.V + kGemmBN - 1) / kGemmBN;
+  w.ctrl = c.take<int>(kCtrlBytes);
+  if (which == TT_WS_ATTN || which == TT_WS_LOOP) {
+    const AttnGeom g = attn_geom(d);
+    if (g.n_splits > 1) {
+      w.part_o = c.take<float>(g.part_o_bytes);
+      w.part_ml = c.take<float>(g.part_ml_bytes);
+    }
+  }
+  if (which == TT_WS_VOCAB || which == TT_WS_LOOP) {
+    w.rowlist = c.take<int>(rows * sizeof(int));
+    w.tvec = c.take<float>((size_t)d.B * sizeof(float));
+    w.y_c = c.take<uint16_t>(rows * d.H * 2);
+    w.part_v = c.take<float>(n_vt * rows * sizeof(float));
+    w.part_z = c.take<float>(n_vt * rows * sizeof(float));
+    w.part_a = c.take<int>(n_vt * rows * sizeof(int));
+  }
+  if (which == TT_WS_LOOP) {
+    const size_t n_qkv = (size_t)d.H + 2 * (size_t)d.Hkv * d.dh;
+    w.egath = c.take<uint16_t>(rows * d.H * 2);
+    w.qkv = c.take<uint16_t>(rows * n_qkv * 2);
+    w.attn_out = c.take<uint16_t>(rows * d.H * 2);
+  }
+  w.total = (c.off + 255) & ~size_t(255);
+  return w;
+}
+
+static tt_status check_ws(const tt_dims& d, int which, void* ws, size_t ws_bytes, Ws* out) {
+  TT_CHECK(check_ptr(ws, "ws", true));
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(TT_ERR_INVALID_ARG, "ws is not 256-byte aligned");
+  *out = carve(d, which, ws);
+  if (ws_bytes < out->total)
+    return fail(TT_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, out->total);
+  return TT_OK;
+}
+
+// ---------------------------------------------------------- stage helpers
+struct AttnMaps {
+  CUtensorMap q, kc, vc, kb, vb;
+};
+
+static tt_status build_attn_maps(const tt_dims& d, const AttnGeom& g, const tt_bf16* q, int ldq,
+                                 const tt_bf16* kb, const tt_bf16* vb, int ldkv,
+                                 const tt_bf16* kc, const tt_bf16* vc, AttnMaps* m) {
+  const uint64_t rows_ctx = (uint64_t)d.B * d.Hkv * std::max(d.L_cap, 1);
+  bool ok = make_tmap_3d(&m->q, q, d.dh, d.Hq, (uint64_t)d.B * d.S, (uint64_t)d.dh * 2,
+                         (uint64_t)ldq * 2, 64, g.G, g.s_per_half) &&
+            make_tmap_3d(&m->kb, kb, d.dh, d.Hkv, (uint64_t)d.B * d.S, (uint64_t)d.dh * 2,
+                         (uint64_t)ldkv * 2, 64, 1, d.S) &&
+            make_tmap_3d(&m->vb, vb, d.dh, d.Hkv, (uint64_t)d.B * d.S, (uint64_t)d.dh * 2,
+                         (uint64_t)ldkv * 2, 64, 1, d.S) &&
+            make_tmap_2d(&m->kc, kc, d.dh, rows_ctx, (uint64_t)d.dh * 2, 64, kAttnBN) &&
+            make_tmap_2d(&m->vc, vc, d.dh, rows_ctx, (uint64_t)d.dh * 2, 64, kAttnBN);
+  if (!ok) return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the attention operands");
+  return TT_OK;
+}
+
+static tt_status run_attn(const tt_dims& d, const AttnGeom& g, const AttnMaps& m,
+                          const int32_t* ctx_len, tt_bf16* out, const Ws& w, const int* active,
+                          cudaStream_t st) {
+  AttnArgs a;
+  a.B = d.B;
+  a.S = d.S;
+  a.Hq = d.Hq;
+  a.Hkv = d.Hkv;
+  a.dh = d.dh;
+  a.G = g.G;
+  a.L_cap = d.L_cap;
+  a.ctx_len = ctx_len;
+  a.active = active;
+  a.s_per_half = g.s_per_half;
+  a.rows_per_half = g.rows_per_half;
+  a.halves = g.halves;
+  a.n_qtiles = g.n_qtiles;
+  a.n_splits = g.n_splits;
+  a.chunk = g.chunk;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.dh));
+  a.out = out;
+  a.ldo = d.H;
+  a.part_o = w.part_o;
+  a.part_ml = w.part_ml;
+  a.err = w.ctrl;
+  TT_LAUNCH(TT_K_ATTN, st, launch_attn(m.q, m.kc, m.vc, m.kb, m.vb, a, st));
+  if (g.n_splits > 1) TT_LAUNCH(TT_K_MERGE, st, launch_attn_merge(a, st));
+  return TT_OK;
+}
+
+static tt_status run_vocab_gemm(const tt_dims& d, const Ws& w, const tt_bf16* W,
+                                float logit_scale, const int* M_dev, const int* active,
+                                cudaStream_t st) {
+  const int rows = d.B * d.S;
+  CUtensorMap tmA, tmB;
+  if (!make_tmap_2d(&tmA, w.y_c, d.H, rows, (uint64_t)d.H * 2, kGemmBK, kGemmBM) ||
+      !make_tmap_2d(&tmB, W, d.H, d.V, (uint64_t)d.H * 2, kGemmBK, kGemmBN))
+    return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the vocab GEMM");
+  GemmArgs a{};
+  a.M_alloc = rows;
+  a.M_dev = M_dev;
+  a.active = active;
+  a.N = d.V;
+  a.K = d.H;
+  a.part_v = w.part_v;
+  a.part_z = w.part_z;
+  a.part_a = w.part_a;
+  a.part_ld = rows;
+  a.scale_log2 = (float)(logit_scale * 1.4426950408889634);
+  a.err = w.ctrl;
+  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((d.V + kGemmBN - 1) / kGemmBN);
+  TT_LAUNCH(TT_K_GEMM_VOCAB, st, launch_gemm_vocab(tmA, tmB, a, std::min(tiles, kNumSMs), st));
+  return TT_OK;
+}
+
+static CommitArgs commit_args(const tt_dims& d, const Ws& w, float gamma, float logit_scale,
+                              int32_t* tokens, uint8_t* masked) {
+  CommitArgs c{};
+  c.B = d.B;
+  c.S = d.S;
+  c.n_vt = (d.V + kGemmBN - 1) / kGemmBN;
+  c.part_ld = d.B * d.S;
+  c.part_v = w.part_v;
+  c.part_z = w.part_z;
+  c.part_a = w.part_a;
+  c.scale_log2 = (float)(logit_scale * 1.4426950408889634);
+  c.gamma = gamma;
+  c.rowlist = w.rowlist;
+  c.M_dev = w.ctrl + CTRL_M;
+  c.tokens = tokens;
+  c.masked = masked;
+  c.ctrl = w.ctrl;
+  return c;
+}
+
+static tt_status read_ctrl(const Ws& w, cudaStream_t st, int* host) {
+  TT_CUDA(cudaMemcpyAsync(host, w.ctrl, 8 * sizeof(int), cudaMemcpyDeviceToHost, st));
+  TT_CUDA(cudaStreamSynchronize(st));
+  return TT_OK;
+}
+
+}  // namespace tt
+
+using namespace tt;
+
+extern "C" {
+
+const char* tt_status_string(tt_status s) {
+  switch (s) {
+    case TT_OK: return "TT_OK";
+    case TT_ERR_INVALID_ARG: return "TT_ERR_INVALID_ARG";
+    case TT_ERR_UNSUPPORTED: return "TT_ERR_UNSUPPORTED";
+    case TT_ERR_WORKSPACE: return "TT_ERR_WORKSPACE";
+    case TT_ERR_CUDA: return "TT_ERR_CUDA";
+    case TT_ERR_TIMEOUT: return "TT_ERR_TIMEOUT";
+    case TT_ERR_INTERNAL: return "TT_ERR_INTERNAL";
+  }
+  return "TT_ERR_UNKNOWN";
+}
+
+const char* tt_last_error(void) { return g_err; }
+
+uint64_t tt_launch_count(void) { return g_launches.load(); }
+
+tt_status tt_profile_enable(int32_t on) {
+  if (on) {
+    prof_harvest();
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (int k = 0; k < TT_K_COUNT; ++k) {
+      g_prof_ms[k] = 0.0;
+      g_prof_n[k] = 0;
+    }
+  }
+  g_prof_on.store(on != 0);
+  return TT_OK;
+}
+
+tt_status tt_profile_read(int32_t kind, double* total_ms, int64_t* launches) {
+  if (kind < 0 || kind >= TT_K_COUNT) return fail(TT_ERR_INVALID_ARG, "kind=%d", kind);
+  if (total_ms == nullptr || launches == nullptr)
+    return fail(TT_ERR_INVALID_ARG, "output pointer is NULL");
+  prof_harvest();
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  *total_ms = g_prof_ms[kind];
+  *launches = g_prof_n[kind];
+  return TT_OK;
+}
+
+tt_status tt_set_attn_splits(int32_t n_splits) {
+  if (n_splits < 0 || n_splits > 64)
+    return fail(TT_ERR_INVALID_ARG, "n_splits=%d not in [0, 64]", n_splits);
+  g_forced_splits.store(n_splits);
+  return TT_OK;
+}
+
+size_t tt_workspace_bytes(const tt_dims* d, int which) {
+  if (check_dims(d) != TT_OK) return 0;
+  if (which < TT_WS_ATTN || which > TT_WS_LOOP) {
+    fail(TT_ERR_INVALID_ARG, "unknown workspace kind %d", which);
+    return 0;
+  }
+  return carve(*d, which, nullptr).total;
+}
+
+tt_status tt_device_status(void* ws, void* stream) {
+  TT_CHECK(check_ptr(ws, "ws", true));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int h[2] = {0, 0};
+  TT_CUDA(cudaStreamSynchronize(st));
+  TT_CUDA(cudaMemcpy(h, ws, sizeof h, cudaMemcpyDeviceToHost));
+  if (h[0] != 0) {
+    TT_CUDA(cudaMemset(ws, 0, sizeof h));
+    return fail((tt_status)h[0], "device reported %s at tag 0x%x",
+                tt_status_string((tt_status)h[0]), h[1]);
+  }
+  return TT_OK;
+}
+
+tt_status tt_block_denoise_attn(const tt_dims* d, const tt_bf16* q_blk, const tt_bf16* k_blk,
+                                const tt_bf16* v_blk, const tt_bf16* k_ctx,
+                                const tt_bf16* v_ctx, const int32_t* ctx_len, tt_bf16* out,
+                                void* ws, size_t ws_bytes, void* stream) {
+  TT_CHECK(check_dims(d));
+  TT_CHECK(check_ptr(q_blk, "q_blk", true));
+  TT_CHECK(check_ptr(k_blk, "k_blk", true));
+  TT_CHECK(check_ptr(v_blk, "v_blk", true));
+  TT_CHECK(check_ptr(k_ctx, "k_ctx", true));
+  TT_CHECK(check_ptr(v_ctx, "v_ctx", true));
+  TT_CHECK(check_ptr(ctx_len, "ctx_len", false));
+  TT_CHECK(check_ptr(out, "out", true));
+  Ws w;
+  TT_CHECK(check_ws(*d, TT_WS_ATTN, ws, ws_bytes, &w));
+  const AttnGeom g = attn_geom(*d);
+  AttnMaps m;
+  TT_CHECK(build_attn_maps(*d, g, q_blk, d->Hq * d->dh, k_blk, v_blk, d->Hkv * d->dh, k_ctx,
+                           v_ctx, &m));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TT_CUDA(cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st));
+  return run_attn(*d, g, m, ctx_len, out, w, nullptr, st);
+}
+
+tt_status tt_adaln_modulate(const tt_dims* d, const tt_bf16* x, const tt_bf16* shift_scale,
+                            const float* t, tt_bf16* y, void* ws, size_t ws_bytes,
+                            void* stream) {
+  TT_CHECK(check_dims(d));
+  TT_CHECK(check_ptr(x, "x", true));
+  TT_CHECK(check_ptr(shift_scale, "shift_scale", true));
+  TT_CHECK(check_ptr(t, "t", false));
+  TT_CHECK(check_ptr(y, "y", true));
+  if (x == y) return fail(TT_ERR_INVALID_ARG, "y may not alias x");
+  Ws w;
+  TT_CHECK(check_ws(*d, TT_WS_ADALN, ws, ws_bytes, &w));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TT_CUDA(cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st));
+  TT_LAUNCH(TT_K_ADALN, st, launch_adaln(x, shift_scale, t, y, d->B * d->S, d->S, d->H, nullptr,
+                                         nullptr, nullptr, st));
+  return TT_OK;
+}
+
+tt_status tt_vocab_confidence_commit(const tt_dims* d, const tt_bf16* y, const tt_bf16* w,
+                                     float gamma, float logit_scale, int32_t* tokens,
+                                     uint8_t* masked, float* conf_out, int32_t* argmax_out,
+                                     int32_t* n_committed, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  TT_CHECK(check_dims(d));
+  TT_CHECK(check_ptr(y, "y", true));
+  TT_CHECK(check_ptr(w, "w", true));
+  TT_CHECK(check_ptr(tokens, "tokens", false));
+  TT_CHECK(check_ptr(masked, "masked", false));
+  if (!(gamma > 0.f && gamma <= 1.f))
+    return fail(TT_ERR_INVALID_ARG, "gamma=%g not in (0, 1]", (double)gamma);
+  if (!(logit_scale > 0.f) || !std::isfinite(logit_scale))
+    return fail(TT_ERR_INVALID_ARG, "logit_scale=%g must be finite and > 0", (double)logit_scale);
+  Ws ws_;
+  TT_CHECK(check_ws(*d, TT_WS_VOCAB, ws, ws_bytes, &ws_));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  TT_CUDA(cudaMemsetAsync(ws_.ctrl, 0, kCtrlBytes, st));
+  PlanArgs p{d->B, d->S, masked, ws_.rowlist, ws_.tvec, ws_.ctrl, 0};
+  TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
+  TT_LAUNCH(TT_K_GATHER, st, launch_gather_rows(y, d->H, ws_.y_c, d->H, ws_.rowlist, ws_.ctrl + CTRL_M,
+                             d->B * d->S, nullptr, st));
+  TT_CHECK(run_vocab_gemm(*d, ws_, w, logit_scale, ws_.ctrl + CTRL_M, nullptr, st));
+  CommitArgs c = commit_args(*d, ws_, gamma, logit_scale, tokens, masked);
+  c.conf_out = conf_out;
+  c.argmax_out = argmax_out;
+  c.n_committed = n_committed;
+  TT_LAUNCH(TT_K_COMMIT, st, launch_commit(c, st));
+  return TT_OK;
+}
+
+tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt_bf16* v_ctx,
+                                const int32_t* ctx_len, const tt_bf16* emb,
+                                const tt_bf16* e_mask, const tt_bf16* u_t,
+                                const tt_bf16* shift_scale, const tt_bf16* W, float gamma,
+                                float logit_scale, int32_t max_steps, int32_t* tokens,
+                                uint8_t* masked, int32_t* steps_taken, int32_t* commit_step,
+                                int32_t* steps_run, void* ws, size_t ws_bytes, void* stream) {
+  TT_CHECK(check_dims(d));
+  TT_CHECK(check_ptr(k_ctx, "k_ctx", true));
+  TT_CHECK(check_ptr(v_ctx, "v_ctx", true));
+  TT_CHECK(check_ptr(ctx_len, "ctx_len", false));
+  TT_CHECK(check_ptr(emb, "emb", true));
+  TT_CHECK(check_ptr(e_mask, "e_mask", true));
+  TT_CHECK(check_ptr(u_t, "u_t", true));
+  TT_CHECK(check_ptr(shift_scale, "shift_scale", true));
+  TT_CHECK(check_ptr(W, "w", true));
+  TT_CHECK(check_ptr(tokens, "tokens", false));
+  TT_CHECK(check_ptr(masked, "masked", false));
+  TT_CHECK(check_ptr(steps_taken, "steps_taken", false));
+  TT_CHECK(check_ptr(commit_step, "commit_step", false));
+  if (!(gamma > 0.f && gamma <= 1.f))
+    return fail(TT_ERR_INVALID_ARG, "gamma=%g not in (0, 1]", (double)gamma);
+  if (!(logit_scale > 0.f) || !std::isfinite(logit_scale))
+    return fail(TT_ERR_INVALID_ARG, "logit_scale=%g must be finite and > 0", (double)logit_scale);
+  if (max_steps < 1 || max_steps > 1024)
+    return fail(TT_ERR_INVALID_ARG, "max_steps=%d not in [1, 1024]", max_steps);
+  Ws w;
+  TT_CHECK(check_ws(*d, TT_WS_LOOP, ws, ws_bytes, &w));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int rows = d->B * d->S;
+  const int n_qkv = d->H + 2 * d->Hkv * d->dh;
+  const AttnGeom g = attn_geom(*d);
+
+  CUtensorMap tmE, tmU;
+  if (!make_tmap_2d(&tmE, w.egath, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM) ||
+      !make_tmap_2d(&tmU, u_t, d->H, n_qkv, (uint64_t)d->H * 2, kGemmBK, kGemmBN))
+    return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
+  AttnMaps m;
+  TT_CHECK(build_attn_maps(*d, g, w.qkv, n_qkv, w.qkv + d->H, w.qkv + d->H + d->Hkv * d->dh,
+                           n_qkv, k_ctx, v_ctx, &m));
+
+  TT_CUDA(cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st));
+  TT_LAUNCH(TT_K_INIT, st, launch_loop_init(d->B, d->S, steps_taken, commit_step, w.ctrl, st));
+  const int* active = w.ctrl + CTRL_ACTIVE;
+  GemmArgs ga{};
+  ga.M_alloc = rows;
+  ga.active = active;
+  ga.N = n_qkv;
+  ga.K = d->H;
+  ga.C = w.qkv;
+  ga.ldc = n_qkv;
+  ga.err = w.ctrl;
+  const int qkv_tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kGemmBN - 1) / kGemmBN);
+  PlanArgs p{d->B, d->S, masked, w.rowlist, w.tvec, w.ctrl, 1};
+  for (int step = 0; step < max_steps; ++step) {
+    TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
+    TT_LAUNCH(TT_K_EMBED, st, launch_embed(tokens, masked, emb, e_mask, w.egath, rows, d->H, d->V, active, w.ctrl,
+                         st));
+    TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(tmE, tmU, ga, std::min(qkv_tiles, kNumSMs), st));
+    TT_CHECK(run_attn(*d, g, m, ctx_len, w.attn_out, w, active, st));
+    TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, shift_scale, w.tvec, w.y_c, rows, d->S,
+                                           d->H, w.rowlist, w.ctrl + CTRL_M, active, st));
+    TT_CHECK(run_vocab_gemm(*d, w, W, logit_scale, w.ctrl + CTRL_M, active, st));
+    CommitArgs c = commit_args(*d, w, gamma, logit_scale, tokens, masked);
+    c.commit_step = commit_step;
+    c.steps_taken = steps_taken;
+    c.step = step;
+    c.active = active;
+    TT_LAUNCH(TT_K_COMMIT, st, launch_commit(c, st));
+  }
+  PlanArgs pf = p;
+  pf.count_step = 0;
+  TT_LAUNCH(TT_K_PLAN, st, launch_plan(pf, st));
+  int h[8];
+  TT_CHECK(read_ctrl(w, st, h));
+  if (g_prof_on.load()) prof_harvest();
+  if (steps_run != nullptr) *steps_run = h[CTRL_STEPS_RUN];
+  if (h[CTRL_ERR] != 0)
+    return fail((tt_status)h[CTRL_ERR], "device reported %s at tag 0x%x",
+                tt_status_string((tt_status)h[CTRL_ERR]), h[CTRL_ERR_WHERE]);
+  return TT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,160 @@
+// Internal definitions shared by the translation units of libtwotower.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/twotower.h"
+
+namespace tt {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
+constexpr int kNumSMs = 148;
+
+// Control block: the first 256 bytes of every workspace.
+enum CtrlWord {
+  CTRL_ERR = 0,        // first device error code (0 = none)
+  CTRL_ERR_WHERE = 1,  // where it was raised (kernel-specific tag)
+  CTRL_REMAINING = 2,  // masked positions left after the last commit
+  CTRL_M = 3,          // masked rows of the current step (vocab GEMM rows)
+  CTRL_ACTIVE = 4,     // 1 while the loop still has masked positions
+  CTRL_STEPS_RUN = 5,  // loop steps that did work
+  CTRL_WORDS = 64
+};
+constexpr size_t kCtrlBytes = CTRL_WORDS * sizeof(int);
+
+// Device-side error tags (CTRL_ERR_WHERE).
+enum WhereTag {
+  WHERE_GEMM_PRODUCER = 0x100,
+  WHERE_GEMM_MMA = 0x101,
+  WHERE_GEMM_EPI = 0x102,
+  WHERE_ATTN_PRODUCER = 0x200,
+  WHERE_ATTN_MMA = 0x201,
+  WHERE_ATTN_SOFTMAX = 0x202,
+  WHERE_COMMIT_NAN = 0x300,
+  WHERE_GATHER_TOKEN = 0x301,
+};
+
+// ------------------------------------------------------------------ GEMM
+// C = A[M, K] . B[N, K]^T with both operands K-major bf16.  BM=128, BN=256,
+// BK=64.  Two epilogues: vocabulary statistics (per row and 256-wide column
+// tile: max logit, sum of exp relative to it, argmax) or a plain bf16 store.
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
+constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
+constexpr size_t kGemmStageBytes = (kGemmBM + kGemmBN) * kGemmBK * 2;
+constexpr size_t kGemmSmemBytes = kGemmStages * kGemmStageBytes + 1024 + 256;
+
+struct GemmArgs {
+  int M_alloc;          // rows present in A's tensor map
+  const int* M_dev;     // device row count (nullptr: M_alloc); rows >= M are ignored
+  const int* active;    // optional device flag: kernel returns at once if *active == 0
+  int N, K;             // N: columns of C (any multiple of 8); K multiple of 64
+  // vocabulary-statistics epilogue
+  float* part_v;        // [n_tiles_n][part_ld] max raw logit of the tile
+  float* part_z;        // [n_tiles_n][part_ld] sum exp2(l*c - max*c)
+  int* part_a;          // [n_tiles_n][part_ld] argmax column (lowest on ties)
+  int part_ld;
+  float scale_log2;     // c = logit_scale * log2(e)
+  // bf16 epilogue
+  uint16_t* C;
+  int ldc;
+  int* err;             // control block
+};
+
+cudaError_t launch_gemm_vocab(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
+                              int grid, cudaStream_t st);
+cudaError_t launch_gemm_bf16(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
+                             int grid, cudaStream_t st);
+
+// ------------------------------------------------------------- attention
+constexpr int kAttnBN = 64;        // keys per tile
+constexpr int kAttnStages = 4;
+constexpr int kAttnThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (2 x 128 rows)
+
+struct AttnArgs {
+  int B, S, Hq, Hkv, dh, G, L_cap;
+  const int* ctx_len;
+  const int* active;    // optional device flag
+  int s_per_half;       // block positions per 128-row half
+  int rows_per_half;    // s_per_half * G
+  int halves;           // halves per CTA (1 or 2)
+  int n_qtiles;         // CTAs along the query axis per (b, g)
+  int n_splits;         // key splits
+  int chunk;            // context keys per split (multiple of kAttnBN)
+  float scale_log2;     // log2(e) / sqrt(dh)
+  uint16_t* out;        // bf16 [B*S, ldo]
+  int ldo;
+  float* part_o;        // [units][256][dh] unnormalised partial outputs
+  float* part_ml;       // [units][256][2] (running max in log2 units, sum)
+  int* err;
+};
+size_t attn_smem_bytes(int dh, int halves);
+cudaError_t launch_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKc, const CUtensorMap& tmVc,
+                        const CUtensorMap& tmKb, const CUtensorMap& tmVb, const AttnArgs& a,
+                        cudaStream_t st);
+cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t st);
+
+// ------------------------------------------------------ small kernels
+struct PlanArgs {
+  int B, S;
+  const uint8_t* masked;
+  int* rowlist;     // [B*S] compact list of masked rows (b*S+s)
+  float* t;         // [B]   masked fraction at the start of the step
+  int* ctrl;        // writes CTRL_M, CTRL_REMAINING, CTRL_ACTIVE, CTRL_STEPS_RUN
+  int count_step;   // 1: bump CTRL_STEPS_RUN when active
+};
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st);
+
+cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
+                         uint16_t* y, int rows, int S, int H, const int* rowlist,
+                         const int* M_dev, const int* active, cudaStream_t st);
+
+cudaError_t launch_gather_rows(const uint16_t* src, int ld_src, uint16_t* dst, int H,
+                               const int* rowlist, const int* M_dev, int max_rows,
+                               const int* active, cudaStream_t st);
+
+cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_t* emb,
+                         const uint16_t* e_mask, uint16_t* dst, int rows, int H, int V,
+                         const int* active, int* err, cudaStream_t st);
+
+struct CommitArgs {
+  int B, S, n_vt, part_ld;
+  const float* part_v;
+  const float* part_z;
+  const int* part_a;
+  float scale_log2;
+  float gamma;
+  const int* rowlist;   // compact row -> b*S+s
+  const int* M_dev;
+  int* tokens;
+  uint8_t* masked;
+  float* conf_out;      // optional [B*S]
+  int* argmax_out;      // optional [B*S]
+  int* n_committed;     // optional [B]
+  int* commit_step;     // optional [B*S]
+  int* steps_taken;     // optional [B]
+  int step;
+  const int* active;
+  int* ctrl;
+};
+cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
+
+cudaError_t launch_loop_init(int B, int S, int* steps_taken, int* commit_step, int* ctrl,
+                             cudaStream_t st);
+
+// ---------------------------------------------------------------- host
+// Tensor-map construction (driver entry point fetched at run time, so the
+// library loads without a GPU driver present).
+bool make_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                  uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0, uint32_t b1,
+                  uint32_t b2);
+
+void count_launch(int n = 1);
+
+// Profiler hooks (no-ops unless tt_profile_enable(1)): bracket one launch.
+void prof_begin(int kind, cudaStream_t st);
+void prof_end(int kind, cudaStream_t st);
+
+}  // namespace tt

@@ -1,0 +1,363 @@
+// The light kernels of the denoise step: step planning (masked-row list and
+// timesteps), adaLN-single modulation, row gathers, block re-embedding and
+// the confidence commit.  All are bandwidth- or latency-bound and tiny next
+// to the attention and the vocabulary GEMM.
+#include <math.h>
+
+#include "tt_ptx.cuh"
+
+namespace tt {
+
+namespace {
+
+// ------------------------------------------------------------------ plan
+// Compact list of masked rows (b*S + s) in row order, the per-sequence
+// timestep t_b = masked count / S, and the step's control words.
+__global__ void __launch_bounds__(1024) plan_kernel(const PlanArgs a) {
+  __shared__ int warp_tot[32];
+  __shared__ int running;
+  const int n = a.B * a.S;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) running = 0;
+  __syncthreads();
+  for (int base = 0; base < n; base += 1024) {
+    const int i = base + tid;
+    const int f = (i < n && a.masked[i] != 0) ? 1 : 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    const int before_in_warp = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[warp] = __popc(bal);
+    __syncthreads();
+    int before_warps = 0, total = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = warp_tot[w];
+      before_warps += (w < warp) ? c : 0;
+      total += c;
+    }
+    if (f) a.rowlist[running + before_warps + before_in_warp] = i;
+    __syncthreads();
+    if (tid == 0) running += total;
+    __syncthreads();
+  }
+  for (int b = tid; b < a.B; b += 1024) {
+    int c = 0;
+    for (int s = 0; s < a.S; ++s) c += a.masked[b * a.S + s] != 0;
+    a.t[b] = (float)c / (float)a.S;
+  }
+  if (tid == 0) {
+    const int M = running;
+    a.ctrl[CTRL_M] = M;
+    a.ctrl[CTRL_REMAINING] = M;
+    a.ctrl[CTRL_ACTIVE] = M > 0 ? 1 : 0;
+    if (a.count_step && M > 0) a.ctrl[CTRL_STEPS_RUN] += 1;
+  }
+}
+
+// ----------------------------------------------------------------- adaLN
+// One CTA per output row.  y = LN(x) * (1 + E1 + cos(t w)) + E0 + sin(t w),
+// w_i = 10000^(-i/H): the adaLN-single reading of this library.
+constexpr int kAdaThreads = 256;
+constexpr int kAdaMaxVec = 4;  // H <= 256 threads * 4 vectors * 8 = 8192
+
+__device__ __forceinline__ float block_sum(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = 0.f;
+  for (int w = 0; w < kAdaThreads / 32; ++w) s += red[w];
+  return s;
+}
+
+__global__ void __launch_bounds__(kAdaThreads)
+    adaln_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ ss,
+                 const float* __restrict__ t, uint16_t* __restrict__ y, int rows, int S, int H,
+                 const int* __restrict__ rowlist, const int* M_dev, const int* active) {
+  __shared__ float red[kAdaThreads / 32];
+  if (active != nullptr && *active == 0) return;
+  const int M = M_dev != nullptr ? *M_dev : rows;
+  const int j = blockIdx.x;
+  if (j >= M) return;
+  const int src = rowlist != nullptr ? rowlist[j] : j;
+  const float tb = t[src / S];
+  const int nvec = H / 8;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)src * H);
+  float v[kAdaMaxVec][8];
+  float s = 0.f;
+#pragma unroll
+  for (int k = 0; k < kAdaMaxVec; ++k) {
+    const int vi = threadIdx.x + k * kAdaThreads;
+    if (vi < nvec) {
+      const uint4 u = xr[vi];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[k][2 * e] = __uint_as_float(w[e] << 16);
+        v[k][2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s += v[k][e];
+    }
+  }
+  const float mean = block_sum(s, red) / (float)H;
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < kAdaMaxVec; ++k) {
+    const int vi = threadIdx.x + k * kAdaThreads;
+    if (vi < nvec) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = v[k][e] - mean;
+        q += d * d;
+      }
+    }
+  }
+  const float var = block_sum(q, red) / (float)H;
+  const float rstd = rsqrtf(var + 1e-6f);
+  const float lw = -13.287712379549449f / (float)H;  // -log2(10000) / H
+  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)j * H);
+  const uint4* e0 = reinterpret_cast<const uint4*>(ss);
+  const uint4* e1 = reinterpret_cast<const uint4*>(ss + H);
+#pragma unroll
+  for (int k = 0; k < kAdaMaxVec; ++k) {
+    const int vi = threadIdx.x + k * kAdaThreads;
+    if (vi < nvec) {
+      const uint4 a0 = e0[vi], a1 = e1[vi];
+      const uint32_t sh[4] = {a0.x, a0.y, a0.z, a0.w};
+      const uint32_t sc[4] = {a1.x, a1.y, a1.z, a1.w};
+      float out[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int i = vi * 8 + e;
+        const float w = exp2f((float)i * lw);
+        float sn, cs;
+        sincosf(tb * w, &sn, &cs);
+        const uint32_t hs = (e & 1) ? (sh[e >> 1] & 0xffff0000u) : (sh[e >> 1] << 16);
+        const uint32_t hc = (e & 1) ? (sc[e >> 1] & 0xffff0000u) : (sc[e >> 1] << 16);
+        const float shift = __uint_as_float(hs) + sn;
+        const float scale = __uint_as_float(hc) + cs;
+        out[e] = (v[k][e] - mean) * rstd * (1.f + scale) + shift;
+      }
+      uint4 o;
+      o.x = pack_bf16x2(out[0], out[1]);
+      o.y = pack_bf16x2(out[2], out[3]);
+      o.z = pack_bf16x2(out[4], out[5]);
+      o.w = pack_bf16x2(out[6], out[7]);
+      yr[vi] = o;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- gathers
+__global__ void __launch_bounds__(256)
+    gather_rows_kernel(const uint16_t* __restrict__ src, int ld_src, uint16_t* __restrict__ dst,
+                       int H, const int* __restrict__ rowlist, const int* M_dev, int max_rows,
+                       const int* active) {
+  if (active != nullptr && *active == 0) return;
+  const int M = M_dev != nullptr ? min(*M_dev, max_rows) : max_rows;
+  const int j = blockIdx.x;
+  if (j >= M) return;
+  const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)rowlist[j] * ld_src);
+  uint4* d = reinterpret_cast<uint4*>(dst + (size_t)j * H);
+  for (int i = threadIdx.x; i < H / 8; i += blockDim.x) d[i] = s[i];
+}
+
+// e[row] = masked ? e_mask : Emb[token]; an out-of-range token of a committed
+// position is reported (TT_ERR_INTERNAL) and embedded as e_mask.
+__global__ void __launch_bounds__(256)
+    embed_kernel(const int* __restrict__ tokens, const uint8_t* __restrict__ masked,
+                 const uint16_t* __restrict__ emb, const uint16_t* __restrict__ e_mask,
+                 uint16_t* __restrict__ dst, int rows, int H, int V, const int* active,
+                 int* err) {
+  if (active != nullptr && *active == 0) return;
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  const uint16_t* src = e_mask;
+  if (masked[row] == 0) {
+    const int tok = tokens[row];
+    if (tok >= 0 && tok < V) {
+      src = emb + (size_t)tok * H;
+    } else if (threadIdx.x == 0) {
+      atomicCAS(err, 0, (int)TT_ERR_INTERNAL);
+      atomicCAS(err + 1, 0, (int)WHERE_GATHER_TOKEN);
+    }
+  }
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+  uint4* d = reinterpret_cast<uint4*>(dst + (size_t)row * H);
+  for (int i = threadIdx.x; i < H / 8; i += blockDim.x) d[i] = s[i];
+}
+
+// ---------------------------------------------------------------- commit
+// One CTA per sequence, one warp per block position.  A masked position's
+// 256-column tile statistics are merged into its confidence
+//   conf = 1 / sum_t z_t 2^(c*(v_t - v*)),  token = argmax column of the
+// tile with the largest v_t (lowest tile on ties, hence lowest id);
+// then warp 0 applies the commit rule across the block.
+__global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
+  __shared__ float s_conf[32];
+  __shared__ int s_tok[32];
+  __shared__ int s_mask[32];
+  if (a.active != nullptr && *a.active == 0) return;
+  const int b = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.S;
+  const int M = a.M_dev != nullptr ? *a.M_dev : a.B * S;
+  if (warp < S) {
+    const int row = b * S + warp;
+    const int is_m = a.masked[row] != 0;
+    float conf = -1.f;
+    int tok = -1;
+    if (is_m) {
+      // compact index of this row: rowlist is sorted, so search it
+      int lo = 0, hi = M - 1, j = -1;
+      while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int v = a.rowlist[mid];
+        if (v == row) {
+          j = mid;
+          break;
+        }
+        if (v < row) lo = mid + 1; else hi = mid - 1;
+      }
+      if (j >= 0) {
+        float bv = -INFINITY;
+        int bt = 0x7fffffff;
+        for (int t = lane; t < a.n_vt; t += 32) {
+          const float v = a.part_v[(size_t)t * a.part_ld + j];
+          if (v > bv || (v == bv && t < bt)) {
+            bv = v;
+            bt = t;
+          }
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+          const int ot = __shfl_xor_sync(0xffffffffu, bt, o);
+          if (ov > bv || (ov == bv && ot < bt)) {
+            bv = ov;
+            bt = ot;
+          }
+        }
+        const float mstar = bv * a.scale_log2;
+        float Z = 0.f;
+        for (int t = lane; t < a.n_vt; t += 32) {
+          const size_t o = (size_t)t * a.part_ld + j;
+          Z += a.part_z[o] * ex2(a.part_v[o] * a.scale_log2 - mstar);
+        }
+        for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+        conf = 1.f / Z;
+        tok = (bt < a.n_vt) ? a.part_a[(size_t)bt * a.part_ld + j] : -1;
+      }
+    }
+    if (lane == 0) {
+      s_conf[warp] = conf;
+      s_tok[warp] = tok;
+      s_mask[warp] = is_m;
+    }
+  }
+  __syncthreads();
+  if (warp != 0) return;
+  const int s = lane;
+  const bool in = s < S;
+  const int row = b * S + s;
+  const int is_m = in ? s_mask[s] : 0;
+  float cf = in ? s_conf[s] : -1.f;
+  const int tok = in ? s_tok[s] : -1;
+  const bool bad = is_m && !(cf >= 0.f && cf <= 1.0001f);  // NaN or impossible value
+  if (__any_sync(0xffffffffu, bad) && lane == 0) {
+    atomicCAS(a.ctrl + CTRL_ERR, 0, (int)TT_ERR_INTERNAL);
+    atomicCAS(a.ctrl + CTRL_ERR_WHERE, 0, (int)WHERE_COMMIT_NAN);
+  }
+  if (bad) cf = -1.f;
+  const bool qual = is_m && cf >= a.gamma && tok >= 0;
+  const unsigned qmask = __ballot_sync(0xffffffffu, qual);
+  const unsigned mmask = __ballot_sync(0xffffffffu, is_m != 0);
+  bool commit = qual;
+  if (qmask == 0 && mmask != 0) {
+    // fallback: the most confident masked position, lowest s on ties
+    float bc = is_m ? cf : -INFINITY;
+    int bs = is_m ? s : 0x7fffffff;
+    for (int o = 16; o > 0; o >>= 1) {
+      const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
+      const int os = __shfl_xor_sync(0xffffffffu, bs, o);
+      if (oc > bc || (oc == bc && os < bs)) {
+        bc = oc;
+        bs = os;
+      }
+    }
+    commit = is_m && s == bs;
+  }
+  if (in) {
+    if (commit) {
+      a.tokens[row] = tok >= 0 ? tok : 0;
+      a.masked[row] = 0;
+      if (a.commit_step != nullptr) a.commit_step[row] = a.step;
+    }
+    if (a.conf_out != nullptr) a.conf_out[row] = is_m ? s_conf[s] : -1.f;
+    if (a.argmax_out != nullptr) a.argmax_out[row] = is_m ? tok : -1;
+  }
+  const unsigned cmask = __ballot_sync(0xffffffffu, commit);
+  if (lane == 0) {
+    if (a.n_committed != nullptr) a.n_committed[b] = __popc(cmask);
+    if (a.steps_taken != nullptr && mmask != 0) a.steps_taken[b] = a.step + 1;
+  }
+}
+
+__global__ void loop_init_kernel(int B, int S, int* steps_taken, int* commit_step) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < B) steps_taken[i] = 0;
+  if (i < B * S) commit_step[i] = -1;
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st) {
+  plan_kernel<<<1, 1024, 0, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
+                         uint16_t* y, int rows, int S, int H, const int* rowlist,
+                         const int* M_dev, const int* active, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  adaln_kernel<<<rows, kAdaThreads, 0, st>>>(x, shift_scale, t, y, rows, S, H, rowlist, M_dev,
+                                             active);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const uint16_t* src, int ld_src, uint16_t* dst, int H,
+                               const int* rowlist, const int* M_dev, int max_rows,
+                               const int* active, cudaStream_t st) {
+  if (max_rows <= 0) return cudaSuccess;
+  gather_rows_kernel<<<max_rows, 256, 0, st>>>(src, ld_src, dst, H, rowlist, M_dev, max_rows,
+                                               active);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_t* emb,
+                         const uint16_t* e_mask, uint16_t* dst, int rows, int H, int V,
+                         const int* active, int* err, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  embed_kernel<<<rows, 256, 0, st>>>(tokens, masked, emb, e_mask, dst, rows, H, V, active, err);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
+  commit_kernel<<<a.B, a.S * 32, 0, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_loop_init(int B, int S, int* steps_taken, int* commit_step, int* ctrl,
+                             cudaStream_t st) {
+  (void)ctrl;
+  const int n = B * S;
+  loop_init_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, S, steps_taken, commit_step);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace tt

@@ -1,0 +1,227 @@
+/*
+ * libtwotower - block-wise diffusion denoise step on one B200 (sm_100a).
+ *
+ * The operations follow "Nemotron-TwoTower: Diffusion Language Modeling with
+ * Pretrained Autoregressive Context" (gist.science technical summary, sections
+ * Architecture, Generation Process, Training and Conditioning) and the
+ * snilld.dk TwoTower article (sections "Hvad TwoTower aendrer teknisk",
+ * "Blockwise generering i praksis").  The pages fix the method qualitatively;
+ * the numeric readings this library takes are stated beside each call.
+ *
+ * Conventions for every call
+ *  - All tensor pointers are DEVICE pointers, allocated and owned by the
+ *    caller.  The library never allocates device or pinned memory; scratch
+ *    space comes from a caller-provided workspace sized by tt_workspace_bytes.
+ *  - bf16 tensors are passed as tt_bf16 (the 16-bit pattern) and are dense,
+ *    row-major, with the layouts given below.  Base pointers of bf16 tensors
+ *    and workspaces must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream unless stated otherwise.
+ *  - Argument errors are detected on the host before any launch; the call
+ *    then returns an error code, launches nothing and modifies nothing.
+ *    tt_last_error() gives a thread-local description of the last failure.
+ *  - Errors a kernel detects (a bounded wait that timed out, an out-of-range
+ *    token id, a non-finite confidence) are recorded in the first 4 bytes of
+ *    the workspace and reported by tt_device_status() or, for the loop, by
+ *    the loop's own return code.
+ *  - Inputs are never modified, except `tokens` and `masked`, which are
+ *    in/out state of the commit step and of the loop.
+ *
+ * Supported shapes: dh in {64, 128}; S in {16, 32}; H == Hq*dh with H a
+ * multiple of 64, at most 8192; G = Hq/Hkv a power of two, at most 128; V >= 2;
+ * B >= 1; 0 <= ctx_len[b] <= L_cap.  Other shapes return TT_ERR_UNSUPPORTED.
+ */
+#ifndef TWOTOWER_H
+#define TWOTOWER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TT_API __attribute__((visibility("default")))
+#else
+#define TT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t tt_bf16; /* bit pattern of one bfloat16 value */
+
+typedef enum {
+  TT_OK = 0,
+  TT_ERR_INVALID_ARG = 1, /* null pointer, bad size, misaligned pointer, gamma out of (0,1] */
+  TT_ERR_UNSUPPORTED = 2, /* shape outside the supported set above */
+  TT_ERR_WORKSPACE = 3,   /* workspace smaller than tt_workspace_bytes() */
+  TT_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (text in tt_last_error) */
+  TT_ERR_TIMEOUT = 5,     /* a kernel's bounded wait gave up (recorded on the device) */
+  TT_ERR_INTERNAL = 6     /* device-detected inconsistency (bad token id, NaN confidence) */
+} tt_status;
+
+/* Problem sizes.  B sequences, block size S, Hq query heads, Hkv KV heads,
+ * head size dh, hidden size H (= Hq*dh), vocabulary V, context capacity
+ * L_cap (rows allocated per sequence and KV head in the context cache). */
+typedef struct {
+  int32_t B, S, Hq, Hkv, dh, H, V, L_cap;
+} tt_dims;
+
+/* Which call a workspace is sized for. */
+enum { TT_WS_ATTN = 0, TT_WS_ADALN = 1, TT_WS_VOCAB = 2, TT_WS_LOOP = 3 };
+
+/* Human-readable name of a status code (static string). */
+TT_API const char* tt_status_string(tt_status s);
+
+/* Description of the last error raised on the calling thread ("" if none). */
+TT_API const char* tt_last_error(void);
+
+/* Bytes of workspace the call `which` needs for dims `d`; 0 if `d` is invalid
+ * (tt_last_error says why). */
+TT_API size_t tt_workspace_bytes(const tt_dims* d, int which);
+
+/* Synchronises `stream`, then reads and clears the device error word at the
+ * start of workspace `ws`.  Returns TT_OK, TT_ERR_TIMEOUT, TT_ERR_INTERNAL or
+ * TT_ERR_CUDA. */
+TT_API tt_status tt_device_status(void* ws, void* stream);
+
+/* Number of kernels this library has launched in this process so far. */
+TT_API uint64_t tt_launch_count(void);
+
+/* Number of key splits the attention uses (0 = choose automatically, the
+ * default; otherwise at most 64).  Process-wide; results are independent of
+ * it up to float rounding. */
+TT_API tt_status tt_set_attn_splits(int32_t n_splits);
+
+/* Kernel kinds of the per-kernel profiler. */
+enum {
+  TT_K_PLAN = 0, TT_K_EMBED = 1, TT_K_GEMM_QKV = 2, TT_K_ATTN = 3, TT_K_MERGE = 4,
+  TT_K_ADALN = 5, TT_K_GEMM_VOCAB = 6, TT_K_COMMIT = 7, TT_K_GATHER = 8, TT_K_INIT = 9,
+  TT_K_COUNT = 10
+};
+
+/* Per-kernel profiler: while enabled, every kernel this library launches is
+ * bracketed by two CUDA events recorded on the caller's stream.  on = 1
+ * clears the table and starts recording, on = 0 stops.  Off by default; it
+ * adds two event records per launch and nothing else. */
+TT_API tt_status tt_profile_enable(int32_t on);
+
+/* Total device time (ms) and launch count of kernel kind `kind` since the
+ * last tt_profile_enable(1).  Waits for the recorded events to complete. */
+TT_API tt_status tt_profile_read(int32_t kind, double* total_ms, int64_t* launches);
+
+/*
+ * a1 - block-denoise attention of one denoiser layer.
+ * Source: gist.science summary, "Architecture" (bidirectional block attention
+ * plus attention to the corresponding layer of the frozen context tower) and
+ * "Generation Process" (each layer attends to the context KV cache of past
+ * blocks and to the block's own bidirectional KV).
+ *
+ * For every sequence b, query head h (KV head g = h / (Hq/Hkv)) and block
+ * position s:
+ *   out[b,s,h,:] = softmax_j( q_blk[b,s,h,:] . key_j / sqrt(dh) ) value_j
+ * over the keys [k_ctx[b,g,0:ctx_len[b],:] ; k_blk[b,0:S,g,:]] and the
+ * matching values: one joint softmax, no mask inside the block, no
+ * positional encoding.  Rows of the context cache at or past ctx_len[b] are
+ * never used.  fp32 accumulation, bf16 result.
+ *
+ *   q_blk   bf16 [B, S, Hq, dh]
+ *   k_blk   bf16 [B, S, Hkv, dh]       v_blk bf16 [B, S, Hkv, dh]
+ *   k_ctx   bf16 [B, Hkv, L_cap, dh]   v_ctx bf16 [B, Hkv, L_cap, dh]
+ *   ctx_len int32 [B] (device)
+ *   out     bf16 [B, S, Hq, dh]  (= [B*S, H])
+ *   ws      workspace of at least tt_workspace_bytes(d, TT_WS_ATTN) bytes
+ */
+TT_API tt_status tt_block_denoise_attn(const tt_dims* d, const tt_bf16* q_blk, const tt_bf16* k_blk,
+                                const tt_bf16* v_blk, const tt_bf16* k_ctx,
+                                const tt_bf16* v_ctx, const int32_t* ctx_len, tt_bf16* out,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * a2 - adaLN-single time modulation.
+ * Source: gist.science summary, "Training and Conditioning" (time conditioning
+ * through adaptive layer normalisation); snilld.dk, every layer modulated by a
+ * small adaLN-single block.  Reading of this library (the pages give no
+ * formula): for row r of sequence b = r / S,
+ *   [shift ; scale] = shift_scale + phi(t[b]),
+ *   phi(t) = [sin(t*w_i) for i < H] ++ [cos(t*w_i) for i < H], w_i = 10000^(-i/H),
+ *   y[r] = LN(x[r]) * (1 + scale) + shift,
+ * LN without affine parameters, biased variance, eps 1e-6.
+ *
+ *   x           bf16 [B*S, H]
+ *   shift_scale bf16 [2, H]   (row 0 shift, row 1 scale)
+ *   t           float [B] (device)
+ *   y           bf16 [B*S, H]   (may not alias x)
+ *   ws          workspace of at least tt_workspace_bytes(d, TT_WS_ADALN) bytes
+ */
+TT_API tt_status tt_adaln_modulate(const tt_dims* d, const tt_bf16* x, const tt_bf16* shift_scale,
+                            const float* t, tt_bf16* y, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * a3 + a4 - vocabulary projection, confidence and commit.
+ * Source: gist.science summary, "Training and Conditioning", Sampling:
+ * all masked positions are predicted in parallel; confident ones commit,
+ * uncertain ones stay masked, so the number committed per step adapts.
+ * Commit rule of this library: among positions with masked[b,s] != 0,
+ *   logits = logit_scale * y[b*S+s,:] . w[v,:]   (fp32 accumulation),
+ *   conf   = max_v softmax(logits),  tok = argmax_v (lowest id on ties);
+ * every one with conf >= gamma commits tok; if none in sequence b does, the
+ * single masked position with the largest conf commits (lowest s on ties).
+ * Committed positions get tokens[b,s] = tok and masked[b,s] = 0; positions
+ * already committed never change.  Logits are never written to memory.
+ *
+ *   y           bf16 [B*S, H]   (rows of unmasked positions are not read)
+ *   w           bf16 [V, H]     (one row per token: the "out x in" layout)
+ *   gamma       threshold in (0, 1];  logit_scale > 0 (1 = plain softmax)
+ *   tokens      int32 [B, S] in/out;  masked uint8 [B, S] in/out (1 = masked)
+ *   conf_out    float [B, S]  confidence of positions masked on entry, -1 elsewhere
+ *   argmax_out  int32 [B, S]  argmax of positions masked on entry, -1 elsewhere
+ *   n_committed int32 [B]     positions committed in this call
+ *   ws          workspace of at least tt_workspace_bytes(d, TT_WS_VOCAB) bytes
+ */
+TT_API tt_status tt_vocab_confidence_commit(const tt_dims* d, const tt_bf16* y, const tt_bf16* w,
+                                     float gamma, float logit_scale, int32_t* tokens,
+                                     uint8_t* masked, float* conf_out, int32_t* argmax_out,
+                                     int32_t* n_committed, void* ws, size_t ws_bytes,
+                                     void* stream);
+
+/*
+ * a5 + a6 - the denoise loop of one block: repeat
+ *   embed (Emb[token] for committed positions, e_mask for masked ones)
+ *   -> [q | k | v] = e . u_t^T  (one linear update, bf16 result)
+ *   -> tt_block_denoise_attn -> tt_adaln_modulate (t_b = masked count / S)
+ *   -> tt_vocab_confidence_commit
+ * until no position is masked or max_steps steps have run.
+ * Source: gist.science summary, "Generation Process" (the denoiser refines a
+ * block of S masked tokens over T steps; the context tower only updates after
+ * the block commits, so k_ctx / v_ctx are fixed here).
+ *
+ *   k_ctx, v_ctx, ctx_len  as in tt_block_denoise_attn
+ *   emb          bf16 [V, H]   token embedding table
+ *   e_mask       bf16 [H]      embedding of a masked position
+ *   u_t          bf16 [H + 2*Hkv*dh, H]   linear update, output-major:
+ *                rows [0,H) give q, [H, H+Hkv*dh) give k, the rest give v
+ *   shift_scale  bf16 [2, H];  w bf16 [V, H];  gamma, logit_scale as above
+ *   max_steps    1..1024 (S is always enough: every step commits at least
+ *                one position of every sequence that still has one masked)
+ *   tokens, masked  in/out state [B, S] (device); a partly committed block
+ *                resumes from where it is
+ *   steps_taken  int32 [B] (device): steps sequence b took in this call
+ *   commit_step  int32 [B, S] (device): step index at which (b,s) committed
+ *                in this call, -1 if it was committed on entry
+ *   steps_run    optional host int32*: number of steps that did work
+ *   ws           workspace of at least tt_workspace_bytes(d, TT_WS_LOOP) bytes
+ * Blocking: returns after the stream has finished the loop (one host
+ * synchronisation at the end, none per step).
+ */
+TT_API tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt_bf16* v_ctx,
+                                const int32_t* ctx_len, const tt_bf16* emb,
+                                const tt_bf16* e_mask, const tt_bf16* u_t,
+                                const tt_bf16* shift_scale, const tt_bf16* w, float gamma,
+                                float logit_scale, int32_t max_steps, int32_t* tokens,
+                                uint8_t* masked, int32_t* steps_taken, int32_t* commit_step,
+                                int32_t* steps_run, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TWOTOWER_H */

@@ -227,9 +227,9 @@ def vocab_confidence(y: np.ndarray, w_bits: np.ndarray, logit_scale: float = 1.0
     """conf, token and top-2 margins for each row of y against bf16 W.
 
     Rows are independent; they are processed a block at a time only to bound
-    memory (W is widened to float64 once).
+    memory.  ``w_bits`` may also be W already widened to float64.
     """
-    w = from_bf16(w_bits)
+    w = w_bits if w_bits.dtype == np.float64 else from_bf16(w_bits)
     R = y.shape[0]
     conf = np.empty(R)
     tok = np.empty(R, dtype=np.int64)
@@ -364,6 +364,7 @@ def denoise_block_loop(inp: dict, gamma: float, logit_scale: float = 1.0,
     v_ctx = from_bf16(inp["v_ctx"])
     E = from_bf16(inp["shift_scale"])
     u_t = from_bf16(inp["u_t"])
+    w = from_bf16(inp["w"])
     steps_taken = np.zeros(B, dtype=np.int64)
     commit_step = np.full((B, S), -1, dtype=np.int64)
     max_steps = S if max_steps is None else max_steps
@@ -379,7 +380,7 @@ def denoise_block_loop(inp: dict, gamma: float, logit_scale: float = 1.0,
         active = masked.any(axis=1)
         e = embed_block(tokens, masked, inp["emb"], inp["e_mask"])
         q, k, v = linear_update(e, u_t, Hq, Hkv, dh)
-        r = denoise_step(q, k, v, k_ctx, v_ctx, inp["ctx_len"], E, inp["w"], tokens, masked,
+        r = denoise_step(q, k, v, k_ctx, v_ctx, inp["ctx_len"], E, w, tokens, masked,
                          gamma, logit_scale)
         commit_step[r["committed"]] = step
         steps_taken[active] = step + 1

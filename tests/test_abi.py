@@ -1,0 +1,136 @@
+"""The C-ABI library loads, exports every declared symbol, and its host-side
+argument checks reject bad calls before anything reaches a GPU.
+
+No GPU needed: validation runs on the host and returns before any CUDA call,
+so fake (never dereferenced) pointers are enough here.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_wise_diffusion_b200 as tt
+import tt_inputs
+from block_wise_diffusion_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "twotower.h")
+FAKE = 1 << 20  # 16-byte aligned, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return tt.lib()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"TT_API\s+[\w\s\*]+?\b(tt_\w+)\s*\(", src)))
+
+
+def test_header_and_binding_agree():
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    assert sorted(tt.EXPORTS) == syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_status_strings(L):
+    for code, name in tt.STATUS.items():
+        assert tt.tt_status_string(code) == name
+    assert tt.tt_status_string(99) == "TT_ERR_UNKNOWN"
+
+
+def _d(**kw):
+    base = dict(B=8, S=16, Hq=32, Hkv=2, dh=128, V=131072, L_cap=4096)
+    base.update(kw)
+    return tt.Dims(base["B"], base["S"], base["Hq"], base["Hkv"], base["dh"],
+                   base.get("H", base["Hq"] * base["dh"]), base["V"], base["L_cap"])
+
+
+def test_workspace_sizes(L):
+    d = _d()
+    attn = tt.tt_workspace_bytes(d, tt.TT_WS_ATTN)
+    vocab = tt.tt_workspace_bytes(d, tt.TT_WS_VOCAB)
+    loop = tt.tt_workspace_bytes(d, tt.TT_WS_LOOP)
+    assert tt.tt_workspace_bytes(d, tt.TT_WS_ADALN) == 256
+    assert loop >= vocab and loop >= attn
+    # vocab: 128 rows of y (1 MiB) + 512 tiles x 128 rows x 12 B of tile statistics
+    assert vocab >= 128 * 4096 * 2 + 512 * 128 * 12
+    # all positions of all sequences fit one query tile when S*G <= 256
+    tiny = tt.dims(tt_inputs.workload("tiny"))
+    assert tt.tt_workspace_bytes(tiny, tt.TT_WS_LOOP) > 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(S=8), 2), (dict(dh=96), 2), (dict(Hkv=3), 1), (dict(Hq=24, Hkv=2), 2),
+    (dict(H=1000), 1), (dict(B=0), 1), (dict(V=1), 1), (dict(L_cap=-1), 1),
+])
+def test_bad_dims_rejected(L, kw, code):
+    d = _d(**kw)
+    assert L.tt_workspace_bytes(ctypes.byref(d), 0) == 0
+    r = L.tt_block_denoise_attn(ctypes.byref(d), *([FAKE] * 7), FAKE, 1 << 40, None)
+    assert r == code, tt.tt_last_error()
+    assert tt.tt_last_error()
+
+
+def test_pointer_and_workspace_checks(L):
+    d = _d()
+    ws_need = tt.tt_workspace_bytes(d, tt.TT_WS_ATTN)
+    args = [FAKE] * 7
+    r = L.tt_block_denoise_attn(ctypes.byref(d), *args, FAKE, ws_need - 1, None)
+    assert r == 3 and "workspace" in tt.tt_last_error()
+    bad = list(args)
+    bad[0] = None
+    assert L.tt_block_denoise_attn(ctypes.byref(d), *bad, FAKE, ws_need, None) == 1
+    assert "q_blk" in tt.tt_last_error()
+    bad[0] = FAKE + 2                          # misaligned for TMA
+    assert L.tt_block_denoise_attn(ctypes.byref(d), *bad, FAKE, ws_need, None) == 1
+    assert "aligned" in tt.tt_last_error()
+    assert L.tt_block_denoise_attn(ctypes.byref(d), *args, FAKE + 16, ws_need, None) == 1
+    assert L.tt_adaln_modulate(ctypes.byref(d), FAKE, FAKE, FAKE, FAKE, FAKE, 256, None) == 1
+
+
+def test_commit_and_loop_argument_checks(L):
+    d = _d()
+    wsb = tt.tt_workspace_bytes(d, tt.TT_WS_VOCAB)
+    call = lambda g, s: L.tt_vocab_confidence_commit(
+        ctypes.byref(d), FAKE, FAKE, ctypes.c_float(g), ctypes.c_float(s), FAKE, FAKE, FAKE,
+        FAKE, FAKE, FAKE, wsb, None)
+    assert call(0.0, 1.0) == 1
+    assert call(1.5, 1.0) == 1
+    assert call(0.8, 0.0) == 1
+    assert call(0.8, float("inf")) == 1
+    wsl = tt.tt_workspace_bytes(d, tt.TT_WS_LOOP)
+    loop = lambda ms: L.tt_denoise_block_loop(
+        ctypes.byref(d), *([FAKE] * 8), ctypes.c_float(0.8), ctypes.c_float(1.0), ms,
+        *([FAKE] * 4), None, FAKE, wsl, None)
+    assert loop(0) == 1
+    assert loop(2000) == 1
+
+
+def test_split_knob(L):
+    with pytest.raises(tt.TTError):
+        tt.tt_set_attn_splits(65)
+    d = _d(B=1, L_cap=65536)
+    tt.tt_set_attn_splits(1)
+    one = tt.tt_workspace_bytes(d, tt.TT_WS_ATTN)
+    tt.tt_set_attn_splits(8)
+    eight = tt.tt_workspace_bytes(d, tt.TT_WS_ATTN)
+    tt.tt_set_attn_splits(0)
+    assert one == 256 and eight > one
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    d = _d()
+    x = torch.zeros(4)
+    with pytest.raises(ValueError):
+        tt.tt_adaln_modulate(d, x, x, x, x, x)

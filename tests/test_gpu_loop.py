@@ -1,0 +1,143 @@
+"""Parity of tt_denoise_block_loop with the oracle's loop, step by step.
+
+The oracle is teacher-forced: at every step it starts from the GPU's state
+(rebuilt from commit_step and the final tokens), so one excluded near tie
+cannot cascade.  Each step's commit set and committed tokens must then match
+bit for bit, outside the near-tie exclusions of tests/_gpu.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_wise_diffusion_b200 as tt
+import tt_inputs
+from oracle import twotower_oracle as O
+from tests import _gpu as G
+
+pytestmark = pytest.mark.gpu
+
+LOOP_INPUTS = ["k_ctx", "v_ctx", "shift_scale", "w", "emb", "e_mask", "u_t"]
+
+
+def run_loop_gpu(d, inp, gamma, logit_scale, max_steps=None):
+    D = tt.dims(d)
+    dv = {k: G.dev_bf16(inp[k]) for k in LOOP_INPUTS}
+    tokens = G.dev(inp["tokens"])
+    masked = G.dev(inp["masked"])
+    steps_taken = torch.full((d.B,), -7, dtype=torch.int32, device="cuda")
+    commit_step = torch.full((d.B, d.S), -7, dtype=torch.int32, device="cuda")
+    ws = G.workspace(D, tt.TT_WS_LOOP)
+    n = tt.tt_denoise_block_loop(D, dv["k_ctx"], dv["v_ctx"], G.dev(inp["ctx_len"]), dv["emb"],
+                                 dv["e_mask"], dv["u_t"], dv["shift_scale"], dv["w"], gamma,
+                                 logit_scale, max_steps or d.S, tokens, masked, steps_taken,
+                                 commit_step, ws)
+    return dict(tokens=tokens.cpu().numpy(), masked=masked.cpu().numpy(),
+                steps_taken=steps_taken.cpu().numpy(), commit_step=commit_step.cpu().numpy(),
+                steps_run=n)
+
+
+def slice_batch(inp, bsel):
+    out = dict(inp)
+    for k in ("k_ctx", "v_ctx", "ctx_len", "tokens", "masked"):
+        out[k] = inp[k][bsel]
+    return out
+
+
+def compare_teacher_forced(inp, g, gamma, logit_scale, bsel=None):
+    """Re-run the oracle from the GPU's state at every step; return counts."""
+    if bsel is not None:
+        inp = slice_batch(inp, bsel)
+        g = {k: (v[bsel] if isinstance(v, np.ndarray) else v) for k, v in g.items()}
+    m0 = inp["masked"].astype(bool)
+    cs = g["commit_step"]
+
+    def state(step):
+        done = (cs >= 0) & (cs < step)
+        tok = np.where(done, g["tokens"], inp["tokens"])
+        return tok, m0 & ~done
+
+    r = O.denoise_block_loop(inp, gamma, logit_scale, max_steps=int(cs.max()) + 1, teacher=state)
+    n_cmp = n_ex = 0
+    for k, st in enumerate(r["trace"]):
+        tok_k, m_k = state(k)
+        for b in range(m_k.shape[0]):
+            if not m_k[b].any():
+                continue
+            gpu_c = cs[b] == k
+            ora_c = st["committed"][b]
+            conf = st["conf"][b]
+            ex = (m_k[b] & G.derived_excluded_threshold(conf, gamma)).any()
+            ex |= (ora_c & G.derived_excluded_argmax(st["gap_l"][b])).any()
+            if st["fallback"][b]:
+                cb = np.sort(conf[m_k[b]])[::-1]
+                ex |= len(cb) > 1 and cb[0] != cb[1] and (cb[0] - cb[1]) / cb[0] < G.TIE_FALLBACK_REL
+            if ex:
+                n_ex += 1
+                continue
+            n_cmp += 1
+            np.testing.assert_array_equal(gpu_c, ora_c, err_msg=f"step {k} seq {b}")
+            np.testing.assert_array_equal(g["tokens"][b][gpu_c], st["tok"][b][ora_c],
+                                          err_msg=f"step {k} seq {b} tokens")
+    return n_cmp, n_ex
+
+
+def check_invariants(d, inp, g):
+    m0 = inp["masked"].astype(bool)
+    assert not g["masked"].any()
+    np.testing.assert_array_equal(g["tokens"][~m0], inp["tokens"][~m0])     # never change
+    assert np.all(g["commit_step"][~m0] == -1)
+    assert np.all(g["commit_step"][m0] >= 0)
+    assert np.all((g["tokens"] >= 0) & (g["tokens"] < d.V))
+    n0 = m0.sum(axis=1)
+    assert np.all(g["steps_taken"] <= n0)
+    assert np.all((g["steps_taken"] >= 1) | (n0 == 0))
+    # every step commits at least one position of every sequence still masked
+    for b in range(d.B):
+        if n0[b]:
+            steps = set(g["commit_step"][b][m0[b]].tolist())
+            assert steps == set(range(g["steps_taken"][b]))
+    assert g["steps_run"] == g["steps_taken"].max()
+
+
+@pytest.mark.parametrize("gamma,logit_scale", [(0.8, 1.0), (0.5, 12.0), (0.95, 40.0)])
+def test_loop_tiny(gamma, logit_scale):
+    d = tt_inputs.workload("tiny", B=3, precommit=("uniform", 0.0, 0.75))
+    inp = tt_inputs.generate(d, seed=31)
+    g = run_loop_gpu(d, inp, gamma, logit_scale)
+    check_invariants(d, inp, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, gamma, logit_scale)
+    assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
+
+
+def test_loop_canonical_scale_commits_in_position_order():
+    d = tt_inputs.workload("tiny", B=2)
+    inp = tt_inputs.generate(d, seed=32)
+    g = run_loop_gpu(d, inp, 0.8, 1.0)
+    check_invariants(d, inp, g)
+    # identical masked positions tie; the lowest position commits first
+    np.testing.assert_array_equal(g["commit_step"], np.tile(np.arange(16), (2, 1)))
+    compare_teacher_forced(inp, g, 0.8, 1.0)
+
+
+def test_loop_resume_equals_single_call():
+    d = tt_inputs.workload("tiny", B=2)
+    inp = tt_inputs.generate(d, seed=33)
+    full = run_loop_gpu(d, inp, 0.5, 12.0)
+    part = run_loop_gpu(d, inp, 0.5, 12.0, max_steps=1)
+    assert part["masked"].any()
+    inp2 = dict(inp, tokens=part["tokens"], masked=part["masked"])
+    rest = run_loop_gpu(d, inp2, 0.5, 12.0)
+    np.testing.assert_array_equal(rest["tokens"], full["tokens"])
+
+
+@pytest.mark.parametrize("logit_scale", [1.0, 8.0])
+def test_loop_full_mid_shape_sampled_sequences(logit_scale):
+    d = tt_inputs.workload("mid")
+    inp = tt_inputs.generate(d, seed=0)
+    g = run_loop_gpu(d, inp, 0.8, logit_scale)
+    check_invariants(d, inp, g)
+    if logit_scale == 1.0:
+        assert g["steps_run"] == 16
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, bsel=np.array([0, 5]))
+    print(f"mid loop scale={logit_scale}: compared {n_cmp} sequence-steps, excluded {n_ex}")
+    assert n_cmp > 0 and n_ex <= 2
