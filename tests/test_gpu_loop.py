@@ -122,12 +122,15 @@ def test_loop_canonical_scale_commits_in_position_order():
 def test_loop_resume_equals_single_call():
     d = tt_inputs.workload("tiny", B=2)
     inp = tt_inputs.generate(d, seed=33)
-    full = run_loop_gpu(d, inp, 0.5, 12.0)
-    part = run_loop_gpu(d, inp, 0.5, 12.0, max_steps=1)
-    assert part["masked"].any()
+    # unit logit scale: one commit per sequence per step, so a 3-step call
+    # leaves 13 masked positions to resume from
+    full = run_loop_gpu(d, inp, 0.8, 1.0)
+    part = run_loop_gpu(d, inp, 0.8, 1.0, max_steps=3)
+    assert part["masked"].sum(axis=1).tolist() == [13, 13]
     inp2 = dict(inp, tokens=part["tokens"], masked=part["masked"])
-    rest = run_loop_gpu(d, inp2, 0.5, 12.0)
+    rest = run_loop_gpu(d, inp2, 0.8, 1.0)
     np.testing.assert_array_equal(rest["tokens"], full["tokens"])
+    assert rest["steps_run"] == 13
 
 
 @pytest.mark.parametrize("logit_scale", [1.0, 8.0])
