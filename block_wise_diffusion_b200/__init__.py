@@ -15,7 +15,7 @@ import os
 __all__ = [
     "TTError", "Dims", "lib", "lib_path", "dims", "workspace", "tt_workspace_bytes",
     "tt_block_denoise_attn", "tt_adaln_modulate", "tt_vocab_confidence_commit",
-    "tt_denoise_block_loop", "tt_device_status", "tt_launch_count", "tt_set_attn_splits",
+    "tt_denoise_block_loop", "tt_vocab_confidence_commit_noalloc", "tt_device_status", "tt_launch_count", "tt_set_attn_splits",
     "tt_status_string", "tt_last_error", "EXPORTS", "tt_profile_enable", "tt_profile_read",
     "profile_table", "KERNEL_KINDS",
     "TT_WS_ATTN", "TT_WS_ADALN", "TT_WS_VOCAB", "TT_WS_LOOP",
@@ -33,6 +33,7 @@ EXPORTS = (
     "tt_status_string", "tt_last_error", "tt_workspace_bytes", "tt_device_status",
     "tt_launch_count", "tt_set_attn_splits", "tt_block_denoise_attn", "tt_adaln_modulate",
     "tt_vocab_confidence_commit", "tt_denoise_block_loop", "tt_profile_enable", "tt_profile_read",
+    "tt_vocab_confidence_commit_noalloc",
 )
 KERNEL_KINDS = ("plan", "embed", "gemm_qkv", "attn", "merge", "adaln", "gemm_vocab", "commit",
                 "gather", "init")
@@ -85,6 +86,9 @@ def lib() -> ctypes.CDLL:
         L.tt_vocab_confidence_commit.argtypes = (
             [ctypes.POINTER(Dims), _P, _P, ctypes.c_float, ctypes.c_float] + [_P] * 5
             + [_P, ctypes.c_size_t, _P])
+        L.tt_vocab_confidence_commit_noalloc.restype = ctypes.c_int
+        L.tt_vocab_confidence_commit_noalloc.argtypes = (
+            [ctypes.POINTER(Dims), _P, _P, ctypes.c_float, ctypes.c_float] + [_P] * 5 + [_P])
         L.tt_denoise_block_loop.restype = ctypes.c_int
         L.tt_denoise_block_loop.argtypes = (
             [ctypes.POINTER(Dims)] + [_P] * 8 + [ctypes.c_float, ctypes.c_float, ctypes.c_int32]
@@ -198,6 +202,18 @@ def tt_vocab_confidence_commit(d: Dims, y, w, gamma: float, logit_scale: float, 
         ctypes.byref(d), _ptr(y), _ptr(w), float(gamma), float(logit_scale), _ptr(tokens),
         _ptr(masked), _ptr(conf_out), _ptr(argmax_out), _ptr(n_committed), _ptr(ws), ws.numel(),
         _stream(stream)), "tt_vocab_confidence_commit")
+
+
+def tt_vocab_confidence_commit_noalloc(d: Dims, y, w, gamma: float, logit_scale: float,
+                                       tokens, masked, conf_out, argmax_out, n_committed,
+                                       stream=None) -> None:
+    """tt_vocab_confidence_commit without a workspace, for callers that cannot
+    allocate device memory; its scratch is a 16 MiB array built into the
+    library (calls that overlap on the GPU must be serialised)."""
+    _check(lib().tt_vocab_confidence_commit_noalloc(
+        ctypes.byref(d), _ptr(y), _ptr(w), float(gamma), float(logit_scale), _ptr(tokens),
+        _ptr(masked), _ptr(conf_out), _ptr(argmax_out), _ptr(n_committed), _stream(stream)),
+        "tt_vocab_confidence_commit_noalloc")
 
 
 def tt_denoise_block_loop(d: Dims, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale, w,

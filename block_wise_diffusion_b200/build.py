@@ -13,7 +13,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtwotower.so")
-SOURCES = ["tt_api.cu", "tt_gemm.cu", "tt_attn.cu", "tt_small.cu"]
+SOURCES = ["tt_api.cu", "tt_gemm.cu", "tt_attn.cu", "tt_small.cu", "tt_noalloc.cu"]
 HEADERS = ["tt_internal.h", "tt_ptx.cuh", os.path.join("..", "..", "include", "twotower.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

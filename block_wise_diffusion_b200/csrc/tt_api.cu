@@ -276,6 +276,9 @@ static tt_status check_ws(const tt_dims& d, int which, void* ws, size_t ws_bytes
   return TT_OK;
 }
 
+tt_status set_error(tt_status s, const char* msg) { return fail(s, "%s", msg); }
+tt_status check_dims_public(const tt_dims* d) { return check_dims(d); }
+
 // ---------------------------------------------------------- stage helpers
 struct AttnMaps {
   CUtensorMap q, kc, vc, kb, vb;

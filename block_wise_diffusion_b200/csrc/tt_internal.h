@@ -153,6 +153,11 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, ui
 
 void count_launch(int n = 1);
 
+// Record `msg` as the calling thread's last error and return `s`.
+tt_status set_error(tt_status s, const char* msg);
+// The shape checks of the public entry points.
+tt_status check_dims_public(const tt_dims* d);
+
 // Profiler hooks (no-ops unless tt_profile_enable(1)): bracket one launch.
 void prof_begin(int kind, cudaStream_t st);
 void prof_end(int kind, cudaStream_t st);

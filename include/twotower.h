@@ -221,6 +221,40 @@ TT_API tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, c
                                 uint8_t* masked, int32_t* steps_taken, int32_t* commit_step,
                                 int32_t* steps_run, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Allocation-free variant of tt_vocab_confidence_commit.
+ * The paper has no counterpart: this entry point exists for callers that
+ * cannot provide a workspace - code running inside another runtime's
+ * execution hook where device allocation is not allowed (an inference
+ * engine's plugin callback, say), a process whose device memory is fully
+ * reserved by its own pool, or a C caller with no allocator at all.
+ *
+ * Same arguments, results and commit rule as tt_vocab_confidence_commit,
+ * minus the workspace.  Its scratch is one built-in device array of 16 MiB
+ * (16777216 bytes) that every GPU which loads this library holds until the
+ * process exits.  A problem whose scratch exceeds it - 256 bytes of control
+ * words, the masked-row list (B*S*4 bytes), B*4 bytes of timesteps,
+ * B*S*H*2 bytes of gathered rows and three B*S*ceil(V/256)*4-byte arrays of
+ * tile statistics, each rounded up to 256 bytes - is rejected with
+ * TT_ERR_WORKSPACE before any launch.  It allocates nothing:
+ * no cudaMalloc/cudaFree and no allocating library routine.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents;
+ *    the call clears what must start at zero.  Calls whose work overlaps on
+ *    the GPU (different streams, or several host threads) race on it:
+ *    serialise them.
+ *  - Device-detected errors (a timed-out wait, a non-finite confidence) are
+ *    recorded in the array only; this variant does not report them.
+ */
+TT_API tt_status tt_vocab_confidence_commit_noalloc(const tt_dims* d, const tt_bf16* y,
+                                                    const tt_bf16* w, float gamma,
+                                                    float logit_scale, int32_t* tokens,
+                                                    uint8_t* masked, float* conf_out,
+                                                    int32_t* argmax_out, int32_t* n_committed,
+                                                    void* stream);
+
 #ifdef __cplusplus
 }
 #endif
