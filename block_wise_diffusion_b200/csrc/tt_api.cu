@@ -207,6 +207,18 @@ static AttnGeom attn_geom(const tt_dims& d) {
   return g;
 }
 
+// K splits of the linear-update GEMM: enough (tile, K range) units to fill
+// the SMs when the block has few rows; a power of two dividing H/64.
+static int qkv_ksplit(const tt_dims& d) {
+  const int rows = d.B * d.S;
+  const int n_qkv = d.H + 2 * d.Hkv * d.dh;
+  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kQkvBN - 1) / kQkvBN);
+  const int kb = d.H / kGemmBK;
+  int k = 1;
+  while (2 * k <= kb && kb % (2 * k) == 0 && tiles * 2 * k <= kNumSMs) k *= 2;
+  return k;
+}
+
 struct Carver {
   uint8_t* base;
   size_t off = 0;
@@ -229,9 +241,8 @@ struct Ws {
   uint16_t* y_c = nullptr;
   float* part_o = nullptr;
   float* part_ml = nullptr;
-  float* part_v = nullptr;
-  float* part_z = nullptr;
-  int* part_a = nullptr;
+  float4* stats = nullptr;
+  float* qkv_partial = nullptr;
   size_t total = 0;
 };
 
@@ -239,7 +250,7 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   Ws w;
   const size_t rows = (size_t)d.B * d.S;
-  const size_t n_vt = (size_t)(d.V + kGemmBN - 1) / kGemmBN;
+  const size_t n_vt = (size_t)(d.V + kVocabBN - 1) / kVocabBN;
   w.ctrl = c.take<int>(kCtrlBytes);
   if (which == TT_WS_ATTN || which == TT_WS_LOOP) {
     const AttnGeom g = attn_geom(d);
@@ -252,15 +263,15 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     w.rowlist = c.take<int>(rows * sizeof(int));
     w.tvec = c.take<float>((size_t)d.B * sizeof(float));
     w.y_c = c.take<uint16_t>(rows * d.H * 2);
-    w.part_v = c.take<float>(n_vt * rows * sizeof(float));
-    w.part_z = c.take<float>(n_vt * rows * sizeof(float));
-    w.part_a = c.take<int>(n_vt * rows * sizeof(int));
+    w.stats = c.take<float4>(n_vt * rows * sizeof(float4));
   }
   if (which == TT_WS_LOOP) {
     const size_t n_qkv = (size_t)d.H + 2 * (size_t)d.Hkv * d.dh;
     w.egath = c.take<uint16_t>(rows * d.H * 2);
     w.qkv = c.take<uint16_t>(rows * n_qkv * 2);
     w.attn_out = c.take<uint16_t>(rows * d.H * 2);
+    const int ks = qkv_ksplit(d);
+    if (ks > 1) w.qkv_partial = c.take<float>((size_t)ks * rows * n_qkv * sizeof(float));
   }
   w.total = (c.off + 255) & ~size_t(255);
   return w;
@@ -300,9 +311,8 @@ static tt_status build_attn_maps(const tt_dims& d, const AttnGeom& g, const tt_b
   return TT_OK;
 }
 
-static tt_status run_attn(const tt_dims& d, const AttnGeom& g, const AttnMaps& m,
-                          const int32_t* ctx_len, tt_bf16* out, const Ws& w, const int* active,
-                          cudaStream_t st) {
+static AttnArgs attn_args(const tt_dims& d, const AttnGeom& g, const int32_t* ctx_len,
+                          tt_bf16* out, const Ws& w, const int* active) {
   AttnArgs a;
   a.B = d.B;
   a.S = d.S;
@@ -325,8 +335,17 @@ static tt_status run_attn(const tt_dims& d, const AttnGeom& g, const AttnMaps& m
   a.part_o = w.part_o;
   a.part_ml = w.part_ml;
   a.err = w.ctrl;
+  return a;
+}
+
+// The attention launch; with `merge` the split partials are combined into
+// `out` by the merge kernel (the loop fuses that merge into adaLN instead).
+static tt_status run_attn(const tt_dims& d, const AttnGeom& g, const AttnMaps& m,
+                          const int32_t* ctx_len, tt_bf16* out, const Ws& w, const int* active,
+                          bool merge, cudaStream_t st) {
+  const AttnArgs a = attn_args(d, g, ctx_len, out, w, active);
   TT_LAUNCH(TT_K_ATTN, st, launch_attn(m.q, m.kc, m.vc, m.kb, m.vb, a, st));
-  if (g.n_splits > 1) TT_LAUNCH(TT_K_MERGE, st, launch_attn_merge(a, st));
+  if (merge && g.n_splits > 1) TT_LAUNCH(TT_K_MERGE, st, launch_attn_merge(a, st));
   return TT_OK;
 }
 
@@ -336,7 +355,7 @@ static tt_status run_vocab_gemm(const tt_dims& d, const Ws& w, const tt_bf16* W,
   const int rows = d.B * d.S;
   CUtensorMap tmA, tmB;
   if (!make_tmap_2d(&tmA, w.y_c, d.H, rows, (uint64_t)d.H * 2, kGemmBK, kGemmBM) ||
-      !make_tmap_2d(&tmB, W, d.H, d.V, (uint64_t)d.H * 2, kGemmBK, kGemmBN))
+      !make_tmap_2d(&tmB, W, d.H, d.V, (uint64_t)d.H * 2, kGemmBK, kVocabBN))
     return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the vocab GEMM");
   GemmArgs a{};
   a.M_alloc = rows;
@@ -344,13 +363,10 @@ static tt_status run_vocab_gemm(const tt_dims& d, const Ws& w, const tt_bf16* W,
   a.active = active;
   a.N = d.V;
   a.K = d.H;
-  a.part_v = w.part_v;
-  a.part_z = w.part_z;
-  a.part_a = w.part_a;
-  a.part_ld = rows;
+  a.stats = w.stats;
   a.scale_log2 = (float)(logit_scale * 1.4426950408889634);
   a.err = w.ctrl;
-  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((d.V + kGemmBN - 1) / kGemmBN);
+  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((d.V + kVocabBN - 1) / kVocabBN);
   TT_LAUNCH(TT_K_GEMM_VOCAB, st, launch_gemm_vocab(tmA, tmB, a, std::min(tiles, kNumSMs), st));
   return TT_OK;
 }
@@ -360,11 +376,8 @@ static CommitArgs commit_args(const tt_dims& d, const Ws& w, float gamma, float 
   CommitArgs c{};
   c.B = d.B;
   c.S = d.S;
-  c.n_vt = (d.V + kGemmBN - 1) / kGemmBN;
-  c.part_ld = d.B * d.S;
-  c.part_v = w.part_v;
-  c.part_z = w.part_z;
-  c.part_a = w.part_a;
+  c.n_vt = (d.V + kVocabBN - 1) / kVocabBN;
+  c.stats = w.stats;
   c.scale_log2 = (float)(logit_scale * 1.4426950408889634);
   c.gamma = gamma;
   c.rowlist = w.rowlist;
@@ -478,7 +491,7 @@ tt_status tt_block_denoise_attn(const tt_dims* d, const tt_bf16* q_blk, const tt
                            v_ctx, &m));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   TT_CUDA(cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st));
-  return run_attn(*d, g, m, ctx_len, out, w, nullptr, st);
+  return run_attn(*d, g, m, ctx_len, out, w, nullptr, true, st);
 }
 
 tt_status tt_adaln_modulate(const tt_dims* d, const tt_bf16* x, const tt_bf16* shift_scale,
@@ -565,7 +578,7 @@ tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt
 
   CUtensorMap tmE, tmU;
   if (!make_tmap_2d(&tmE, w.egath, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM) ||
-      !make_tmap_2d(&tmU, u_t, d->H, n_qkv, (uint64_t)d->H * 2, kGemmBK, kGemmBN))
+      !make_tmap_2d(&tmU, u_t, d->H, n_qkv, (uint64_t)d->H * 2, kGemmBK, kQkvBN))
     return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
   AttnMaps m;
   TT_CHECK(build_attn_maps(*d, g, w.qkv, n_qkv, w.qkv + d->H, w.qkv + d->H + d->Hkv * d->dh,
@@ -582,27 +595,44 @@ tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt
   ga.C = w.qkv;
   ga.ldc = n_qkv;
   ga.err = w.ctrl;
-  const int qkv_tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kGemmBN - 1) / kGemmBN);
-  PlanArgs p{d->B, d->S, masked, w.rowlist, w.tvec, w.ctrl, 1};
+  ga.ksplit = qkv_ksplit(*d);
+  ga.partial = w.qkv_partial;
+  const int qkv_tiles =
+      ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kQkvBN - 1) / kQkvBN) * ga.ksplit;
+  // Step 0's plan and the embedding of every position; afterwards the commit
+  // kernel re-embeds what it commits and its last CTA plans the next step.
+  PlanArgs p{d->B, d->S, masked, w.rowlist, w.tvec, w.ctrl, 0};
+  TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
+  TT_LAUNCH(TT_K_EMBED, st, launch_embed(tokens, masked, emb, e_mask, w.egath, rows, d->H, d->V,
+                                         active, w.ctrl, st));
   for (int step = 0; step < max_steps; ++step) {
-    TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
-    TT_LAUNCH(TT_K_EMBED, st, launch_embed(tokens, masked, emb, e_mask, w.egath, rows, d->H, d->V, active, w.ctrl,
-                         st));
     TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(tmE, tmU, ga, std::min(qkv_tiles, kNumSMs), st));
-    TT_CHECK(run_attn(*d, g, m, ctx_len, w.attn_out, w, active, st));
-    TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, shift_scale, w.tvec, w.y_c, rows, d->S,
-                                           d->H, w.rowlist, w.ctrl + CTRL_M, active, st));
+    if (ga.ksplit > 1)
+      TT_LAUNCH(TT_K_GEMM_QKV, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
+                                                        w.qkv, n_qkv, active, st));
+    TT_CHECK(run_attn(*d, g, m, ctx_len, w.attn_out, w, active, false, st));
+    if (g.n_splits > 1) {
+      const AttnArgs aa = attn_args(*d, g, ctx_len, w.attn_out, w, active);
+      TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, shift_scale, w.tvec, w.y_c, w.rowlist,
+                                                   w.ctrl + CTRL_M, rows, st));
+    } else {
+      TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, shift_scale, w.tvec, w.y_c, rows, d->S,
+                                             d->H, w.rowlist, w.ctrl + CTRL_M, active, st));
+    }
     TT_CHECK(run_vocab_gemm(*d, w, W, logit_scale, w.ctrl + CTRL_M, active, st));
     CommitArgs c = commit_args(*d, w, gamma, logit_scale, tokens, masked);
     c.commit_step = commit_step;
     c.steps_taken = steps_taken;
     c.step = step;
     c.active = active;
+    c.emb = emb;
+    c.egath = w.egath;
+    c.H = d->H;
+    c.plan_next = 1;
+    c.plan_rowlist = w.rowlist;
+    c.plan_t = w.tvec;
     TT_LAUNCH(TT_K_COMMIT, st, launch_commit(c, st));
   }
-  PlanArgs pf = p;
-  pf.count_step = 0;
-  TT_LAUNCH(TT_K_PLAN, st, launch_plan(pf, st));
   int h[8];
   TT_CHECK(read_ctrl(w, st, h));
   if (g_prof_on.load()) prof_harvest();

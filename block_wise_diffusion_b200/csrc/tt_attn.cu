@@ -25,6 +25,11 @@
 
 #include "tt_ptx.cuh"
 
+// Timeline hooks for instrumented builds; empty in the library build.
+#ifndef TT_TRACE_POINT
+#define TT_TRACE_POINT(cond, slot, t)
+#endif
+
 namespace tt {
 
 namespace {
@@ -71,10 +76,56 @@ __device__ __forceinline__ TileInfo tile_info(int t, int has_blk, int k0, int k1
   return ti;
 }
 
+// Row max over the valid columns of a 64-key score tile (thread = row).
+template <bool kFull>
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[64], int nvalid) {
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 64; j += 4) {
+    const float v0 = __uint_as_float(sr[j]), v1 = __uint_as_float(sr[j + 1]);
+    const float v2 = __uint_as_float(sr[j + 2]), v3 = __uint_as_float(sr[j + 3]);
+    if (kFull) {
+      m0 = fmaxf(m0, v0);
+      m1 = fmaxf(m1, v1);
+      m2 = fmaxf(m2, v2);
+      m3 = fmaxf(m3, v3);
+    } else {
+      m0 = (j < nvalid) ? fmaxf(m0, v0) : m0;
+      m1 = (j + 1 < nvalid) ? fmaxf(m1, v1) : m1;
+      m2 = (j + 2 < nvalid) ? fmaxf(m2, v2) : m2;
+      m3 = (j + 3 < nvalid) ? fmaxf(m3, v3) : m3;
+    }
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+
+// p = exp2(s*c - m) for the valid columns (0 elsewhere), packed to bf16
+// pairs; returns the row sum of p.
+template <bool kFull>
+__device__ __forceinline__ float exp_pack(const uint32_t (&sr)[64], int nvalid, float c, float m,
+                                          uint32_t (&pk)[32]) {
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+  for (int j = 0; j < 64; j += 2) {
+    float p0 = ex2(fmaf(__uint_as_float(sr[j]), c, -m));
+    float p1 = ex2(fmaf(__uint_as_float(sr[j + 1]), c, -m));
+    if (!kFull) {
+      p0 = (j < nvalid) ? p0 : 0.f;
+      p1 = (j + 1 < nvalid) ? p1 : 0.f;
+    }
+    s0 += p0;
+    s1 += p1;
+    pk[j >> 1] = pack_bf16x2(p0, p1);
+  }
+  return s0 + s1;
+}
+
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                 const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKb,
                 const __grid_constant__ CUtensorMap tmVb, const AttnArgs a) {
+  griddep_launch();
+  griddep_wait();
   extern __shared__ uint8_t smem_raw[];
   if (a.active != nullptr && *a.active == 0) return;
   const int split = blockIdx.x, qt = blockIdx.y, pair = blockIdx.z;
@@ -111,16 +162,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = kv_full + kAttnStages;
-  uint64_t* s_full = kv_empty + kAttnStages;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
+  uint64_t* s_full = kv_empty + kAttnStages;  // [half][buffer]
+  uint64_t* p_full = s_full + 4;              // [half]: P written (and O corrected)
+  uint64_t* pv_done = p_full + 2;             // [half]: last P.V of the half finished
+  uint64_t* o_full = pv_done + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t tmem_cols = (halves * (64 + dh) <= 128) ? 128u
-                             : (halves * (64 + dh) <= 256) ? 256u
-                                                          : 512u;
+  // TMEM: S[half][buffer] (64 fp32 columns each, double-buffered so the next
+  // tile's scores are computed while this tile's softmax runs), then O[half].
+  const uint32_t tmem_need = halves * (2 * kAttnBN + dh);
+  const uint32_t tmem_cols = tmem_need <= 128 ? 128u : tmem_need <= 256 ? 256u : 512u;
+  const uint32_t tO0 = halves * 2 * kAttnBN;
 
   // Rows of a half that the Q box does not cover must be finite (they only
   // produce output rows that are discarded): clear Q when the box is short.
@@ -136,9 +190,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
+    for (int i = 0; i < 4; ++i) mbar_init(&s_full[i], 1);
     for (int h = 0; h < 2; ++h) {
-      mbar_init(&s_full[h], 1);
       mbar_init(&p_full[h], 128);
+      mbar_init(&pv_done[h], 1);
     }
     mbar_init(o_full, 1);
     *abort_flag = 0;
@@ -171,6 +226,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int st = t % kAttnStages;
         const uint32_t ph = (uint32_t)(t / kAttnStages) & 1u;
         if (!mbar_wait(&kv_empty[st], ph ^ 1u, a.err, abort_flag, WHERE_ATTN_PRODUCER)) break;
+        TT_TRACE_POINT(true, 0, t);
         const TileInfo ti = tile_info(t, has_blk, k0, k1, a.S);
         uint8_t* dk = sK + st * nsub * kSub;
         uint8_t* dv = sV + st * nsub * kSub;
@@ -196,13 +252,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t idS = idesc_bf16(128, kAttnBN, false, false);
     const uint32_t idO = idesc_bf16(128, dh, false, true);
     const uint32_t q0 = smem_u32(sQ), k0s = smem_u32(sK), v0s = smem_u32(sV), p0s = smem_u32(sP);
-    auto issue_S = [&](int h, int st) {
+    auto issue_S = [&](int h, int st, int buf) {
       for (int kk = 0; kk < dh / 16; ++kk) {
         const int xh = kk >> 2;
         const uint32_t off = (uint32_t)(kk & 3) * 32;
         const uint64_t ad = sdesc_sw128(q0 + (h * nsub + xh) * kQSub + off, 16, 1024);
         const uint64_t bd = sdesc_sw128(k0s + (st * nsub + xh) * kSub + off, 16, 1024);
-        umma_bf16_ss(tmem + h * 64, ad, bd, idS, kk > 0);
+        umma_bf16_ss(tmem + (h * 2 + buf) * kAttnBN, ad, bd, idS, kk > 0);
       }
     };
     auto issue_PV = [&](int h, int st, bool acc) {
@@ -210,7 +266,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint64_t ad = sdesc_sw128(p0s + h * kPHalf + kk * 32, 16, 1024);
         // V as an MN-major operand: 64-wide dh blocks kSub apart, 8-key groups 1 KB apart.
         const uint64_t bd = sdesc_sw128(v0s + st * nsub * kSub + kk * 2048, kSub, 1024);
-        umma_bf16_ss(tmem + halves * 64 + h * dh, ad, bd, idO, (acc || kk > 0) ? 1u : 0u);
+        umma_bf16_ss(tmem + tO0 + h * dh, ad, bd, idO, (acc || kk > 0) ? 1u : 0u);
       }
     };
     // V rows past the valid keys of a tile may hold anything (other
@@ -228,54 +284,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       __syncwarp();
     };
-    bool ok = mbar_wait(q_full, 0, a.err, abort_flag, WHERE_ATTN_MMA);
-    if (ok) ok = mbar_wait(&kv_full[0], 0, a.err, abort_flag, WHERE_ATTN_MMA);
-    if (ok) {
+    // Issue order: scores run two tiles ahead (S(0), S(1) up front), and in
+    // each iteration P(t).V is issued for each half the moment its softmax
+    // has written P, before S(t+2) - so a P.V never queues behind the next
+    // tile's score MMAs and the softmax never waits for its P buffer.
+    // S(t+2) reuses the buffer of tile t, which the softmax released with P(t).
+    auto issue_scores = [&](int tt) -> bool {
+      const int stt = tt % kAttnStages;
+      if (!mbar_wait(&kv_full[stt], (uint32_t)(tt / kAttnStages) & 1u, a.err, abort_flag,
+                     WHERE_ATTN_MMA))
+        return false;
+      TT_TRACE_POINT(lane == 0, 1, tt);
       tc_fence_after();
-      prep(0, 0);
+      prep(tt, stt);
       if (lane == 0) {
-        issue_S(0, 0);
-        umma_commit(&s_full[0]);
-        if (halves == 2) {
-          issue_S(1, 0);
-          umma_commit(&s_full[1]);
+        for (int h = 0; h < halves; ++h) {
+          issue_S(h, stt, tt & 1);
+          umma_commit(&s_full[h * 2 + (tt & 1)]);
         }
       }
       __syncwarp();
-    }
+      TT_TRACE_POINT(lane == 0, 2, tt);
+      return true;
+    };
+    bool ok = mbar_wait(q_full, 0, a.err, abort_flag, WHERE_ATTN_MMA);
+    for (int tt = 0; ok && tt < 2 && tt < n_tiles; ++tt) ok = issue_scores(tt);
     for (int t = 0; ok && t < n_tiles; ++t) {
       const int st = t % kAttnStages;
-      const int t1 = t + 1;
-      const int st1 = t1 % kAttnStages;
-      const uint32_t ph1 = (uint32_t)(t1 / kAttnStages) & 1u;
-      if (!mbar_wait(&p_full[0], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_MMA)) break;
-      tc_fence_after();
-      if (lane == 0) issue_PV(0, st, t > 0);
-      __syncwarp();
-      if (t1 < n_tiles) {
-        if (!mbar_wait(&kv_full[st1], ph1, a.err, abort_flag, WHERE_ATTN_MMA)) break;
+      for (int h = 0; h < halves; ++h) {
+        if (!mbar_wait(&p_full[h], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_MMA)) {
+          ok = false;
+          break;
+        }
+        TT_TRACE_POINT(lane == 0, 3 + h, t);
         tc_fence_after();
-        prep(t1, st1);
         if (lane == 0) {
-          issue_S(0, st1);
-          umma_commit(&s_full[0]);
+          issue_PV(h, st, t > 0);
+          umma_commit(&pv_done[h]);
         }
         __syncwarp();
       }
-      if (halves == 2) {
-        if (!mbar_wait(&p_full[1], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_MMA)) break;
-        tc_fence_after();
-        if (lane == 0) issue_PV(1, st, t > 0);
-        __syncwarp();
-      }
-      if (lane == 0) {
-        umma_commit(&kv_empty[st]);
-        if (halves == 2 && t1 < n_tiles) {
-          issue_S(1, st1);
-          umma_commit(&s_full[1]);
-        }
-      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(&kv_empty[st]);
       __syncwarp();
+      if (t + 2 < n_tiles) ok = issue_scores(t + 2);
     }
     if (lane == 0) umma_commit(o_full);
     __syncwarp();
@@ -286,29 +338,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int r = q * 32 + lane;
     if (wg < halves) {
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-      const uint32_t tS = tmem + wg * 64 + lane_off;
-      const uint32_t tO = tmem + halves * 64 + wg * dh + lane_off;
+      const uint32_t tS = tmem + wg * 2 * kAttnBN + lane_off;
+      const uint32_t tO = tmem + tO0 + wg * dh + lane_off;
       uint8_t* prow = sP + wg * kPHalf + r * 128;
       const float c = a.scale_log2;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int t = 0; t < n_tiles; ++t) {
-        if (!mbar_wait(&s_full[wg], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
+        const int buf = t & 1;
+        if (!mbar_wait(&s_full[wg * 2 + buf], (uint32_t)(t >> 1) & 1u, a.err, abort_flag,
+                       WHERE_ATTN_SOFTMAX)) {
           ok = false;
           break;
         }
+        TT_TRACE_POINT(lane == 0 && q == 0, 5 + 5 * wg, t);
         tc_fence_after();
         const int nvalid = tile_info(t, has_blk, k0, k1, a.S).nvalid;
         uint32_t sr[64];
-        tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(tS + buf * kAttnBN, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(tS + buf * kAttnBN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
         tmem_wait_ld();
-        float mx = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          const float v = __uint_as_float(sr[j]);
-          mx = (j < nvalid) ? fmaxf(mx, v) : mx;
-        }
+        TT_TRACE_POINT(lane == 0 && q == 0, 6 + 5 * wg, t);
+        const bool full = nvalid == kAttnBN;
+        float mx = full ? row_max<true>(sr, nvalid) : row_max<false>(sr, nvalid);
         const float mxs = mx * c;
         const bool need = mxs > m + kRescaleThreshold;
         float alpha = 1.f;
@@ -317,29 +369,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m = mxs;
         }
         l *= alpha;
-        if (t > 0 && __any_sync(0xffffffffu, need)) {
-          for (int c0 = 0; c0 < dh; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(tO + c0, o);
+        // P(t-1).V must have finished before O is rescaled or P rewritten.
+        if (t > 0) {
+          if (!mbar_wait(&pv_done[wg], (uint32_t)(t - 1) & 1u, a.err, abort_flag,
+                         WHERE_ATTN_SOFTMAX)) {
+            ok = false;
+            break;
           }
-          tmem_wait_st();
-        }
-        float sum = 0.f;
-        uint32_t pk[32];
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, need)) {
+            for (int c0 = 0; c0 < dh; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(tO + c0, o);
+              tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 64; j += 2) {
-          const float e0 = ex2(fmaf(__uint_as_float(sr[j]), c, -m));
-          const float e1 = ex2(fmaf(__uint_as_float(sr[j + 1]), c, -m));
-          const float p0 = (j < nvalid) ? e0 : 0.f;
-          const float p1 = (j + 1 < nvalid) ? e1 : 0.f;
-          sum += p0 + p1;
-          pk[j >> 1] = pack_bf16x2(p0, p1);
+              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+              tmem_st32(tO + c0, o);
+            }
+            tmem_wait_st();
+          }
         }
-        l += sum;
+        TT_TRACE_POINT(lane == 0 && q == 0, 7 + 5 * wg, t);
+        uint32_t pk[32];
+        l += full ? exp_pack<true>(sr, nvalid, c, m, pk) : exp_pack<false>(sr, nvalid, c, m, pk);
+        TT_TRACE_POINT(lane == 0 && q == 0, 8 + 5 * wg, t);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int phys = j ^ (r & 7);
@@ -349,6 +402,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&p_full[wg]);
+        TT_TRACE_POINT(lane == 0 && q == 0, 9 + 5 * wg, t);
       }
       if (ok && mbar_wait(o_full, 0, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
         tc_fence_after();
@@ -409,6 +463,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // One warp per query row: combine the splits' partials,
 //   O = sum_i 2^(m_i - m*) O_i / sum_i 2^(m_i - m*) l_i.
 __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a) {
+  griddep_launch();
+  griddep_wait();
   if (a.active != nullptr && *a.active == 0) return;
   const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -467,17 +523,13 @@ cudaError_t launch_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKc, const C
       cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.n_splits, a.n_qtiles, a.B * a.Hkv);
-  attn_kernel<<<grid, kAttnThreads, smem, st>>>(tmQ, tmKc, tmVc, tmKb, tmVb, a);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(attn_kernel, grid, dim3(kAttnThreads), smem, st, tmQ, tmKc, tmVc, tmKb, tmVb, a);
 }
 
 cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t st) {
   const long long warps = (long long)a.B * a.Hkv * a.n_qtiles * 256;
   const int blocks = (int)((warps * 32 + 255) / 256);
-  attn_merge_kernel<<<blocks, 256, 0, st>>>(a);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(attn_merge_kernel, dim3(blocks), dim3(256), 0, st, a);
 }
 
 }  // namespace tt

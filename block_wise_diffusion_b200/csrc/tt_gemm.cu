@@ -22,39 +22,45 @@ namespace tt {
 namespace {
 
 constexpr uint32_t kStageA = kGemmBM * kGemmBK * 2;  // 16 KB
-constexpr uint32_t kStageB = kGemmBN * kGemmBK * 2;  // 32 KB
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int EPI>  // 0: vocabulary statistics, 1: bf16 store
+// EPI 0: vocabulary statistics, 1: bf16 store.  BN: tile width (N of the
+// MMA, a multiple of 16 up to 256); STAGES: depth of the TMA ring.
+template <int EPI, int BN, int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs a) {
+  griddep_launch();
+  griddep_wait();
   extern __shared__ uint8_t smem_raw[];
   if (a.active != nullptr && *a.active == 0) return;
   const int M = a.M_dev != nullptr ? min(*a.M_dev, a.M_alloc) : a.M_alloc;
   if (M <= 0) return;
   const int num_m = (M + kGemmBM - 1) / kGemmBM;
-  const int num_n = (a.N + kGemmBN - 1) / kGemmBN;
+  constexpr uint32_t kStageB = BN * kGemmBK * 2;
+  const int num_n = (a.N + BN - 1) / BN;
   const int tiles = num_m * num_n;
-  if ((int)blockIdx.x >= tiles) return;
-  const int kb_n = a.K / kGemmBK;
+  const int ksplit = (EPI == 1 && a.ksplit > 1) ? a.ksplit : 1;
+  const int units = tiles * ksplit;  // work unit = (tile, K range)
+  if ((int)blockIdx.x >= units) return;
+  const int kb_per = (a.K / kGemmBK) / ksplit;
 
   uint8_t* base = align1024(smem_raw);
   uint8_t* sA = base;
-  uint8_t* sB = base + kGemmStages * kStageA;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + kGemmStages * kStageB);
-  uint64_t* empty = full + kGemmStages;
-  uint64_t* accf = empty + kGemmStages;
+  uint8_t* sB = base + STAGES * kStageA;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * kStageB);
+  uint64_t* empty = full + STAGES;
+  uint64_t* accf = empty + STAGES;
   uint64_t* acce = accf + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acce + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kGemmStages; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
@@ -84,9 +90,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+      for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
+        const int tile = u / ksplit;
         const int m = tile % num_m, n = tile / num_m;
-        for (int kb = 0; kb < kb_n; ++kb) {
+        const int kb0 = (u - tile * ksplit) * kb_per;
+        for (int kb = kb0; kb < kb0 + kb_per; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1, a.err, abort_flag, WHERE_GEMM_PRODUCER)) {
             ok = false;
             break;
@@ -94,9 +102,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           mbar_arrive_expect_tx(&full[stage], kStageA + kStageB);
           tma_load_2d_hint(sA + stage * kStageA, &tmA, &full[stage], kb * kGemmBK, m * kGemmBM,
                            pol_a);
-          tma_load_2d_hint(sB + stage * kStageB, &tmB, &full[stage], kb * kGemmBK, n * kGemmBN,
+          tma_load_2d_hint(sB + stage * kStageB, &tmB, &full[stage], kb * kGemmBK, n * BN,
                            num_m == 1 ? pol_b : pol_a);
-          if (++stage == kGemmStages) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
@@ -105,17 +113,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
-    constexpr uint32_t idesc = idesc_bf16(kGemmBM, kGemmBN, false, false);
+    constexpr uint32_t idesc = idesc_bf16(kGemmBM, BN, false, false);
     int stage = 0;
     uint32_t phase = 0;
     int acc = 0;
     uint32_t acc_phase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+    for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
       if (!mbar_wait(&acce[acc], acc_phase ^ 1, a.err, abort_flag, WHERE_GEMM_MMA)) break;
       tc_fence_after();
-      const uint32_t d = tmem + acc * kGemmBN;
-      for (int kb = 0; kb < kb_n; ++kb) {
+      const uint32_t d = tmem + acc * BN;
+      for (int kb = 0; kb < kb_per; ++kb) {
         if (!mbar_wait(&full[stage], phase, a.err, abort_flag, WHERE_GEMM_MMA)) {
           ok = false;
           break;
@@ -132,7 +140,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           umma_commit(&empty[stage]);
         }
         __syncwarp();
-        if (++stage == kGemmStages) {
+        if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
         }
@@ -148,13 +156,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      const int tile = u / ksplit;
       const int m = tile % num_m, n = tile / num_m;
       if (!mbar_wait(&accf[acc], acc_phase, a.err, abort_flag, WHERE_GEMM_EPI)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem + acc * kGemmBN + ((uint32_t)(q * 32) << 16);
+      const uint32_t tbase = tmem + acc * BN + ((uint32_t)(q * 32) << 16);
       const int row = m * kGemmBM + q * 32 + lane;
-      const int ncols = min(kGemmBN, a.N - n * kGemmBN);
+      const int ncols = min(BN, a.N - n * BN);
       const int nchunks = (ncols + 31) >> 5;
       if constexpr (EPI == 0) {
         const float c = a.scale_log2;
@@ -192,19 +201,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce[acc]);
-        if (row < M) {
-          const size_t o = (size_t)n * a.part_ld + row;
-          a.part_v[o] = best;
-          a.part_z[o] = z;
-          a.part_a[o] = n * kGemmBN + bidx;
-        }
-      } else {
+        if (row < M)
+          a.stats[(size_t)row * num_n + n] =
+              make_float4(best, z, __int_as_float(n * BN + bidx), 0.f);
+      } else if (ksplit == 1) {
         for (int ch = 0; ch < nchunks; ++ch) {
           uint32_t r[32];
           tmem_ld32(tbase + ch * 32, r);
           tmem_wait_ld();
           if (row < M) {
-            const int col0 = n * kGemmBN + ch * 32;
+            const int col0 = n * BN + ch * 32;
             uint16_t* dst = a.C + (size_t)row * a.ldc + col0;
             const int lim = ncols - ch * 32;  // multiple of 8 when < 32
 #pragma unroll
@@ -217,6 +223,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 w.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
                 *reinterpret_cast<uint4*>(dst + 8 * v) = w;
               }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acce[acc]);
+      } else {
+        // split-K: store this K range's fp32 partial tile
+        const int ks = u - tile * ksplit;
+        float* prow = a.partial + ((size_t)ks * a.M_alloc + row) * a.N + n * BN;
+        for (int ch = 0; ch < nchunks; ++ch) {
+          uint32_t r[32];
+          tmem_ld32(tbase + ch * 32, r);
+          tmem_wait_ld();
+          if (row < M) {
+            const int lim = ncols - ch * 32;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              if (v * 4 < lim)
+                __stcg(reinterpret_cast<float4*>(prow + ch * 32 + 4 * v),
+                       make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
             }
           }
         }
@@ -237,27 +265,63 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
-template <int EPI>
+__global__ void __launch_bounds__(256)
+    splitk_reduce_kernel(const float* __restrict__ partial, int ksplit, int rows, int N,
+                         uint16_t* __restrict__ C, int ldc, const int* active) {
+  griddep_launch();
+  griddep_wait();
+  if (active != nullptr && *active == 0) return;
+  const int per_row = N / 8;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)rows * per_row) return;
+  const int row = (int)(i / per_row), c8 = (int)(i % per_row) * 8;
+  const size_t plane = (size_t)rows * N;
+  const float* p = partial + (size_t)row * N + c8;
+  float4 x0 = __ldcg(reinterpret_cast<const float4*>(p));
+  float4 x1 = __ldcg(reinterpret_cast<const float4*>(p + 4));
+  for (int k = 1; k < ksplit; ++k) {
+    const float4 y0 = __ldcg(reinterpret_cast<const float4*>(p + k * plane));
+    const float4 y1 = __ldcg(reinterpret_cast<const float4*>(p + k * plane + 4));
+    x0.x += y0.x; x0.y += y0.y; x0.z += y0.z; x0.w += y0.w;
+    x1.x += y1.x; x1.y += y1.y; x1.z += y1.z; x1.w += y1.w;
+  }
+  uint4 w;
+  w.x = pack_bf16x2(x0.x, x0.y);
+  w.y = pack_bf16x2(x0.z, x0.w);
+  w.z = pack_bf16x2(x1.x, x1.y);
+  w.w = pack_bf16x2(x1.z, x1.w);
+  *reinterpret_cast<uint4*>(C + (size_t)row * ldc + c8) = w;
+}
+
+template <int EPI, int BN, int STAGES>
 cudaError_t launch_gemm(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
                         int grid, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kGemmSmemBytes);
+  constexpr size_t smem = gemm_smem_bytes(BN, STAGES);
+  static_assert(smem <= 232448, "shared memory per CTA");
+  static_assert(2 * BN <= 512, "two accumulators must fit TMEM");
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<EPI, BN, STAGES>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  gemm_kernel<EPI><<<grid, kGemmThreads, kGemmSmemBytes, st>>>(tmA, tmB, a);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(gemm_kernel<EPI, BN, STAGES>, dim3(grid), dim3(kGemmThreads), smem, st, tmA,
+                  tmB, a);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_vocab(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
                               int grid, cudaStream_t st) {
-  return launch_gemm<0>(tmA, tmB, a, grid, st);
+  return launch_gemm<0, kVocabBN, kVocabStages>(tmA, tmB, a, grid, st);
 }
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
                              int grid, cudaStream_t st) {
-  return launch_gemm<1>(tmA, tmB, a, grid, st);
+  return launch_gemm<1, kQkvBN, kQkvStages>(tmA, tmB, a, grid, st);
+}
+
+cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int N, uint16_t* C,
+                                 int ldc, const int* active, cudaStream_t st) {
+  const long long threads = (long long)rows * (N / 8);
+  return launch_k(splitk_reduce_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st,
+                  partial, ksplit, rows, N, C, ldc, active);
 }
 
 }  // namespace tt

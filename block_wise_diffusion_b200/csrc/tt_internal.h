@@ -19,6 +19,7 @@ enum CtrlWord {
   CTRL_M = 3,          // masked rows of the current step (vocab GEMM rows)
   CTRL_ACTIVE = 4,     // 1 while the loop still has masked positions
   CTRL_STEPS_RUN = 5,  // loop steps that did work
+  CTRL_DONE = 6,       // commit CTAs finished in this step (last one plans the next)
   CTRL_WORDS = 64
 };
 constexpr size_t kCtrlBytes = CTRL_WORDS * sizeof(int);
@@ -39,25 +40,34 @@ enum WhereTag {
 // C = A[M, K] . B[N, K]^T with both operands K-major bf16.  BM=128, BN=256,
 // BK=64.  Two epilogues: vocabulary statistics (per row and 256-wide column
 // tile: max logit, sum of exp relative to it, argmax) or a plain bf16 store.
-constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
+// Tile widths: the vocabulary GEMM uses N tiles of 224 columns (131072
+// columns -> 586 tiles, 3.96 per SM, so the last round is nearly full) with
+// a 5-deep ring; the linear update uses 256-column tiles with a 4-deep ring.
+constexpr int kGemmBM = 128, kGemmBK = 64;
+constexpr int kVocabBN = 224, kVocabStages = 5;
+constexpr int kQkvBN = 256, kQkvStages = 4;
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
-constexpr size_t kGemmStageBytes = (kGemmBM + kGemmBN) * kGemmBK * 2;
-constexpr size_t kGemmSmemBytes = kGemmStages * kGemmStageBytes + 1024 + 256;
+constexpr size_t gemm_smem_bytes(int bn, int stages) {
+  return (size_t)stages * (kGemmBM + bn) * kGemmBK * 2 + 1024 + 256;
+}
 
 struct GemmArgs {
   int M_alloc;          // rows present in A's tensor map
   const int* M_dev;     // device row count (nullptr: M_alloc); rows >= M are ignored
   const int* active;    // optional device flag: kernel returns at once if *active == 0
   int N, K;             // N: columns of C (any multiple of 8); K multiple of 64
-  // vocabulary-statistics epilogue
-  float* part_v;        // [n_tiles_n][part_ld] max raw logit of the tile
-  float* part_z;        // [n_tiles_n][part_ld] sum exp2(l*c - max*c)
-  int* part_a;          // [n_tiles_n][part_ld] argmax column (lowest on ties)
-  int part_ld;
+  // vocabulary-statistics epilogue: stats[row * n_tiles_n + tile] =
+  //   {max raw logit, sum exp2(l*c - max*c), argmax column (int bits), 0}
+  float4* stats;        // [row][ceil(N / kVocabBN)]
   float scale_log2;     // c = logit_scale * log2(e)
   // bf16 epilogue
   uint16_t* C;
   int ldc;
+  // split-K (bf16 epilogue only): K is cut into ksplit ranges handled by
+  // different CTAs, each storing its fp32 partial tile to
+  // partial[ks][M_alloc][N]; splitk_reduce sums them into C.
+  int ksplit;
+  float* partial;
   int* err;             // control block
 };
 
@@ -65,6 +75,9 @@ cudaError_t launch_gemm_vocab(const CUtensorMap& tmA, const CUtensorMap& tmB, co
                               int grid, cudaStream_t st);
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
                              int grid, cudaStream_t st);
+// C[r, :] = bf16(sum_k partial[k][r][:]) for r < rows (N multiple of 8).
+cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int N, uint16_t* C,
+                                 int ldc, const int* active, cudaStream_t st);
 
 // ------------------------------------------------------------- attention
 constexpr int kAttnBN = 64;        // keys per tile
@@ -101,13 +114,18 @@ struct PlanArgs {
   int* rowlist;     // [B*S] compact list of masked rows (b*S+s)
   float* t;         // [B]   masked fraction at the start of the step
   int* ctrl;        // writes CTRL_M, CTRL_REMAINING, CTRL_ACTIVE, CTRL_STEPS_RUN
-  int count_step;   // 1: bump CTRL_STEPS_RUN when active
+  int count_step;   // unused (kept for layout); steps are counted by the commit kernel
 };
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st);
 
 cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
                          uint16_t* y, int rows, int S, int H, const int* rowlist,
                          const int* M_dev, const int* active, cudaStream_t st);
+
+// Split merge + adaLN for the masked rows of the loop (attention split > 1).
+cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, const float* t,
+                               uint16_t* y, const int* rowlist, const int* M_dev, int max_rows,
+                               cudaStream_t st);
 
 cudaError_t launch_gather_rows(const uint16_t* src, int ld_src, uint16_t* dst, int H,
                                const int* rowlist, const int* M_dev, int max_rows,
@@ -118,10 +136,8 @@ cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_
                          const int* active, int* err, cudaStream_t st);
 
 struct CommitArgs {
-  int B, S, n_vt, part_ld;
-  const float* part_v;
-  const float* part_z;
-  const int* part_a;
+  int B, S, n_vt;
+  const float4* stats;  // [compact row][n_vt] tile statistics of the vocab GEMM
   float scale_log2;
   float gamma;
   const int* rowlist;   // compact row -> b*S+s
@@ -136,6 +152,13 @@ struct CommitArgs {
   int step;
   const int* active;
   int* ctrl;
+  // loop only: re-embedding of newly committed positions and next-step plan
+  const uint16_t* emb;  // [V, H]
+  uint16_t* egath;      // [B*S, H] or nullptr
+  int H;
+  int plan_next;        // 1: the last CTA plans the next step into plan_rowlist / plan_t
+  int* plan_rowlist;
+  float* plan_t;
 };
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 
@@ -157,6 +180,28 @@ void count_launch(int n = 1);
 tt_status set_error(tt_status s, const char* msg);
 // The shape checks of the public entry points.
 tt_status check_dims_public(const tt_dims* d);
+
+// Launch with programmatic dependent launch allowed: the kernel may be
+// scheduled while its predecessor in the stream is still finishing; every
+// kernel of this library executes griddepcontrol.wait before it reads
+// anything a predecessor wrote, so only launch latency is overlapped.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  count_launch();
+  return e;
+}
 
 // Profiler hooks (no-ops unless tt_profile_enable(1)): bracket one launch.
 void prof_begin(int kind, cudaStream_t st);

@@ -70,15 +70,13 @@ extern "C" tt_status tt_vocab_confidence_commit_noalloc(
 
   // Scratch layout, checked against the built-in maximum before any launch.
   const size_t rows = (size_t)d->B * d->S;
-  const size_t n_vt = (size_t)(d->V + kGemmBN - 1) / kGemmBN;
+  const size_t n_vt = (size_t)(d->V + kVocabBN - 1) / kVocabBN;
   size_t off = 0;
   const size_t o_ctrl = off;    off = up256(off + kCtrlBytes);
   const size_t o_rows = off;    off = up256(off + rows * sizeof(int));
   const size_t o_t = off;       off = up256(off + (size_t)d->B * sizeof(float));
   const size_t o_yc = off;      off = up256(off + rows * (size_t)d->H * 2);
-  const size_t o_pv = off;      off = up256(off + n_vt * rows * sizeof(float));
-  const size_t o_pz = off;      off = up256(off + n_vt * rows * sizeof(float));
-  const size_t o_pa = off;      off = up256(off + n_vt * rows * sizeof(int));
+  const size_t o_st = off;      off = up256(off + n_vt * rows * sizeof(float4));
   if (off > kNoAllocScratchBytes) {
     char msg[200];
     snprintf(msg, sizeof msg,
@@ -96,9 +94,7 @@ extern "C" tt_status tt_vocab_confidence_commit_noalloc(
   int* rowlist = reinterpret_cast<int*>(sb + o_rows);
   float* tvec = reinterpret_cast<float*>(sb + o_t);
   uint16_t* y_c = reinterpret_cast<uint16_t*>(sb + o_yc);
-  float* part_v = reinterpret_cast<float*>(sb + o_pv);
-  float* part_z = reinterpret_cast<float*>(sb + o_pz);
-  int* part_a = reinterpret_cast<int*>(sb + o_pa);
+  float4* stats = reinterpret_cast<float4*>(sb + o_st);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
   // The array keeps the previous call's contents: the control block (row
@@ -115,17 +111,14 @@ extern "C" tt_status tt_vocab_confidence_commit_noalloc(
 
   CUtensorMap tmA, tmB;
   if (!make_tmap_2d(&tmA, y_c, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM) ||
-      !make_tmap_2d(&tmB, w, d->H, d->V, (uint64_t)d->H * 2, kGemmBK, kGemmBN))
+      !make_tmap_2d(&tmB, w, d->H, d->V, (uint64_t)d->H * 2, kGemmBK, kVocabBN))
     return set_error(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the vocab GEMM");
   GemmArgs g{};
   g.M_alloc = (int)rows;
   g.M_dev = ctrl + CTRL_M;
   g.N = d->V;
   g.K = d->H;
-  g.part_v = part_v;
-  g.part_z = part_z;
-  g.part_a = part_a;
-  g.part_ld = (int)rows;
+  g.stats = stats;
   g.scale_log2 = (float)(logit_scale * 1.4426950408889634);
   g.err = ctrl;
   const int tiles = (int)(((rows + kGemmBM - 1) / kGemmBM) * n_vt);
@@ -136,10 +129,7 @@ extern "C" tt_status tt_vocab_confidence_commit_noalloc(
   c.B = d->B;
   c.S = d->S;
   c.n_vt = (int)n_vt;
-  c.part_ld = (int)rows;
-  c.part_v = part_v;
-  c.part_z = part_z;
-  c.part_a = part_a;
+  c.stats = stats;
   c.scale_log2 = g.scale_log2;
   c.gamma = gamma;
   c.rowlist = rowlist;

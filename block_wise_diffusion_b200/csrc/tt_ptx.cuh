@@ -23,6 +23,15 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// ---------------------------------------------- programmatic dependent launch
+// Let the next kernel in the stream be scheduled now.
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the preceding kernel has completed and its writes are visible
+// (a no-op when the kernel was launched without the dependent-launch attribute).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
@@ -57,8 +66,10 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
                                                    volatile int* abort_flag, int where) {
   const uint64_t t0 = global_ns();
   for (uint32_t i = 0;; ++i) {
-    if (*abort_flag) return false;
+    // A completed phase wins over the abort flag, so threads waiting on the
+    // same phase all see the same outcome.
     if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
     if ((i & 255u) == 255u && global_ns() - t0 > kWaitLimitNs) {
       if (err) {
         atomicCAS(err, 0, (int)TT_ERR_TIMEOUT);
@@ -216,6 +227,11 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Barrier among `count` threads of the CTA on hardware barrier `id` (id > 0).
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // ------------------------------------------------------------ arithmetic

@@ -12,23 +12,27 @@ namespace {
 
 // ------------------------------------------------------------------ plan
 // Compact list of masked rows (b*S + s) in row order, the per-sequence
-// timestep t_b = masked count / S, and the step's control words.
-__global__ void __launch_bounds__(1024) plan_kernel(const PlanArgs a) {
+// timestep t_b = masked count / S, and the step's control words, computed by
+// one CTA of any size (a multiple of 32 threads).  `masked` is read through
+// volatile loads: in the commit kernel it was just written by other CTAs.
+__device__ void plan_block(const PlanArgs& a) {
   __shared__ int warp_tot[32];
   __shared__ int running;
+  const volatile uint8_t* masked = a.masked;
   const int n = a.B * a.S;
+  const int nt = blockDim.x, nw = nt >> 5;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) running = 0;
   __syncthreads();
-  for (int base = 0; base < n; base += 1024) {
+  for (int base = 0; base < n; base += nt) {
     const int i = base + tid;
-    const int f = (i < n && a.masked[i] != 0) ? 1 : 0;
+    const int f = (i < n && masked[i] != 0) ? 1 : 0;
     const unsigned bal = __ballot_sync(0xffffffffu, f);
     const int before_in_warp = __popc(bal & ((1u << lane) - 1u));
     if (lane == 0) warp_tot[warp] = __popc(bal);
     __syncthreads();
     int before_warps = 0, total = 0;
-    for (int w = 0; w < 32; ++w) {
+    for (int w = 0; w < nw; ++w) {
       const int c = warp_tot[w];
       before_warps += (w < warp) ? c : 0;
       total += c;
@@ -38,9 +42,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const PlanArgs a) {
     if (tid == 0) running += total;
     __syncthreads();
   }
-  for (int b = tid; b < a.B; b += 1024) {
+  for (int b = tid; b < a.B; b += nt) {
     int c = 0;
-    for (int s = 0; s < a.S; ++s) c += a.masked[b * a.S + s] != 0;
+    for (int s = 0; s < a.S; ++s) c += masked[b * a.S + s] != 0;
     a.t[b] = (float)c / (float)a.S;
   }
   if (tid == 0) {
@@ -48,8 +52,13 @@ __global__ void __launch_bounds__(1024) plan_kernel(const PlanArgs a) {
     a.ctrl[CTRL_M] = M;
     a.ctrl[CTRL_REMAINING] = M;
     a.ctrl[CTRL_ACTIVE] = M > 0 ? 1 : 0;
-    if (a.count_step && M > 0) a.ctrl[CTRL_STEPS_RUN] += 1;
   }
+}
+
+__global__ void __launch_bounds__(1024) plan_kernel(const PlanArgs a) {
+  griddep_launch();
+  griddep_wait();
+  plan_block(a);
 }
 
 // ----------------------------------------------------------------- adaLN
@@ -69,10 +78,67 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return s;
 }
 
+// LayerNorm of the row held in v (8 values per vector, vectors threadIdx.x +
+// k*kAdaThreads) followed by the time modulation; writes the bf16 row yr.
+__device__ __forceinline__ void adaln_finish(float (&v)[kAdaMaxVec][8], float s, int H, float tb,
+                                             const uint16_t* __restrict__ ss,
+                                             uint16_t* __restrict__ yrow, float* red) {
+  const int nvec = H / 8;
+  const float mean = block_sum(s, red) / (float)H;
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < kAdaMaxVec; ++k) {
+    const int vi = threadIdx.x + k * kAdaThreads;
+    if (vi < nvec) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float d = v[k][e] - mean;
+        q += d * d;
+      }
+    }
+  }
+  const float var = block_sum(q, red) / (float)H;
+  const float rstd = rsqrtf(var + 1e-6f);
+  const float lw = -13.287712379549449f / (float)H;  // -log2(10000) / H
+  uint4* yr = reinterpret_cast<uint4*>(yrow);
+  const uint4* e0 = reinterpret_cast<const uint4*>(ss);
+  const uint4* e1 = reinterpret_cast<const uint4*>(ss + H);
+#pragma unroll
+  for (int k = 0; k < kAdaMaxVec; ++k) {
+    const int vi = threadIdx.x + k * kAdaThreads;
+    if (vi < nvec) {
+      const uint4 a0 = e0[vi], a1 = e1[vi];
+      const uint32_t sh[4] = {a0.x, a0.y, a0.z, a0.w};
+      const uint32_t sc[4] = {a1.x, a1.y, a1.z, a1.w};
+      float out[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int i = vi * 8 + e;
+        const float w = ex2((float)i * lw);
+        float sn, cs;
+        __sincosf(tb * w, &sn, &cs);  // |t w| <= 1: abs error ~1e-6, far below bf16 output
+        const uint32_t hs = (e & 1) ? (sh[e >> 1] & 0xffff0000u) : (sh[e >> 1] << 16);
+        const uint32_t hc = (e & 1) ? (sc[e >> 1] & 0xffff0000u) : (sc[e >> 1] << 16);
+        const float shift = __uint_as_float(hs) + sn;
+        const float scale = __uint_as_float(hc) + cs;
+        out[e] = (v[k][e] - mean) * rstd * (1.f + scale) + shift;
+      }
+      uint4 o;
+      o.x = pack_bf16x2(out[0], out[1]);
+      o.y = pack_bf16x2(out[2], out[3]);
+      o.z = pack_bf16x2(out[4], out[5]);
+      o.w = pack_bf16x2(out[6], out[7]);
+      yr[vi] = o;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kAdaThreads)
     adaln_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ ss,
                  const float* __restrict__ t, uint16_t* __restrict__ y, int rows, int S, int H,
                  const int* __restrict__ rowlist, const int* M_dev, const int* active) {
+  griddep_launch();
+  griddep_wait();
   __shared__ float red[kAdaThreads / 32];
   if (active != nullptr && *active == 0) return;
   const int M = M_dev != nullptr ? *M_dev : rows;
@@ -99,53 +165,69 @@ __global__ void __launch_bounds__(kAdaThreads)
       for (int e = 0; e < 8; ++e) s += v[k][e];
     }
   }
-  const float mean = block_sum(s, red) / (float)H;
-  float q = 0.f;
+  adaln_finish(v, s, H, tb, ss, y + (size_t)j * H, red);
+}
+
+// Attention split merge fused with adaLN (block loop): one CTA per masked
+// row (b, s).  For each query head the split partials are combined,
+//   o = sum_i 2^(m_i - m*) O_i / sum_i 2^(m_i - m*) l_i,
+// rounded to bf16 (the attention output's storage precision), and the whole
+// row then goes through adaln_finish.
+__global__ void __launch_bounds__(kAdaThreads)
+    merge_adaln_kernel(const AttnArgs a, const uint16_t* __restrict__ ss,
+                       const float* __restrict__ t, uint16_t* __restrict__ y,
+                       const int* __restrict__ rowlist, const int* M_dev) {
+  griddep_launch();
+  griddep_wait();
+  __shared__ float red[kAdaThreads / 32];
+  if (a.active != nullptr && *a.active == 0) return;
+  const int j = blockIdx.x;
+  if (j >= *M_dev) return;
+  const int row = rowlist[j];
+  const int b = row / a.S, s = row % a.S;
+  const int H = a.Hq * a.dh;
+  const int sq = a.halves * a.s_per_half;
+  const int qt = s / sq, within = s % sq;
+  const int hh = within / a.s_per_half, sl = within % a.s_per_half;
+  const float tb = t[b];
+  const int nvec = H / 8;
+  float v[kAdaMaxVec][8];
+  float sum = 0.f;
 #pragma unroll
   for (int k = 0; k < kAdaMaxVec; ++k) {
     const int vi = threadIdx.x + k * kAdaThreads;
     if (vi < nvec) {
+      const int e0 = vi * 8, head = e0 / a.dh, d0 = e0 % a.dh;
+      const int g = head / a.G, jh = head % a.G;
+      const size_t unit0 = (size_t)((b * a.Hkv + g) * a.n_qtiles + qt) * a.n_splits;
+      const int r256 = hh * 128 + sl * a.G + jh;
+      float mstar = -INFINITY;
+      for (int sp = 0; sp < a.n_splits; ++sp) {
+        const size_t pr = (unit0 + sp) * 256 + r256;
+        if (a.part_ml[pr * 2 + 1] > 0.f) mstar = fmaxf(mstar, a.part_ml[pr * 2]);
+      }
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float den = 0.f;
+      for (int sp = 0; sp < a.n_splits; ++sp) {
+        const size_t pr = (unit0 + sp) * 256 + r256;
+        const float ls = a.part_ml[pr * 2 + 1];
+        if (!(ls > 0.f)) continue;
+        const float w = ex2(a.part_ml[pr * 2] - mstar);
+        den += w * ls;
+        const float4* po = reinterpret_cast<const float4*>(a.part_o + pr * a.dh + d0);
+        const float4 x0 = po[0], x1 = po[1];
+        acc[0] += w * x0.x; acc[1] += w * x0.y; acc[2] += w * x0.z; acc[3] += w * x0.w;
+        acc[4] += w * x1.x; acc[5] += w * x1.y; acc[6] += w * x1.z; acc[7] += w * x1.w;
+      }
+      const float inv = 1.f / den;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float d = v[k][e] - mean;
-        q += d * d;
+        v[k][e] = __uint_as_float(pack_bf16x2(acc[e] * inv, 0.f) << 16);
+        sum += v[k][e];
       }
     }
   }
-  const float var = block_sum(q, red) / (float)H;
-  const float rstd = rsqrtf(var + 1e-6f);
-  const float lw = -13.287712379549449f / (float)H;  // -log2(10000) / H
-  uint4* yr = reinterpret_cast<uint4*>(y + (size_t)j * H);
-  const uint4* e0 = reinterpret_cast<const uint4*>(ss);
-  const uint4* e1 = reinterpret_cast<const uint4*>(ss + H);
-#pragma unroll
-  for (int k = 0; k < kAdaMaxVec; ++k) {
-    const int vi = threadIdx.x + k * kAdaThreads;
-    if (vi < nvec) {
-      const uint4 a0 = e0[vi], a1 = e1[vi];
-      const uint32_t sh[4] = {a0.x, a0.y, a0.z, a0.w};
-      const uint32_t sc[4] = {a1.x, a1.y, a1.z, a1.w};
-      float out[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int i = vi * 8 + e;
-        const float w = exp2f((float)i * lw);
-        float sn, cs;
-        sincosf(tb * w, &sn, &cs);
-        const uint32_t hs = (e & 1) ? (sh[e >> 1] & 0xffff0000u) : (sh[e >> 1] << 16);
-        const uint32_t hc = (e & 1) ? (sc[e >> 1] & 0xffff0000u) : (sc[e >> 1] << 16);
-        const float shift = __uint_as_float(hs) + sn;
-        const float scale = __uint_as_float(hc) + cs;
-        out[e] = (v[k][e] - mean) * rstd * (1.f + scale) + shift;
-      }
-      uint4 o;
-      o.x = pack_bf16x2(out[0], out[1]);
-      o.y = pack_bf16x2(out[2], out[3]);
-      o.z = pack_bf16x2(out[4], out[5]);
-      o.w = pack_bf16x2(out[6], out[7]);
-      yr[vi] = o;
-    }
-  }
+  adaln_finish(v, sum, H, tb, ss, y + (size_t)j * H, red);
 }
 
 // ---------------------------------------------------------------- gathers
@@ -153,6 +235,8 @@ __global__ void __launch_bounds__(256)
     gather_rows_kernel(const uint16_t* __restrict__ src, int ld_src, uint16_t* __restrict__ dst,
                        int H, const int* __restrict__ rowlist, const int* M_dev, int max_rows,
                        const int* active) {
+  griddep_launch();
+  griddep_wait();
   if (active != nullptr && *active == 0) return;
   const int M = M_dev != nullptr ? min(*M_dev, max_rows) : max_rows;
   const int j = blockIdx.x;
@@ -169,6 +253,8 @@ __global__ void __launch_bounds__(256)
                  const uint16_t* __restrict__ emb, const uint16_t* __restrict__ e_mask,
                  uint16_t* __restrict__ dst, int rows, int H, int V, const int* active,
                  int* err) {
+  griddep_launch();
+  griddep_wait();
   if (active != nullptr && *active == 0) return;
   const int row = blockIdx.x;
   if (row >= rows) return;
@@ -194,9 +280,13 @@ __global__ void __launch_bounds__(256)
 // tile with the largest v_t (lowest tile on ties, hence lowest id);
 // then warp 0 applies the commit rule across the block.
 __global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
+  griddep_launch();
+  griddep_wait();
   __shared__ float s_conf[32];
   __shared__ int s_tok[32];
   __shared__ int s_mask[32];
+  __shared__ int s_com[32];
+  __shared__ int s_last;
   if (a.active != nullptr && *a.active == 0) return;
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -220,11 +310,13 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
         if (v < row) lo = mid + 1; else hi = mid - 1;
       }
       if (j >= 0) {
+        // tiles of row j are contiguous: lane t reads tiles t, t+32, ...
+        const float4* st = a.stats + (size_t)j * a.n_vt;
         float bv = -INFINITY;
         int bt = 0x7fffffff;
         for (int t = lane; t < a.n_vt; t += 32) {
-          const float v = a.part_v[(size_t)t * a.part_ld + j];
-          if (v > bv || (v == bv && t < bt)) {
+          const float v = st[t].x;
+          if (v > bv) {  // t increases per lane, so ties keep the lowest tile
             bv = v;
             bt = t;
           }
@@ -240,12 +332,12 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
         const float mstar = bv * a.scale_log2;
         float Z = 0.f;
         for (int t = lane; t < a.n_vt; t += 32) {
-          const size_t o = (size_t)t * a.part_ld + j;
-          Z += a.part_z[o] * ex2(a.part_v[o] * a.scale_log2 - mstar);
+          const float4 q = st[t];
+          Z += q.y * ex2(q.x * a.scale_log2 - mstar);
         }
         for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
         conf = 1.f / Z;
-        tok = (bt < a.n_vt) ? a.part_a[(size_t)bt * a.part_ld + j] : -1;
+        tok = (bt < a.n_vt) ? __float_as_int(st[bt].z) : -1;
       }
     }
     if (lane == 0) {
@@ -255,54 +347,80 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
     }
   }
   __syncthreads();
-  if (warp != 0) return;
-  const int s = lane;
-  const bool in = s < S;
-  const int row = b * S + s;
-  const int is_m = in ? s_mask[s] : 0;
-  float cf = in ? s_conf[s] : -1.f;
-  const int tok = in ? s_tok[s] : -1;
-  const bool bad = is_m && !(cf >= 0.f && cf <= 1.0001f);  // NaN or impossible value
-  if (__any_sync(0xffffffffu, bad) && lane == 0) {
-    atomicCAS(a.ctrl + CTRL_ERR, 0, (int)TT_ERR_INTERNAL);
-    atomicCAS(a.ctrl + CTRL_ERR_WHERE, 0, (int)WHERE_COMMIT_NAN);
-  }
-  if (bad) cf = -1.f;
-  const bool qual = is_m && cf >= a.gamma && tok >= 0;
-  const unsigned qmask = __ballot_sync(0xffffffffu, qual);
-  const unsigned mmask = __ballot_sync(0xffffffffu, is_m != 0);
-  bool commit = qual;
-  if (qmask == 0 && mmask != 0) {
-    // fallback: the most confident masked position, lowest s on ties
-    float bc = is_m ? cf : -INFINITY;
-    int bs = is_m ? s : 0x7fffffff;
-    for (int o = 16; o > 0; o >>= 1) {
-      const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
-      const int os = __shfl_xor_sync(0xffffffffu, bs, o);
-      if (oc > bc || (oc == bc && os < bs)) {
-        bc = oc;
-        bs = os;
+  if (warp == 0) {
+    const int s = lane;
+    const bool in = s < S;
+    const int row = b * S + s;
+    const int is_m = in ? s_mask[s] : 0;
+    float cf = in ? s_conf[s] : -1.f;
+    const int tok = in ? s_tok[s] : -1;
+    const bool bad = is_m && !(cf >= 0.f && cf <= 1.0001f);  // NaN or impossible value
+    if (__any_sync(0xffffffffu, bad) && lane == 0) {
+      atomicCAS(a.ctrl + CTRL_ERR, 0, (int)TT_ERR_INTERNAL);
+      atomicCAS(a.ctrl + CTRL_ERR_WHERE, 0, (int)WHERE_COMMIT_NAN);
+    }
+    if (bad) cf = -1.f;
+    const bool qual = is_m && cf >= a.gamma && tok >= 0;
+    const unsigned qmask = __ballot_sync(0xffffffffu, qual);
+    const unsigned mmask = __ballot_sync(0xffffffffu, is_m != 0);
+    bool commit = qual;
+    if (qmask == 0 && mmask != 0) {
+      // fallback: the most confident masked position, lowest s on ties
+      float bc = is_m ? cf : -INFINITY;
+      int bs = is_m ? s : 0x7fffffff;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float oc = __shfl_xor_sync(0xffffffffu, bc, o);
+        const int os = __shfl_xor_sync(0xffffffffu, bs, o);
+        if (oc > bc || (oc == bc && os < bs)) {
+          bc = oc;
+          bs = os;
+        }
       }
+      commit = is_m && s == bs;
     }
-    commit = is_m && s == bs;
-  }
-  if (in) {
-    if (commit) {
-      a.tokens[row] = tok >= 0 ? tok : 0;
-      a.masked[row] = 0;
-      if (a.commit_step != nullptr) a.commit_step[row] = a.step;
+    if (in) {
+      s_com[s] = commit ? 1 : 0;
+      if (commit) {
+        s_tok[s] = tok >= 0 ? tok : 0;
+        a.tokens[row] = s_tok[s];
+        a.masked[row] = 0;
+        if (a.commit_step != nullptr) a.commit_step[row] = a.step;
+      }
+      if (a.conf_out != nullptr) a.conf_out[row] = is_m ? s_conf[s] : -1.f;
+      if (a.argmax_out != nullptr) a.argmax_out[row] = is_m ? tok : -1;
     }
-    if (a.conf_out != nullptr) a.conf_out[row] = is_m ? s_conf[s] : -1.f;
-    if (a.argmax_out != nullptr) a.argmax_out[row] = is_m ? tok : -1;
+    const unsigned cmask = __ballot_sync(0xffffffffu, commit);
+    if (lane == 0) {
+      if (a.n_committed != nullptr) a.n_committed[b] = __popc(cmask);
+      if (a.steps_taken != nullptr && mmask != 0) a.steps_taken[b] = a.step + 1;
+    }
   }
-  const unsigned cmask = __ballot_sync(0xffffffffu, commit);
-  if (lane == 0) {
-    if (a.n_committed != nullptr) a.n_committed[b] = __popc(cmask);
-    if (a.steps_taken != nullptr && mmask != 0) a.steps_taken[b] = a.step + 1;
+  __syncthreads();
+  // Loop only: a newly committed position's next embedding is Emb[token].
+  if (a.egath != nullptr && warp < S && s_com[warp]) {
+    const uint4* src = reinterpret_cast<const uint4*>(a.emb + (size_t)s_tok[warp] * a.H);
+    uint4* dst = reinterpret_cast<uint4*>(a.egath + (size_t)(b * S + warp) * a.H);
+    for (int i = lane; i < a.H / 8; i += 32) dst[i] = src[i];
+  }
+  if (!a.plan_next) return;
+  // The last CTA to finish plans the next step (no CTA ever waits for another).
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = atomicAdd(a.ctrl + CTRL_DONE, 1) == a.B - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  PlanArgs p{a.B, S, a.masked, a.plan_rowlist, a.plan_t, a.ctrl, 0};
+  plan_block(p);
+  if (threadIdx.x == 0) {
+    a.ctrl[CTRL_DONE] = 0;
+    a.ctrl[CTRL_STEPS_RUN] += 1;
   }
 }
 
 __global__ void loop_init_kernel(int B, int S, int* steps_taken, int* commit_step) {
+  griddep_launch();
+  griddep_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < B) steps_taken[i] = 0;
   if (i < B * S) commit_step[i] = -1;
@@ -311,53 +429,51 @@ __global__ void loop_init_kernel(int B, int S, int* steps_taken, int* commit_ste
 }  // namespace
 
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st) {
-  plan_kernel<<<1, 1024, 0, st>>>(a);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(plan_kernel, dim3(1), dim3(1024), 0, st, a);
 }
 
 cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
                          uint16_t* y, int rows, int S, int H, const int* rowlist,
                          const int* M_dev, const int* active, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  adaln_kernel<<<rows, kAdaThreads, 0, st>>>(x, shift_scale, t, y, rows, S, H, rowlist, M_dev,
-                                             active);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(adaln_kernel, dim3(rows), dim3(kAdaThreads), 0, st, x, shift_scale, t, y, rows,
+                  S, H, rowlist, M_dev, active);
+}
+
+cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, const float* t,
+                               uint16_t* y, const int* rowlist, const int* M_dev, int max_rows,
+                               cudaStream_t st) {
+  if (max_rows <= 0) return cudaSuccess;
+  return launch_k(merge_adaln_kernel, dim3(max_rows), dim3(kAdaThreads), 0, st, a, shift_scale, t,
+                  y, rowlist, M_dev);
 }
 
 cudaError_t launch_gather_rows(const uint16_t* src, int ld_src, uint16_t* dst, int H,
                                const int* rowlist, const int* M_dev, int max_rows,
                                const int* active, cudaStream_t st) {
   if (max_rows <= 0) return cudaSuccess;
-  gather_rows_kernel<<<max_rows, 256, 0, st>>>(src, ld_src, dst, H, rowlist, M_dev, max_rows,
-                                               active);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(gather_rows_kernel, dim3(max_rows), dim3(256), 0, st, src, ld_src, dst, H,
+                  rowlist, M_dev, max_rows, active);
 }
 
 cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_t* emb,
                          const uint16_t* e_mask, uint16_t* dst, int rows, int H, int V,
                          const int* active, int* err, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  embed_kernel<<<rows, 256, 0, st>>>(tokens, masked, emb, e_mask, dst, rows, H, V, active, err);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(embed_kernel, dim3(rows), dim3(256), 0, st, tokens, masked, emb, e_mask, dst,
+                  rows, H, V, active, err);
 }
 
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
-  commit_kernel<<<a.B, a.S * 32, 0, st>>>(a);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(commit_kernel, dim3(a.B), dim3(a.S * 32), 0, st, a);
 }
 
 cudaError_t launch_loop_init(int B, int S, int* steps_taken, int* commit_step, int* ctrl,
                              cudaStream_t st) {
   (void)ctrl;
   const int n = B * S;
-  loop_init_kernel<<<(n + 255) / 256, 256, 0, st>>>(B, S, steps_taken, commit_step);
-  count_launch();
-  return cudaGetLastError();
+  return launch_k(loop_init_kernel, dim3((n + 255) / 256), dim3(256), 0, st, B, S, steps_taken,
+                  commit_step);
 }
 
 }  // namespace tt
