@@ -17,6 +17,7 @@ __all__ = [
     "tt_block_denoise_attn", "tt_adaln_modulate", "tt_vocab_confidence_commit",
     "tt_denoise_block_loop", "tt_vocab_confidence_commit_noalloc", "tt_device_status", "tt_launch_count", "tt_set_attn_splits",
     "tt_status_string", "tt_last_error", "EXPORTS", "tt_profile_enable", "tt_profile_read",
+    "tt_selftest_timeout",
     "profile_table", "KERNEL_KINDS",
     "TT_WS_ATTN", "TT_WS_ADALN", "TT_WS_VOCAB", "TT_WS_LOOP",
 ]
@@ -33,10 +34,10 @@ EXPORTS = (
     "tt_status_string", "tt_last_error", "tt_workspace_bytes", "tt_device_status",
     "tt_launch_count", "tt_set_attn_splits", "tt_block_denoise_attn", "tt_adaln_modulate",
     "tt_vocab_confidence_commit", "tt_denoise_block_loop", "tt_profile_enable", "tt_profile_read",
-    "tt_vocab_confidence_commit_noalloc",
+    "tt_vocab_confidence_commit_noalloc", "tt_selftest_timeout",
 )
 KERNEL_KINDS = ("plan", "embed", "gemm_qkv", "attn", "merge", "adaln", "gemm_vocab", "commit",
-                "gather", "init")
+                "gather", "init", "splitk_reduce")
 
 
 class TTError(RuntimeError):
@@ -69,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.tt_workspace_bytes.argtypes = [ctypes.POINTER(Dims), ctypes.c_int]
         L.tt_device_status.restype = ctypes.c_int
         L.tt_device_status.argtypes = [_P, _P]
+        L.tt_selftest_timeout.restype = ctypes.c_int
+        L.tt_selftest_timeout.argtypes = [_P, ctypes.c_int32, _P]
         L.tt_launch_count.restype = ctypes.c_uint64
         L.tt_launch_count.argtypes = []
         L.tt_set_attn_splits.restype = ctypes.c_int
@@ -175,6 +178,12 @@ def workspace(d: Dims, which: int, device="cuda"):
     """A torch uint8 device buffer of tt_workspace_bytes(d, which) bytes."""
     import torch
     return torch.empty(tt_workspace_bytes(d, which), dtype=torch.uint8, device=device)
+
+
+def tt_selftest_timeout(ws, limit_us: int, stream=None) -> None:
+    """Make one bounded device wait run out on purpose (see the header)."""
+    _check(lib().tt_selftest_timeout(_ptr(ws), int(limit_us), _stream(stream)),
+           "tt_selftest_timeout")
 
 
 def tt_device_status(ws, stream=None) -> int:

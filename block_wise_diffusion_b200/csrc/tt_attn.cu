@@ -6,21 +6,28 @@
 // one softmax over [context keys ; block keys] per query row.
 //
 // Work unit (one CTA): a KV head g of sequence b, a query tile of up to 256
-// rows (block positions x the G query heads sharing g, packed so one K/V tile
-// feeds every row), and a contiguous split of the context keys.  Split 0 also
-// owns the block's own S keys.  Rows are split into two 128-row halves, each
-// an M=128 tcgen05 tile with its own TMEM accumulators:
-//   S_h  = Q_h . K^T   (TMEM, 64 fp32 columns)    P_h = exp2(S_h*c - m) (smem, bf16)
-//   O_h += P_h . V     (TMEM, dh fp32 columns)
-// Warp 0 streams 64-key K/V tiles by TMA (4-stage ring), warp 1 issues the
-// MMAs in the order S0 S1 | PV0 S0' | PV1 S1' ... so each softmax warpgroup
-// works while the tensor core serves the other half.  Warps 2-5 and 6-9 are
-// the softmax warpgroups: one thread per row (TMEM lane), so row max and row
-// sum need no shuffles.  The running max is only moved (and O rescaled in
-// TMEM) when it grows by more than 2^8, which keeps exp2 in range while
-// skipping most rescales; the final O / l is exact for any stale max.
-// Partials (unnormalised O, max, sum) are merged by attn_merge_kernel when a
-// head is split; with one split the CTA writes the bf16 result itself.
+// rows (block positions x the G query heads sharing g, packed so one K/V
+// tile feeds every row) and a contiguous split of the context keys; split 0
+// also owns the block's own S keys.  The rows form two 128-row halves, each
+// an M=128 tcgen05 tile with its own TMEM columns.  Per 128-key tile i and
+// half h:
+//   S_h  = Q_h . K(i)^T       (TMEM, 128 fp32 columns; Q and K from smem)
+//   P_h  = exp2(S_h*c - m)    (bf16, written back over S_h's columns)
+//   O_h += P_h . V(i)         (TMEM accumulator; A = P_h read from TMEM)
+// so P never goes through shared memory.  Warp 0 streams K (3-slot ring)
+// and V (2-slot ring) by TMA.  Warps 1 and 2 issue the MMAs of half 0 and
+// half 1: P_h(i).V(i) as soon as softmax h has written P_h(i), then S_h(i+1)
+// into the same columns (tcgen05 MMAs of one thread execute in issue order),
+// so neither half's chain ever queues behind the other's.  Warp 3 owns the
+// TMEM allocation and zeroes the V rows past the last valid key that a
+// 16-key MMA step still reads.  Warps 4-7 and
+// 8-11 are the softmax warpgroups of the two halves (two per SMSP, one
+// thread per row = TMEM lane: row max and row sum need no shuffles).  A
+// quarter of the exponentials run on the FMA pipe (exp2_poly) to offload
+// the MUFU unit.  The running max only moves (and O is rescaled in TMEM)
+// when it grows by more than 2^8; the final O / l is exact for any stale
+// max.  With one split the CTA writes the bf16 output; otherwise
+// (unnormalised O, max, sum) partials for a merge kernel.
 #include <math.h>
 
 #include "tt_ptx.cuh"
@@ -34,13 +41,13 @@ namespace tt {
 
 namespace {
 
-constexpr uint32_t kSub = 8192;     // one 64-key x 64-dh bf16 sub-tile (128-byte rows)
-constexpr uint32_t kQSub = 16384;   // one 128-row x 64-dh bf16 sub-tile
-constexpr uint32_t kPHalf = 16384;  // 128 rows x 64 keys bf16
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr int kKSlots = 3, kVSlots = 2;       // K and V ring depths
+constexpr uint32_t kKVSub = kAttnBN * 128;    // 128 keys x 64 dh bf16 (128-byte rows) = 16 KB
+constexpr uint32_t kQSub = 16384;             // 128 rows x 64 dh bf16
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 struct AttnSmem {
-  uint32_t q, k, v, p, bars, total;
+  uint32_t q, k, v, bars, total;
 };
 
 __host__ __device__ inline AttnSmem attn_layout(int dh, int halves) {
@@ -48,9 +55,8 @@ __host__ __device__ inline AttnSmem attn_layout(int dh, int halves) {
   const uint32_t nsub = (uint32_t)dh / 64;
   L.q = 0;
   L.k = L.q + (uint32_t)halves * nsub * kQSub;
-  L.v = L.k + kAttnStages * nsub * kSub;
-  L.p = L.v + kAttnStages * nsub * kSub;
-  L.bars = L.p + 2 * kPHalf;
+  L.v = L.k + kKSlots * nsub * kKVSub;
+  L.bars = L.v + kVSlots * nsub * kKVSub;
   L.total = L.bars + 256;
   return L;
 }
@@ -76,48 +82,29 @@ __device__ __forceinline__ TileInfo tile_info(int t, int has_blk, int k0, int k1
   return ti;
 }
 
-// Row max over the valid columns of a 64-key score tile (thread = row).
-template <bool kFull>
-__device__ __forceinline__ float row_max(const uint32_t (&sr)[64], int nvalid) {
-  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < 64; j += 4) {
-    const float v0 = __uint_as_float(sr[j]), v1 = __uint_as_float(sr[j + 1]);
-    const float v2 = __uint_as_float(sr[j + 2]), v3 = __uint_as_float(sr[j + 3]);
-    if (kFull) {
-      m0 = fmaxf(m0, v0);
-      m1 = fmaxf(m1, v1);
-      m2 = fmaxf(m2, v2);
-      m3 = fmaxf(m3, v3);
-    } else {
-      m0 = (j < nvalid) ? fmaxf(m0, v0) : m0;
-      m1 = (j + 1 < nvalid) ? fmaxf(m1, v1) : m1;
-      m2 = (j + 2 < nvalid) ? fmaxf(m2, v2) : m2;
-      m3 = (j + 3 < nvalid) ? fmaxf(m3, v3) : m3;
-    }
-  }
-  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+// 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit
+// (Cody-Waite style range reduction): n = round(x) by the float trick of
+// adding 1.5 * 2^23 (whose low mantissa bits then hold n), f = x - n in
+// [-1/2, 1/2], 2^f by a cubic fitted for relative error over that interval
+// (Chebyshev-node least squares with Lawson reweighting towards minimax; max
+// relative error 7.5e-5, far below the bf16 rounding P goes through), and
+// 2^n added to the exponent field with integer arithmetic - no conversion
+// instructions, which would run at the MUFU rate.  x <= -126 gives 0.
+__device__ __forceinline__ float exp2_poly(float x) {
+  const float xc = fmaxf(x, -126.0f);
+  const float t = xc + 12582912.0f;  // 1.5 * 2^23
+  const float f = xc - (t - 12582912.0f);
+  const float p = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111251115799f), f,
+                            0.6932609677314758f),
+                       f, 0.9999280571937561f);
+  const int e = (__float_as_int(t) - 0x4B400000) << 23;
+  const float r = __int_as_float(__float_as_int(p) + e);
+  return x > -126.0f ? r : 0.f;
 }
 
-// p = exp2(s*c - m) for the valid columns (0 elsewhere), packed to bf16
-// pairs; returns the row sum of p.
-template <bool kFull>
-__device__ __forceinline__ float exp_pack(const uint32_t (&sr)[64], int nvalid, float c, float m,
-                                          uint32_t (&pk)[32]) {
-  float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-  for (int j = 0; j < 64; j += 2) {
-    float p0 = ex2(fmaf(__uint_as_float(sr[j]), c, -m));
-    float p1 = ex2(fmaf(__uint_as_float(sr[j + 1]), c, -m));
-    if (!kFull) {
-      p0 = (j < nvalid) ? p0 : 0.f;
-      p1 = (j + 1 < nvalid) ? p1 : 0.f;
-    }
-    s0 += p0;
-    s1 += p1;
-    pk[j >> 1] = pack_bf16x2(p0, p1);
-  }
-  return s0 + s1;
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -157,24 +144,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sQ = base + SL.q;
   uint8_t* sK = base + SL.k;
   uint8_t* sV = base + SL.v;
-  uint8_t* sP = base + SL.p;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + SL.bars);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
-  uint64_t* kv_empty = kv_full + kAttnStages;
-  uint64_t* s_full = kv_empty + kAttnStages;  // [half][buffer]
-  uint64_t* p_full = s_full + 4;              // [half]: P written (and O corrected)
-  uint64_t* pv_done = p_full + 2;             // [half]: last P.V of the half finished
-  uint64_t* o_full = pv_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
+  uint64_t* k_full = q_full + 1;         // [kKSlots]
+  uint64_t* k_empty = k_full + kKSlots;  // [kKSlots], one arrival per half
+  uint64_t* v_full = k_empty + kKSlots;  // [kVSlots]
+  uint64_t* v_empty = v_full + kVSlots;  // [kVSlots], one arrival per half
+  uint64_t* v_ready = v_empty + kVSlots; // [kVSlots]: V landed and its padding rows cleared
+  uint64_t* s_full = v_ready + kVSlots;  // [half]: S_h(i) ready (and P_h(i-1).V done)
+  uint64_t* p_full = s_full + 2;         // [half]: P_h(i) written, O_h corrected
+  uint64_t* o_full = p_full + 2;         // [half]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // TMEM: S[half][buffer] (64 fp32 columns each, double-buffered so the next
-  // tile's scores are computed while this tile's softmax runs), then O[half].
-  const uint32_t tmem_need = halves * (2 * kAttnBN + dh);
+  // TMEM: S/P of half h at column h*128, then O of half h at halves*128 + h*dh.
+  const uint32_t tmem_need = halves * (kAttnBN + dh);
   const uint32_t tmem_cols = tmem_need <= 128 ? 128u : tmem_need <= 256 ? 256u : 512u;
-  const uint32_t tO0 = halves * 2 * kAttnBN;
+  const uint32_t tO0 = halves * kAttnBN;
 
   // Rows of a half that the Q box does not cover must be finite (they only
   // produce output rows that are discarded): clear Q when the box is short.
@@ -186,20 +173,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kAttnStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], halves);
     }
-    for (int i = 0; i < 4; ++i) mbar_init(&s_full[i], 1);
+    for (int s = 0; s < kVSlots; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], halves);
+      mbar_init(&v_ready[s], 1);
+    }
     for (int h = 0; h < 2; ++h) {
+      mbar_init(&s_full[h], 1);
       mbar_init(&p_full[h], 128);
-      mbar_init(&pv_done[h], 1);
+      mbar_init(&o_full[h], 1);
     }
-    mbar_init(o_full, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == 3) {
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
@@ -215,7 +206,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmKc);
       prefetch_tmap(&tmVc);
-      const uint64_t pol_kv = policy_evict_first();
+      const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
       mbar_arrive_expect_tx(q_full, (uint32_t)(halves * nsub * a.rows_per_half * 128));
       for (int h = 0; h < halves; ++h)
         for (int xh = 0; xh < nsub; ++xh)
@@ -223,144 +214,172 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                       b * a.S + pos0 + h * a.s_per_half);
       const int row_base = (b * a.Hkv + g) * a.L_cap;
       for (int t = 0; t < n_tiles; ++t) {
-        const int st = t % kAttnStages;
-        const uint32_t ph = (uint32_t)(t / kAttnStages) & 1u;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1u, a.err, abort_flag, WHERE_ATTN_PRODUCER)) break;
-        TT_TRACE_POINT(true, 0, t);
         const TileInfo ti = tile_info(t, has_blk, k0, k1, a.S);
-        uint8_t* dk = sK + st * nsub * kSub;
-        uint8_t* dv = sV + st * nsub * kSub;
-        if (ti.is_blk) {
-          mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(2 * nsub * a.S * 128));
-          for (int xh = 0; xh < nsub; ++xh) {
-            tma_load_3d(dk + xh * kSub, &tmKb, &kv_full[st], xh * 64, g, b * a.S);
-            tma_load_3d(dv + xh * kSub, &tmVb, &kv_full[st], xh * 64, g, b * a.S);
-          }
-        } else {
-          mbar_arrive_expect_tx(&kv_full[st], (uint32_t)(2 * nsub * kSub));
-          for (int xh = 0; xh < nsub; ++xh) {
-            tma_load_2d_hint(dk + xh * kSub, &tmKc, &kv_full[st], xh * 64, row_base + ti.key0,
+        const uint32_t bytes = ti.is_blk ? (uint32_t)(nsub * a.S * 128) : (uint32_t)(nsub * kKVSub);
+        const int ks = t % kKSlots;
+        if (!mbar_wait(&k_empty[ks], ((uint32_t)(t / kKSlots) & 1u) ^ 1u, a.err, abort_flag,
+                       WHERE_ATTN_PRODUCER))
+          break;
+        TT_TRACE_POINT(true, 0, t);
+        uint8_t* dk = sK + ks * nsub * kKVSub;
+        mbar_arrive_expect_tx(&k_full[ks], bytes);
+        for (int xh = 0; xh < nsub; ++xh) {
+          if (ti.is_blk)
+            tma_load_3d(dk + xh * kKVSub, &tmKb, &k_full[ks], xh * 64, g, b * a.S);
+          else
+            tma_load_2d_hint(dk + xh * kKVSub, &tmKc, &k_full[ks], xh * 64, row_base + ti.key0,
                              pol_kv);
-            tma_load_2d_hint(dv + xh * kSub, &tmVc, &kv_full[st], xh * 64, row_base + ti.key0,
+        }
+        const int vs = t % kVSlots;
+        if (!mbar_wait(&v_empty[vs], ((uint32_t)(t / kVSlots) & 1u) ^ 1u, a.err, abort_flag,
+                       WHERE_ATTN_PRODUCER))
+          break;
+        uint8_t* dv = sV + vs * nsub * kKVSub;
+        mbar_arrive_expect_tx(&v_full[vs], bytes);
+        for (int xh = 0; xh < nsub; ++xh) {
+          if (ti.is_blk)
+            tma_load_3d(dv + xh * kKVSub, &tmVb, &v_full[vs], xh * 64, g, b * a.S);
+          else
+            tma_load_2d_hint(dv + xh * kKVSub, &tmVc, &v_full[vs], xh * 64, row_base + ti.key0,
                              pol_kv);
-          }
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
-    const uint32_t idS = idesc_bf16(128, kAttnBN, false, false);
-    const uint32_t idO = idesc_bf16(128, dh, false, true);
-    const uint32_t q0 = smem_u32(sQ), k0s = smem_u32(sK), v0s = smem_u32(sV), p0s = smem_u32(sP);
-    auto issue_S = [&](int h, int st, int buf) {
-      for (int kk = 0; kk < dh / 16; ++kk) {
-        const int xh = kk >> 2;
-        const uint32_t off = (uint32_t)(kk & 3) * 32;
-        const uint64_t ad = sdesc_sw128(q0 + (h * nsub + xh) * kQSub + off, 16, 1024);
-        const uint64_t bd = sdesc_sw128(k0s + (st * nsub + xh) * kSub + off, 16, 1024);
-        umma_bf16_ss(tmem + (h * 2 + buf) * kAttnBN, ad, bd, idS, kk > 0);
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------- MMA issuer of half (warp-1)
+    const int h = warp - 1;
+    if (h < halves) {
+      const uint32_t idS = idesc_bf16(128, kAttnBN, false, false);
+      const uint32_t idO = idesc_bf16(128, dh, false, true);
+      const uint32_t q0 = smem_u32(sQ), k0s = smem_u32(sK), v0s = smem_u32(sV);
+      const uint32_t tS = tmem + h * kAttnBN, tOh = tmem + tO0 + h * dh;
+      // S_h(t) = Q_h . K(t)^T
+      auto scores = [&](int t) -> bool {
+        const int ks = t % kKSlots;
+        if (!mbar_wait(&k_full[ks], (uint32_t)(t / kKSlots) & 1u, a.err, abort_flag,
+                       WHERE_ATTN_MMA))
+          return false;
+        if (h == 0) TT_TRACE_POINT(lane == 0, 1, t);
+        tc_fence_after();
+        if (lane == 0) {
+          for (int kk = 0; kk < dh / 16; ++kk) {
+            const int xh = kk >> 2;
+            const uint32_t off = (uint32_t)(kk & 3) * 32;
+            umma_bf16_ss(tS, sdesc_sw128(q0 + (h * nsub + xh) * kQSub + off, 16, 1024),
+                         sdesc_sw128(k0s + (ks * nsub + xh) * kKVSub + off, 16, 1024), idS,
+                         kk > 0);
+          }
+          umma_commit(&s_full[h]);
+          umma_commit(&k_empty[ks]);
+        }
+        __syncwarp();
+        if (h == 0) TT_TRACE_POINT(lane == 0, 2, t);
+        return true;
+      };
+      // O_h += P_h(t) . V(t), once warp 3 has cleared V(t)'s padding rows
+      auto pv = [&](int t) -> bool {
+        if (!mbar_wait(&p_full[h], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_MMA))
+          return false;
+        TT_TRACE_POINT(lane == 0, 3 + h, t);
+        const int vs = t % kVSlots;
+        const int ksteps = (tile_info(t, has_blk, k0, k1, a.S).nvalid + 15) >> 4;
+        if (!mbar_wait(&v_ready[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
+                       WHERE_ATTN_MMA))
+          return false;
+        tc_fence_after();
+        if (lane == 0) {
+          for (int kk = 0; kk < ksteps; ++kk) {
+            // V as an MN-major operand: 64-wide dh blocks kKVSub apart, 8-key groups 1 KB apart.
+            const uint64_t bd = sdesc_sw128(v0s + vs * nsub * kKVSub + kk * 2048, kKVSub, 1024);
+            umma_bf16_ts(tOh, tS + kk * 8, bd, idO, (t > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&v_empty[vs]);
+        }
+        __syncwarp();
+        return true;
+      };
+      bool ok = mbar_wait(q_full, 0, a.err, abort_flag, WHERE_ATTN_MMA);
+      if (ok) tc_fence_after();
+      if (ok) ok = scores(0);
+      for (int t = 0; ok && t < n_tiles; ++t) {
+        ok = pv(t);
+        if (ok && t + 1 < n_tiles) ok = scores(t + 1);
       }
-    };
-    auto issue_PV = [&](int h, int st, bool acc) {
-      for (int kk = 0; kk < kAttnBN / 16; ++kk) {
-        const uint64_t ad = sdesc_sw128(p0s + h * kPHalf + kk * 32, 16, 1024);
-        // V as an MN-major operand: 64-wide dh blocks kSub apart, 8-key groups 1 KB apart.
-        const uint64_t bd = sdesc_sw128(v0s + st * nsub * kSub + kk * 2048, kSub, 1024);
-        umma_bf16_ss(tmem + tO0 + h * dh, ad, bd, idO, (acc || kk > 0) ? 1u : 0u);
-      }
-    };
-    // V rows past the valid keys of a tile may hold anything (other
-    // sequences' cache rows, stale stages); P is zero there, but 0 * NaN is
-    // NaN, so clear them before the PV product reads the stage.
-    auto prep = [&](int t, int st) {
-      const TileInfo ti = tile_info(t, has_blk, k0, k1, a.S);
-      if (ti.nvalid < kAttnBN) {
-        const int rows = kAttnBN - ti.nvalid;
+      if (lane == 0) umma_commit(&o_full[h]);
+      __syncwarp();
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------- V cleaner
+    // The P.V MMA reads V rows up to the next multiple of 16 past the valid
+    // keys.  Those rows hold whatever the cache holds beyond the context
+    // (or an older tile's rows); P is zero there but 0 * NaN is NaN, so they
+    // are zeroed before either half's MMA may read the slot.
+    for (int t = 0; t < n_tiles; ++t) {
+      const int vs = t % kVSlots;
+      if (!mbar_wait(&v_full[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
+                     WHERE_ATTN_MMA))
+        break;
+      const int nvalid = tile_info(t, has_blk, k0, k1, a.S).nvalid;
+      const int pad = ((nvalid + 15) & ~15) - nvalid;
+      if (pad > 0) {
         for (int xh = 0; xh < nsub; ++xh) {
-          uint4* dst = reinterpret_cast<uint4*>(sV + (st * nsub + xh) * kSub + ti.nvalid * 128);
-          for (int i = lane; i < rows * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+          uint4* dst = reinterpret_cast<uint4*>(sV + (vs * nsub + xh) * kKVSub + nvalid * 128);
+          for (int i = lane; i < pad * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
       }
       __syncwarp();
-    };
-    // Issue order: scores run two tiles ahead (S(0), S(1) up front), and in
-    // each iteration P(t).V is issued for each half the moment its softmax
-    // has written P, before S(t+2) - so a P.V never queues behind the next
-    // tile's score MMAs and the softmax never waits for its P buffer.
-    // S(t+2) reuses the buffer of tile t, which the softmax released with P(t).
-    auto issue_scores = [&](int tt) -> bool {
-      const int stt = tt % kAttnStages;
-      if (!mbar_wait(&kv_full[stt], (uint32_t)(tt / kAttnStages) & 1u, a.err, abort_flag,
-                     WHERE_ATTN_MMA))
-        return false;
-      TT_TRACE_POINT(lane == 0, 1, tt);
-      tc_fence_after();
-      prep(tt, stt);
-      if (lane == 0) {
-        for (int h = 0; h < halves; ++h) {
-          issue_S(h, stt, tt & 1);
-          umma_commit(&s_full[h * 2 + (tt & 1)]);
-        }
-      }
-      __syncwarp();
-      TT_TRACE_POINT(lane == 0, 2, tt);
-      return true;
-    };
-    bool ok = mbar_wait(q_full, 0, a.err, abort_flag, WHERE_ATTN_MMA);
-    for (int tt = 0; ok && tt < 2 && tt < n_tiles; ++tt) ok = issue_scores(tt);
-    for (int t = 0; ok && t < n_tiles; ++t) {
-      const int st = t % kAttnStages;
-      for (int h = 0; h < halves; ++h) {
-        if (!mbar_wait(&p_full[h], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_MMA)) {
-          ok = false;
-          break;
-        }
-        TT_TRACE_POINT(lane == 0, 3 + h, t);
-        tc_fence_after();
-        if (lane == 0) {
-          issue_PV(h, st, t > 0);
-          umma_commit(&pv_done[h]);
-        }
-        __syncwarp();
-      }
-      if (!ok) break;
-      if (lane == 0) umma_commit(&kv_empty[st]);
-      __syncwarp();
-      if (t + 2 < n_tiles) ok = issue_scores(t + 2);
+      if (lane == 0) mbar_arrive(&v_ready[vs]);
     }
-    if (lane == 0) umma_commit(o_full);
-    __syncwarp();
   } else {
     // ---------------------------------------------------- softmax groups
-    const int wg = (warp - 2) >> 2;
+    const int wg = (warp - 4) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     if (wg < halves) {
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-      const uint32_t tS = tmem + wg * 2 * kAttnBN + lane_off;
+      const uint32_t tS = tmem + wg * kAttnBN + lane_off;
       const uint32_t tO = tmem + tO0 + wg * dh + lane_off;
-      uint8_t* prow = sP + wg * kPHalf + r * 128;
       const float c = a.scale_log2;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int t = 0; t < n_tiles; ++t) {
-        const int buf = t & 1;
-        if (!mbar_wait(&s_full[wg * 2 + buf], (uint32_t)(t >> 1) & 1u, a.err, abort_flag,
+        // The two groups take turns (0 on tile t, then 1 on tile t, then 0
+        // on t+1): the tensor core runs one half's P.V and next S while the
+        // other half's softmax runs, instead of both halves contending for
+        // MUFU and then both waiting for their MMAs.  p_full[other] marks
+        // the other group's tile done.
+        if (halves == 2 && (wg == 1 || t > 0) &&
+            !mbar_wait(&p_full[wg ^ 1], (uint32_t)(wg == 1 ? t : t - 1) & 1u, a.err, abort_flag,
                        WHERE_ATTN_SOFTMAX)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&s_full[wg], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
           ok = false;
           break;
         }
         TT_TRACE_POINT(lane == 0 && q == 0, 5 + 5 * wg, t);
         tc_fence_after();
         const int nvalid = tile_info(t, has_blk, k0, k1, a.S).nvalid;
-        uint32_t sr[64];
-        tmem_ld32(tS + buf * kAttnBN, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(tS + buf * kAttnBN + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_wait_ld();
-        TT_TRACE_POINT(lane == 0 && q == 0, 6 + 5 * wg, t);
         const bool full = nvalid == kAttnBN;
-        float mx = full ? row_max<true>(sr, nvalid) : row_max<false>(sr, nvalid);
+        // pass 1: row max over 128 columns, 64 at a time, eight chains
+        float mc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mc[k] = -INFINITY;
+#pragma unroll
+        for (int c0 = 0; c0 < kAttnBN; c0 += 64) {
+          uint32_t sr[64];
+          tmem_ld64(tS + c0, sr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 64; ++j)
+            mc[j & 7] = (full || c0 + j < nvalid) ? fmaxf(mc[j & 7], __uint_as_float(sr[j]))
+                                                   : mc[j & 7];
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
+                               fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
+        TT_TRACE_POINT(lane == 0 && q == 0, 6 + 5 * wg, t);
         const float mxs = mx * c;
         const bool need = mxs > m + kRescaleThreshold;
         float alpha = 1.f;
@@ -369,42 +388,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m = mxs;
         }
         l *= alpha;
-        // P(t-1).V must have finished before O is rescaled or P rewritten.
-        if (t > 0) {
-          if (!mbar_wait(&pv_done[wg], (uint32_t)(t - 1) & 1u, a.err, abort_flag,
-                         WHERE_ATTN_SOFTMAX)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, need)) {
-            for (int c0 = 0; c0 < dh; c0 += 32) {
-              uint32_t o[32];
-              tmem_ld32(tO + c0, o);
-              tmem_wait_ld();
+        // s_full also covers P_h(t-1).V, so O_h is settled here.
+        if (t > 0 && __any_sync(0xffffffffu, need)) {
+          for (int c0 = 0; c0 < dh; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-              tmem_st32(tO + c0, o);
-            }
-            tmem_wait_st();
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+            tmem_st32(tO + c0, o);
           }
         }
         TT_TRACE_POINT(lane == 0 && q == 0, 7 + 5 * wg, t);
-        uint32_t pk[32];
-        l += full ? exp_pack<true>(sr, nvalid, c, m, pk) : exp_pack<false>(sr, nvalid, c, m, pk);
-        TT_TRACE_POINT(lane == 0 && q == 0, 8 + 5 * wg, t);
+        // pass 2: P = exp2(S*c - m) as bf16 pairs over the first 64 columns
+        // (slice 0 is stored before slice 1 is read; slice 1 lands on
+        // columns 32..63, already consumed); one pair in four on the FMA pipe.
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int phys = j ^ (r & 7);
-          *reinterpret_cast<uint4*>(prow + phys * 16) =
-              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        for (int c0 = 0; c0 < kAttnBN; c0 += 64) {
+          uint32_t sr[64], pk[32];
+          tmem_ld64(tS + c0, sr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 64; j += 2) {
+            const float x0 = fmaf(__uint_as_float(sr[j]), c, -m);
+            const float x1 = fmaf(__uint_as_float(sr[j + 1]), c, -m);
+            float p0, p1;
+            if ((j & 7) == 6) {
+              p0 = exp2_poly(x0);
+              p1 = exp2_poly(x1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            if (!full) {
+              p0 = (c0 + j < nvalid) ? p0 : 0.f;
+              p1 = (c0 + j + 1 < nvalid) ? p1 : 0.f;
+            }
+            s0 += p0;
+            s1 += p1;
+            pk[j >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st32(tS + c0 / 2, pk);
         }
-        fence_proxy_async_smem();
+        l += s0 + s1;
+        TT_TRACE_POINT(lane == 0 && q == 0, 8 + 5 * wg, t);
+        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[wg]);
         TT_TRACE_POINT(lane == 0 && q == 0, 9 + 5 * wg, t);
       }
-      if (ok && mbar_wait(o_full, 0, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
+      if (ok && mbar_wait(&o_full[wg], 0, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
         tc_fence_after();
         const bool valid = r < a.rows_per_half;
         const int s = pos0 + wg * a.s_per_half + r / a.G;
@@ -454,7 +488,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == 3) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }

@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tma_load_2d_hint(sA + stage * kStageA, &tmA, &full[stage], kb * kGemmBK, m * kGemmBM,
                            pol_a);
           tma_load_2d_hint(sB + stage * kStageB, &tmB, &full[stage], kb * kGemmBK, n * BN,
-                           num_m == 1 ? pol_b : pol_a);
+                           (a.b_keep || num_m > 1 || n < a.b_keep_tiles) ? pol_a : pol_b);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;

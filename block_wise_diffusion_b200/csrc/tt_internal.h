@@ -15,11 +15,10 @@ constexpr int kNumSMs = 148;
 enum CtrlWord {
   CTRL_ERR = 0,        // first device error code (0 = none)
   CTRL_ERR_WHERE = 1,  // where it was raised (kernel-specific tag)
-  CTRL_REMAINING = 2,  // masked positions left after the last commit
+  CTRL_REMAINING = 2,  // masked positions left (the loop's active flag)
   CTRL_M = 3,          // masked rows of the current step (vocab GEMM rows)
   CTRL_ACTIVE = 4,     // 1 while the loop still has masked positions
   CTRL_STEPS_RUN = 5,  // loop steps that did work
-  CTRL_DONE = 6,       // commit CTAs finished in this step (last one plans the next)
   CTRL_WORDS = 64
 };
 constexpr size_t kCtrlBytes = CTRL_WORDS * sizeof(int);
@@ -34,6 +33,7 @@ enum WhereTag {
   WHERE_ATTN_SOFTMAX = 0x202,
   WHERE_COMMIT_NAN = 0x300,
   WHERE_GATHER_TOKEN = 0x301,
+  WHERE_SELFTEST = 0x400,
 };
 
 // ------------------------------------------------------------------ GEMM
@@ -68,6 +68,9 @@ struct GemmArgs {
   // partial[ks][M_alloc][N]; splitk_reduce sums them into C.
   int ksplit;
   float* partial;
+  int b_keep;           // 1: load B with evict-last (re-read every loop step and small
+                        // enough to stay in L2); 0: streamed, evict-first
+  int b_keep_tiles;     // streamed B: the first b_keep_tiles N tiles still use evict-last
   int* err;             // control block
 };
 
@@ -80,9 +83,10 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int
                                  int ldc, const int* active, cudaStream_t st);
 
 // ------------------------------------------------------------- attention
-constexpr int kAttnBN = 64;        // keys per tile
-constexpr int kAttnStages = 4;
-constexpr int kAttnThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (2 x 128 rows)
+constexpr int kAttnBN = 128;       // keys per tile
+// warp 0 TMA, warps 1-2 MMA (one per 128-row half), warp 3 TMEM allocator,
+// warps 4-7 / 8-11 softmax of half 0 / half 1
+constexpr int kAttnThreads = 384;
 
 struct AttnArgs {
   int B, S, Hq, Hkv, dh, G, L_cap;
@@ -90,13 +94,14 @@ struct AttnArgs {
   const int* active;    // optional device flag
   int s_per_half;       // block positions per 128-row half
   int rows_per_half;    // s_per_half * G
-  int halves;           // halves per CTA (1 or 2)
+  int halves;           // 128-row halves per query tile and CTA (1 or 2)
   int n_qtiles;         // CTAs along the query axis per (b, g)
   int n_splits;         // key splits
   int chunk;            // context keys per split (multiple of kAttnBN)
   float scale_log2;     // log2(e) / sqrt(dh)
   uint16_t* out;        // bf16 [B*S, ldo]
   int ldo;
+  int kv_keep;          // 1: load K/V with evict-last (small cache re-read every step)
   float* part_o;        // [units][256][dh] unnormalised partial outputs
   float* part_ml;       // [units][256][2] (running max in log2 units, sum)
   int* err;
@@ -118,14 +123,17 @@ struct PlanArgs {
 };
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st);
 
+// masked == nullptr: all rows, t[b] per sequence.  Otherwise (block loop)
+// only masked rows, with their compact index and t_b computed in the kernel;
+// writes rowlist[j] and ctrl[CTRL_M].
 cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
-                         uint16_t* y, int rows, int S, int H, const int* rowlist,
-                         const int* M_dev, const int* active, cudaStream_t st);
+                         uint16_t* y, int rows, int S, int H, const uint8_t* masked,
+                         int* rowlist, int* ctrl, const int* active, cudaStream_t st);
 
-// Split merge + adaLN for the masked rows of the loop (attention split > 1).
-cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, const float* t,
-                               uint16_t* y, const int* rowlist, const int* M_dev, int max_rows,
-                               cudaStream_t st);
+// Split merge + adaLN for the masked rows of the loop (attention split > 1);
+// compacts on the fly like launch_adaln's loop mode.
+cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, uint16_t* y,
+                               const uint8_t* masked, int* rowlist, int* ctrl, cudaStream_t st);
 
 cudaError_t launch_gather_rows(const uint16_t* src, int ld_src, uint16_t* dst, int H,
                                const int* rowlist, const int* M_dev, int max_rows,
@@ -156,11 +164,11 @@ struct CommitArgs {
   const uint16_t* emb;  // [V, H]
   uint16_t* egath;      // [B*S, H] or nullptr
   int H;
-  int plan_next;        // 1: the last CTA plans the next step into plan_rowlist / plan_t
-  int* plan_rowlist;
-  float* plan_t;
+  int plan_next;        // 1: decrement ctrl[CTRL_REMAINING] by the commits, count the step
 };
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
+
+cudaError_t launch_selftest_wait(int* ctrl, unsigned long long limit_ns, cudaStream_t st);
 
 cudaError_t launch_loop_init(int B, int S, int* steps_taken, int* commit_step, int* ctrl,
                              cudaStream_t st);

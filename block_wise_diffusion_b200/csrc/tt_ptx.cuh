@@ -59,18 +59,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As above, but a thread whose phase is not yet complete is suspended for up
+// to `hint_ns` (it resumes as soon as the phase completes), so waiting warps
+// leave their SMSP's issue slots to the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+constexpr uint32_t kWaitHintNs = 0;
 
 // Bounded wait for the phase with the given parity.  `abort_flag` is a CTA
 // shared word: once any thread has timed out, later waits return at once.
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, int* err,
-                                                   volatile int* abort_flag, int where) {
+                                                   volatile int* abort_flag, int where,
+                                                   uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = global_ns();
   for (uint32_t i = 0;; ++i) {
     // A completed phase wins over the abort flag, so threads waiting on the
     // same phase all see the same outcome.
-    if (mbar_try_wait(bar, parity)) return true;
+    if (kWaitHintNs ? mbar_try_wait_for(bar, parity, kWaitHintNs) : mbar_try_wait(bar, parity))
+      return true;
     if (*abort_flag) return false;
-    if ((i & 255u) == 255u && global_ns() - t0 > kWaitLimitNs) {
+    if ((i & 255u) == 255u && global_ns() - t0 > limit_ns) {
       if (err) {
         atomicCAS(err, 0, (int)TT_ERR_TIMEOUT);
         atomicCAS(err + 1, 0, where);
@@ -161,6 +178,17 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D(tmem) (+)= A(tmem) * B(smem desc): A is M x K in TMEM (row = lane, two
+// bf16 per 32-bit column, lower k in the low half), B as above.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 // Arrive (once) on `bar` when all previously issued tcgen05.mma of this

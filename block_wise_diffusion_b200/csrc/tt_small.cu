@@ -133,19 +133,70 @@ __device__ __forceinline__ void adaln_finish(float (&v)[kAdaMaxVec][8], float s,
   }
 }
 
+// Block loop, one CTA per block row (all B*S rows are launched): decides
+// whether this CTA's row is still masked and, if so, its index j in the
+// compact list of masked rows (masked rows before it) and its sequence's
+// time t_b = masked count / S.  The CTA of the first masked row publishes the
+// row count (ctrl[CTRL_M]); every CTA records rowlist[j] = row for the commit.
+// Returns false (uniformly) for a committed row.
+__device__ bool loop_row(const uint8_t* __restrict__ masked, int rows, int S, int row,
+                         int* __restrict__ rowlist, int* __restrict__ ctrl, int* j_out,
+                         float* tb_out) {
+  __shared__ int cnt[3][kAdaThreads / 32];
+  if (masked[row] == 0) return false;
+  const int b0 = (row / S) * S;
+  int before = 0, total = 0, seq = 0;
+  for (int i = threadIdx.x; i < rows; i += blockDim.x) {
+    const int f = masked[i] != 0;
+    total += f;
+    before += (i < row) ? f : 0;
+    seq += (i >= b0 && i < b0 + S) ? f : 0;
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+    seq += __shfl_xor_sync(0xffffffffu, seq, o);
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    cnt[0][warp] = before;
+    cnt[1][warp] = total;
+    cnt[2][warp] = seq;
+  }
+  __syncthreads();
+  before = total = seq = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+    before += cnt[0][w];
+    total += cnt[1][w];
+    seq += cnt[2][w];
+  }
+  if (threadIdx.x == 0) {
+    rowlist[before] = row;
+    if (before == 0) ctrl[CTRL_M] = total;
+  }
+  *j_out = before;
+  *tb_out = (float)seq / (float)S;
+  return true;
+}
+
 __global__ void __launch_bounds__(kAdaThreads)
     adaln_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ ss,
                  const float* __restrict__ t, uint16_t* __restrict__ y, int rows, int S, int H,
-                 const int* __restrict__ rowlist, const int* M_dev, const int* active) {
+                 const uint8_t* __restrict__ masked, int* __restrict__ rowlist, int* ctrl,
+                 const int* active) {
   griddep_launch();
   griddep_wait();
   __shared__ float red[kAdaThreads / 32];
   if (active != nullptr && *active == 0) return;
-  const int M = M_dev != nullptr ? *M_dev : rows;
-  const int j = blockIdx.x;
-  if (j >= M) return;
-  const int src = rowlist != nullptr ? rowlist[j] : j;
-  const float tb = t[src / S];
+  // masked == nullptr: every row, t per sequence from `t`; otherwise the block
+  // loop's masked rows only, written compacted.
+  int j = blockIdx.x, src = blockIdx.x;
+  float tb;
+  if (masked == nullptr) {
+    tb = t[src / S];
+  } else if (!loop_row(masked, rows, S, src, rowlist, ctrl, &j, &tb)) {
+    return;
+  }
   const int nvec = H / 8;
   const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)src * H);
   float v[kAdaMaxVec][8];
@@ -175,21 +226,21 @@ __global__ void __launch_bounds__(kAdaThreads)
 // row then goes through adaln_finish.
 __global__ void __launch_bounds__(kAdaThreads)
     merge_adaln_kernel(const AttnArgs a, const uint16_t* __restrict__ ss,
-                       const float* __restrict__ t, uint16_t* __restrict__ y,
-                       const int* __restrict__ rowlist, const int* M_dev) {
+                       uint16_t* __restrict__ y, const uint8_t* __restrict__ masked,
+                       int* __restrict__ rowlist, int* ctrl) {
   griddep_launch();
   griddep_wait();
   __shared__ float red[kAdaThreads / 32];
   if (a.active != nullptr && *a.active == 0) return;
-  const int j = blockIdx.x;
-  if (j >= *M_dev) return;
-  const int row = rowlist[j];
+  const int row = blockIdx.x;
+  int j;
+  float tb;
+  if (!loop_row(masked, a.B * a.S, a.S, row, rowlist, ctrl, &j, &tb)) return;
   const int b = row / a.S, s = row % a.S;
   const int H = a.Hq * a.dh;
   const int sq = a.halves * a.s_per_half;
   const int qt = s / sq, within = s % sq;
   const int hh = within / a.s_per_half, sl = within % a.s_per_half;
-  const float tb = t[b];
   const int nvec = H / 8;
   float v[kAdaMaxVec][8];
   float sum = 0.f;
@@ -286,7 +337,6 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
   __shared__ int s_tok[32];
   __shared__ int s_mask[32];
   __shared__ int s_com[32];
-  __shared__ int s_last;
   if (a.active != nullptr && *a.active == 0) return;
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -378,8 +428,8 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
       }
       commit = is_m && s == bs;
     }
+    s_com[lane] = (in && commit) ? 1 : 0;
     if (in) {
-      s_com[s] = commit ? 1 : 0;
       if (commit) {
         s_tok[s] = tok >= 0 ? tok : 0;
         a.tokens[row] = s_tok[s];
@@ -403,19 +453,30 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
     for (int i = lane; i < a.H / 8; i += 32) dst[i] = src[i];
   }
   if (!a.plan_next) return;
-  // The last CTA to finish plans the next step (no CTA ever waits for another).
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_last = atomicAdd(a.ctrl + CTRL_DONE, 1) == a.B - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  PlanArgs p{a.B, S, a.masked, a.plan_rowlist, a.plan_t, a.ctrl, 0};
-  plan_block(p);
+  // Loop: the remaining-masked counter is also the next step's active flag.
   if (threadIdx.x == 0) {
-    a.ctrl[CTRL_DONE] = 0;
-    a.ctrl[CTRL_STEPS_RUN] += 1;
+    int n = 0;
+    for (int i = 0; i < S; ++i) n += s_com[i];
+    if (n) atomicSub(a.ctrl + CTRL_REMAINING, n);
+    if (b == 0) atomicAdd(a.ctrl + CTRL_STEPS_RUN, 1);
   }
+}
+
+// Failure-detection self test: wait on an mbarrier that nothing will ever
+// complete, with a short limit, so the bounded-wait path records
+// TT_ERR_TIMEOUT in the control block and the kernel returns normally.
+__global__ void selftest_wait_kernel(int* ctrl, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  mbar_wait_slow(&bar, 0, ctrl, &abort_flag, WHERE_SELFTEST, limit_ns);
+  __syncthreads();
+  if (threadIdx.x == 0 && abort_flag == 0) atomicCAS(ctrl, 0, (int)TT_ERR_INTERNAL);
 }
 
 __global__ void loop_init_kernel(int B, int S, int* steps_taken, int* commit_step) {
@@ -433,19 +494,18 @@ cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
-                         uint16_t* y, int rows, int S, int H, const int* rowlist,
-                         const int* M_dev, const int* active, cudaStream_t st) {
+                         uint16_t* y, int rows, int S, int H, const uint8_t* masked,
+                         int* rowlist, int* ctrl, const int* active, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
   return launch_k(adaln_kernel, dim3(rows), dim3(kAdaThreads), 0, st, x, shift_scale, t, y, rows,
-                  S, H, rowlist, M_dev, active);
+                  S, H, masked, rowlist, ctrl, active);
 }
 
-cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, const float* t,
-                               uint16_t* y, const int* rowlist, const int* M_dev, int max_rows,
-                               cudaStream_t st) {
-  if (max_rows <= 0) return cudaSuccess;
-  return launch_k(merge_adaln_kernel, dim3(max_rows), dim3(kAdaThreads), 0, st, a, shift_scale, t,
-                  y, rowlist, M_dev);
+cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, uint16_t* y,
+                               const uint8_t* masked, int* rowlist, int* ctrl, cudaStream_t st) {
+  const int rows = a.B * a.S;
+  return launch_k(merge_adaln_kernel, dim3(rows), dim3(kAdaThreads), 0, st, a, shift_scale, y,
+                  masked, rowlist, ctrl);
 }
 
 cudaError_t launch_gather_rows(const uint16_t* src, int ld_src, uint16_t* dst, int H,
@@ -466,6 +526,12 @@ cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_
 
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
   return launch_k(commit_kernel, dim3(a.B), dim3(a.S * 32), 0, st, a);
+}
+
+cudaError_t launch_selftest_wait(int* ctrl, unsigned long long limit_ns, cudaStream_t st) {
+  selftest_wait_kernel<<<1, 32, 0, st>>>(ctrl, limit_ns);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_loop_init(int B, int S, int* steps_taken, int* commit_step, int* ctrl,

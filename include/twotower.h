@@ -84,6 +84,14 @@ TT_API size_t tt_workspace_bytes(const tt_dims* d, int which);
  * TT_ERR_CUDA. */
 TT_API tt_status tt_device_status(void* ws, void* stream);
 
+/* Failure-detection self test: launches one kernel that waits on a barrier
+ * nothing completes, bounded by limit_us (1 .. 1e6 microseconds), exactly
+ * like the kernels' own pipeline waits.  The wait gives up, records
+ * TT_ERR_TIMEOUT in the control block of `ws` (>= 256 bytes) and the kernel
+ * returns; tt_device_status(ws, stream) then reports TT_ERR_TIMEOUT and the
+ * context stays usable.  Nothing faults and nothing hangs. */
+TT_API tt_status tt_selftest_timeout(void* ws, int32_t limit_us, void* stream);
+
 /* Number of kernels this library has launched in this process so far. */
 TT_API uint64_t tt_launch_count(void);
 
@@ -96,7 +104,7 @@ TT_API tt_status tt_set_attn_splits(int32_t n_splits);
 enum {
   TT_K_PLAN = 0, TT_K_EMBED = 1, TT_K_GEMM_QKV = 2, TT_K_ATTN = 3, TT_K_MERGE = 4,
   TT_K_ADALN = 5, TT_K_GEMM_VOCAB = 6, TT_K_COMMIT = 7, TT_K_GATHER = 8, TT_K_INIT = 9,
-  TT_K_COUNT = 10
+  TT_K_REDUCE = 10, TT_K_COUNT = 11
 };
 
 /* Per-kernel profiler: while enabled, every kernel this library launches is
