@@ -201,6 +201,8 @@ static AttnGeom attn_geom(const tt_dims& d) {
   n = std::min(std::min(n, max_tiles), 64);
   int per = (d.L_cap + n - 1) / n;
   g.chunk = std::max(kAttnBN, (per + kAttnBN - 1) / kAttnBN * kAttnBN);
+  // rounding the chunk up to whole tiles can leave trailing splits empty
+  n = std::max(1, (d.L_cap + g.chunk - 1) / g.chunk);
   g.n_splits = n;
   const size_t rows = (size_t)units * n * 256;
   g.part_o_bytes = n > 1 ? rows * d.dh * sizeof(float) : 0;
@@ -244,6 +246,9 @@ struct Ws {
   float* part_ml = nullptr;
   float4* stats = nullptr;
   float* qkv_partial = nullptr;
+  int* seqcnt = nullptr;     // follows ctrl directly: cleared together
+  float2* rowres = nullptr;
+  size_t ctrl_clear = kCtrlBytes;  // bytes from ctrl to clear at the start of a call
   size_t total = 0;
 };
 
@@ -253,6 +258,10 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
   const size_t rows = (size_t)d.B * d.S;
   const size_t n_vt = (size_t)(d.V + kVocabBN - 1) / kVocabBN;
   w.ctrl = c.take<int>(kCtrlBytes);
+  if (which == TT_WS_VOCAB || which == TT_WS_LOOP) {
+    w.seqcnt = c.take<int>((size_t)d.B * sizeof(int));
+    w.ctrl_clear = c.off;
+  }
   if (which == TT_WS_ATTN || which == TT_WS_LOOP) {
     const AttnGeom g = attn_geom(d);
     if (g.n_splits > 1) {
@@ -261,10 +270,11 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     }
   }
   if (which == TT_WS_VOCAB || which == TT_WS_LOOP) {
-    w.rowlist = c.take<int>(rows * sizeof(int));
+    w.rowlist = c.take<int>(2 * rows * sizeof(int));
     w.tvec = c.take<float>((size_t)d.B * sizeof(float));
     w.y_c = c.take<uint16_t>(rows * d.H * 2);
     w.stats = c.take<float4>(n_vt * rows * sizeof(float4));
+    w.rowres = c.take<float2>(rows * sizeof(float2));
   }
   if (which == TT_WS_LOOP) {
     const size_t n_qkv = (size_t)d.H + 2 * (size_t)d.Hkv * d.dh;
@@ -387,6 +397,8 @@ static CommitArgs commit_args(const tt_dims& d, const Ws& w, float gamma, float 
   c.scale_log2 = (float)(logit_scale * 1.4426950408889634);
   c.gamma = gamma;
   c.rowlist = w.rowlist;
+  c.rowres = w.rowres;
+  c.seqcnt = w.seqcnt;
   c.M_dev = w.ctrl + CTRL_M;
   c.tokens = tokens;
   c.masked = masked;
@@ -546,7 +558,7 @@ tt_status tt_vocab_confidence_commit(const tt_dims* d, const tt_bf16* y, const t
   Ws ws_;
   TT_CHECK(check_ws(*d, TT_WS_VOCAB, ws, ws_bytes, &ws_));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  TT_CUDA(cudaMemsetAsync(ws_.ctrl, 0, kCtrlBytes, st));
+  TT_CUDA(cudaMemsetAsync(ws_.ctrl, 0, ws_.ctrl_clear, st));
   PlanArgs p{d->B, d->S, masked, ws_.rowlist, ws_.tvec, ws_.ctrl, 0};
   TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
   TT_LAUNCH(TT_K_GATHER, st, launch_gather_rows(y, d->H, ws_.y_c, d->H, ws_.rowlist, ws_.ctrl + CTRL_M,
@@ -601,7 +613,7 @@ tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt
   TT_CHECK(build_attn_maps(*d, g, w.qkv, n_qkv, w.qkv + d->H, w.qkv + d->H + d->Hkv * d->dh,
                            n_qkv, k_ctx, v_ctx, &m));
 
-  TT_CUDA(cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st));
+  TT_CUDA(cudaMemsetAsync(w.ctrl, 0, w.ctrl_clear, st));
   TT_LAUNCH(TT_K_INIT, st, launch_loop_init(d->B, d->S, steps_taken, commit_step, w.ctrl, st));
   // a step runs while masked positions remain (commit decrements the count)
   const int* active = w.ctrl + CTRL_REMAINING;

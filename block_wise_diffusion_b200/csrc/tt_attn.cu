@@ -22,8 +22,8 @@
 // TMEM allocation and zeroes the V rows past the last valid key that a
 // 16-key MMA step still reads.  Warps 4-7 and
 // 8-11 are the softmax warpgroups of the two halves (two per SMSP, one
-// thread per row = TMEM lane: row max and row sum need no shuffles).  A
-// quarter of the exponentials run on the FMA pipe (exp2_poly) to offload
+// thread per row = TMEM lane: row max and row sum need no shuffles).  An
+// eighth of the exponentials run on the FMA pipe (exp2_poly) to offload
 // the MUFU unit.  The running max only moves (and O is rescaled in TMEM)
 // when it grows by more than 2^8; the final O / l is exact for any stale
 // max.  With one split the CTA writes the bf16 output; otherwise
@@ -47,7 +47,7 @@ constexpr uint32_t kQSub = 16384;             // 128 rows x 64 dh bf16
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 struct AttnSmem {
-  uint32_t q, k, v, bars, total;
+  uint32_t q, k, v, bars, xchg, total;
 };
 
 __host__ __device__ inline AttnSmem attn_layout(int dh, int halves) {
@@ -57,7 +57,8 @@ __host__ __device__ inline AttnSmem attn_layout(int dh, int halves) {
   L.k = L.q + (uint32_t)halves * nsub * kQSub;
   L.v = L.k + kKSlots * nsub * kKVSub;
   L.bars = L.v + kVSlots * nsub * kKVSub;
-  L.total = L.bars + 256;
+  L.xchg = L.bars + 256;      // row-max exchange: [half][quarter][column half][lane] bf16
+  L.total = L.xchg + 1024;
   return L;
 }
 
@@ -100,11 +101,6 @@ __device__ __forceinline__ float exp2_poly(float x) {
   const int e = (__float_as_int(t) - 0x4B400000) << 23;
   const float r = __int_as_float(__float_as_int(p) + e);
   return x > -126.0f ? r : 0.f;
-}
-
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
-  tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -154,7 +150,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* s_full = v_ready + kVSlots;  // [half]: S_h(i) ready (and P_h(i-1).V done)
   uint64_t* p_full = s_full + 2;         // [half]: P_h(i) written, O_h corrected
   uint64_t* o_full = p_full + 2;         // [half]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
+  uint64_t* xbar = o_full + 2;           // [half][quarter]: both column halves' row maxima written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 8);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -184,9 +181,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&s_full[h], 1);
-      mbar_init(&p_full[h], 128);
+      mbar_init(&p_full[h], 256);
       mbar_init(&o_full[h], 1);
     }
+    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -200,155 +198,168 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const int pos0 = qt * halves * a.s_per_half;  // first block position of this query tile
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmKc);
-      prefetch_tmap(&tmVc);
-      const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
-      mbar_arrive_expect_tx(q_full, (uint32_t)(halves * nsub * a.rows_per_half * 128));
-      for (int h = 0; h < halves; ++h)
-        for (int xh = 0; xh < nsub; ++xh)
-          tma_load_3d(sQ + (h * nsub + xh) * kQSub, &tmQ, q_full, xh * 64, g * a.G,
-                      b * a.S + pos0 + h * a.s_per_half);
-      const int row_base = (b * a.Hkv + g) * a.L_cap;
+  if (warp < 4) {
+    if (warp == 0) {
+      // ------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmKc);
+        prefetch_tmap(&tmVc);
+        const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
+        mbar_arrive_expect_tx(q_full, (uint32_t)(halves * nsub * a.rows_per_half * 128));
+        for (int h = 0; h < halves; ++h)
+          for (int xh = 0; xh < nsub; ++xh)
+            tma_load_3d(sQ + (h * nsub + xh) * kQSub, &tmQ, q_full, xh * 64, g * a.G,
+                        b * a.S + pos0 + h * a.s_per_half);
+        const int row_base = (b * a.Hkv + g) * a.L_cap;
+        for (int t = 0; t < n_tiles; ++t) {
+          const TileInfo ti = tile_info(t, has_blk, k0, k1, a.S);
+          const uint32_t bytes = ti.is_blk ? (uint32_t)(nsub * a.S * 128) : (uint32_t)(nsub * kKVSub);
+          const int ks = t % kKSlots;
+          if (!mbar_wait(&k_empty[ks], ((uint32_t)(t / kKSlots) & 1u) ^ 1u, a.err, abort_flag,
+                         WHERE_ATTN_PRODUCER))
+            break;
+          TT_TRACE_POINT(true, 0, t);
+          uint8_t* dk = sK + ks * nsub * kKVSub;
+          mbar_arrive_expect_tx(&k_full[ks], bytes);
+          for (int xh = 0; xh < nsub; ++xh) {
+            if (ti.is_blk)
+              tma_load_3d(dk + xh * kKVSub, &tmKb, &k_full[ks], xh * 64, g, b * a.S);
+            else
+              tma_load_2d_hint(dk + xh * kKVSub, &tmKc, &k_full[ks], xh * 64, row_base + ti.key0,
+                               pol_kv);
+          }
+          const int vs = t % kVSlots;
+          if (!mbar_wait(&v_empty[vs], ((uint32_t)(t / kVSlots) & 1u) ^ 1u, a.err, abort_flag,
+                         WHERE_ATTN_PRODUCER))
+            break;
+          uint8_t* dv = sV + vs * nsub * kKVSub;
+          mbar_arrive_expect_tx(&v_full[vs], bytes);
+          for (int xh = 0; xh < nsub; ++xh) {
+            if (ti.is_blk)
+              tma_load_3d(dv + xh * kKVSub, &tmVb, &v_full[vs], xh * 64, g, b * a.S);
+            else
+              tma_load_2d_hint(dv + xh * kKVSub, &tmVc, &v_full[vs], xh * 64, row_base + ti.key0,
+                               pol_kv);
+          }
+        }
+      }
+    } else if (warp == 1 || warp == 2) {
+      // ------------------------------------------- MMA issuer of half (warp-1)
+      const int h = warp - 1;
+      if (h < halves) {
+        const uint32_t idS = idesc_bf16(128, kAttnBN, false, false);
+        const uint32_t idO = idesc_bf16(128, dh, false, true);
+        const uint32_t q0 = smem_u32(sQ), k0s = smem_u32(sK), v0s = smem_u32(sV);
+        const uint32_t tS = tmem + h * kAttnBN, tOh = tmem + tO0 + h * dh;
+        // S_h(t) = Q_h . K(t)^T
+        auto scores = [&](int t) -> bool {
+          const int ks = t % kKSlots;
+          if (!mbar_wait(&k_full[ks], (uint32_t)(t / kKSlots) & 1u, a.err, abort_flag,
+                         WHERE_ATTN_MMA))
+            return false;
+          if (h == 0) TT_TRACE_POINT(lane == 0, 1, t);
+          tc_fence_after();
+          if (lane == 0) {
+            for (int kk = 0; kk < dh / 16; ++kk) {
+              const int xh = kk >> 2;
+              const uint32_t off = (uint32_t)(kk & 3) * 32;
+              umma_bf16_ss(tS, sdesc_sw128(q0 + (h * nsub + xh) * kQSub + off, 16, 1024),
+                           sdesc_sw128(k0s + (ks * nsub + xh) * kKVSub + off, 16, 1024), idS,
+                           kk > 0);
+            }
+            umma_commit(&s_full[h]);
+            umma_commit(&k_empty[ks]);
+          }
+          __syncwarp();
+          if (h == 0) TT_TRACE_POINT(lane == 0, 2, t);
+          return true;
+        };
+        // O_h += P_h(t) . V(t), once warp 3 has cleared V(t)'s padding rows
+        auto pv = [&](int t) -> bool {
+          if (!mbar_wait(&p_full[h], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_MMA))
+            return false;
+          TT_TRACE_POINT(lane == 0, 3 + h, t);
+          const int vs = t % kVSlots;
+          const int ksteps = (tile_info(t, has_blk, k0, k1, a.S).nvalid + 15) >> 4;
+          if (!mbar_wait(&v_ready[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
+                         WHERE_ATTN_MMA))
+            return false;
+          tc_fence_after();
+          if (lane == 0) {
+            for (int kk = 0; kk < ksteps; ++kk) {
+              // V as an MN-major operand: 64-wide dh blocks kKVSub apart, 8-key groups 1 KB apart.
+              const uint64_t bd = sdesc_sw128(v0s + vs * nsub * kKVSub + kk * 2048, kKVSub, 1024);
+              // P of keys 0..63 sits in columns 0..31, of keys 64..127 in 64..95
+            umma_bf16_ts(tOh, tS + kk * 8 + (kk >= 4 ? 32 : 0), bd, idO, (t > 0 || kk > 0) ? 1u : 0u);
+            }
+            umma_commit(&v_empty[vs]);
+          }
+          __syncwarp();
+          return true;
+        };
+        bool ok = mbar_wait(q_full, 0, a.err, abort_flag, WHERE_ATTN_MMA);
+        if (ok) tc_fence_after();
+        if (ok) ok = scores(0);
+        for (int t = 0; ok && t < n_tiles; ++t) {
+          ok = pv(t);
+          if (ok && t + 1 < n_tiles) ok = scores(t + 1);
+        }
+        if (lane == 0) umma_commit(&o_full[h]);
+        __syncwarp();
+      }
+    } else {
+      // ------------------------------------------------------- V cleaner
+      // The P.V MMA reads V rows up to the next multiple of 16 past the valid
+      // keys.  Those rows hold whatever the cache holds beyond the context
+      // (or an older tile's rows); P is zero there but 0 * NaN is NaN, so they
+      // are zeroed before either half's MMA may read the slot.
       for (int t = 0; t < n_tiles; ++t) {
-        const TileInfo ti = tile_info(t, has_blk, k0, k1, a.S);
-        const uint32_t bytes = ti.is_blk ? (uint32_t)(nsub * a.S * 128) : (uint32_t)(nsub * kKVSub);
-        const int ks = t % kKSlots;
-        if (!mbar_wait(&k_empty[ks], ((uint32_t)(t / kKSlots) & 1u) ^ 1u, a.err, abort_flag,
-                       WHERE_ATTN_PRODUCER))
-          break;
-        TT_TRACE_POINT(true, 0, t);
-        uint8_t* dk = sK + ks * nsub * kKVSub;
-        mbar_arrive_expect_tx(&k_full[ks], bytes);
-        for (int xh = 0; xh < nsub; ++xh) {
-          if (ti.is_blk)
-            tma_load_3d(dk + xh * kKVSub, &tmKb, &k_full[ks], xh * 64, g, b * a.S);
-          else
-            tma_load_2d_hint(dk + xh * kKVSub, &tmKc, &k_full[ks], xh * 64, row_base + ti.key0,
-                             pol_kv);
-        }
         const int vs = t % kVSlots;
-        if (!mbar_wait(&v_empty[vs], ((uint32_t)(t / kVSlots) & 1u) ^ 1u, a.err, abort_flag,
-                       WHERE_ATTN_PRODUCER))
-          break;
-        uint8_t* dv = sV + vs * nsub * kKVSub;
-        mbar_arrive_expect_tx(&v_full[vs], bytes);
-        for (int xh = 0; xh < nsub; ++xh) {
-          if (ti.is_blk)
-            tma_load_3d(dv + xh * kKVSub, &tmVb, &v_full[vs], xh * 64, g, b * a.S);
-          else
-            tma_load_2d_hint(dv + xh * kKVSub, &tmVc, &v_full[vs], xh * 64, row_base + ti.key0,
-                             pol_kv);
-        }
-      }
-    }
-  } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------- MMA issuer of half (warp-1)
-    const int h = warp - 1;
-    if (h < halves) {
-      const uint32_t idS = idesc_bf16(128, kAttnBN, false, false);
-      const uint32_t idO = idesc_bf16(128, dh, false, true);
-      const uint32_t q0 = smem_u32(sQ), k0s = smem_u32(sK), v0s = smem_u32(sV);
-      const uint32_t tS = tmem + h * kAttnBN, tOh = tmem + tO0 + h * dh;
-      // S_h(t) = Q_h . K(t)^T
-      auto scores = [&](int t) -> bool {
-        const int ks = t % kKSlots;
-        if (!mbar_wait(&k_full[ks], (uint32_t)(t / kKSlots) & 1u, a.err, abort_flag,
+        if (!mbar_wait(&v_full[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
                        WHERE_ATTN_MMA))
-          return false;
-        if (h == 0) TT_TRACE_POINT(lane == 0, 1, t);
-        tc_fence_after();
-        if (lane == 0) {
-          for (int kk = 0; kk < dh / 16; ++kk) {
-            const int xh = kk >> 2;
-            const uint32_t off = (uint32_t)(kk & 3) * 32;
-            umma_bf16_ss(tS, sdesc_sw128(q0 + (h * nsub + xh) * kQSub + off, 16, 1024),
-                         sdesc_sw128(k0s + (ks * nsub + xh) * kKVSub + off, 16, 1024), idS,
-                         kk > 0);
+          break;
+        const int nvalid = tile_info(t, has_blk, k0, k1, a.S).nvalid;
+        const int pad = ((nvalid + 15) & ~15) - nvalid;
+        if (pad > 0) {
+          for (int xh = 0; xh < nsub; ++xh) {
+            uint4* dst = reinterpret_cast<uint4*>(sV + (vs * nsub + xh) * kKVSub + nvalid * 128);
+            for (int i = lane; i < pad * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
           }
-          umma_commit(&s_full[h]);
-          umma_commit(&k_empty[ks]);
+          fence_proxy_async_smem();
         }
         __syncwarp();
-        if (h == 0) TT_TRACE_POINT(lane == 0, 2, t);
-        return true;
-      };
-      // O_h += P_h(t) . V(t), once warp 3 has cleared V(t)'s padding rows
-      auto pv = [&](int t) -> bool {
-        if (!mbar_wait(&p_full[h], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_MMA))
-          return false;
-        TT_TRACE_POINT(lane == 0, 3 + h, t);
-        const int vs = t % kVSlots;
-        const int ksteps = (tile_info(t, has_blk, k0, k1, a.S).nvalid + 15) >> 4;
-        if (!mbar_wait(&v_ready[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
-                       WHERE_ATTN_MMA))
-          return false;
-        tc_fence_after();
-        if (lane == 0) {
-          for (int kk = 0; kk < ksteps; ++kk) {
-            // V as an MN-major operand: 64-wide dh blocks kKVSub apart, 8-key groups 1 KB apart.
-            const uint64_t bd = sdesc_sw128(v0s + vs * nsub * kKVSub + kk * 2048, kKVSub, 1024);
-            umma_bf16_ts(tOh, tS + kk * 8, bd, idO, (t > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&v_empty[vs]);
-        }
-        __syncwarp();
-        return true;
-      };
-      bool ok = mbar_wait(q_full, 0, a.err, abort_flag, WHERE_ATTN_MMA);
-      if (ok) tc_fence_after();
-      if (ok) ok = scores(0);
-      for (int t = 0; ok && t < n_tiles; ++t) {
-        ok = pv(t);
-        if (ok && t + 1 < n_tiles) ok = scores(t + 1);
+        if (lane == 0) mbar_arrive(&v_ready[vs]);
       }
-      if (lane == 0) umma_commit(&o_full[h]);
-      __syncwarp();
-    }
-  } else if (warp == 3) {
-    // ------------------------------------------------------- V cleaner
-    // The P.V MMA reads V rows up to the next multiple of 16 past the valid
-    // keys.  Those rows hold whatever the cache holds beyond the context
-    // (or an older tile's rows); P is zero there but 0 * NaN is NaN, so they
-    // are zeroed before either half's MMA may read the slot.
-    for (int t = 0; t < n_tiles; ++t) {
-      const int vs = t % kVSlots;
-      if (!mbar_wait(&v_full[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
-                     WHERE_ATTN_MMA))
-        break;
-      const int nvalid = tile_info(t, has_blk, k0, k1, a.S).nvalid;
-      const int pad = ((nvalid + 15) & ~15) - nvalid;
-      if (pad > 0) {
-        for (int xh = 0; xh < nsub; ++xh) {
-          uint4* dst = reinterpret_cast<uint4*>(sV + (vs * nsub + xh) * kKVSub + nvalid * 128);
-          for (int i = lane; i < pad * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
-        }
-        fence_proxy_async_smem();
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&v_ready[vs]);
     }
   } else {
     // ---------------------------------------------------- softmax groups
-    const int wg = (warp - 4) >> 2;
+    // Half wg is served by warps 4+8*wg .. 11+8*wg.  Warp w owns the rows of
+    // its TMEM lane quarter q = w % 4 and one column half ch of every tile
+    // (S columns ch*64..+63, the O columns ch*dh/2..+dh/2-1), so two warps
+    // per SMSP share a row: they swap their partial row maxima through
+    // shared memory (as bf16, rounded the same way on both sides, so both
+    // use the identical stabiliser) and add their row sums at the end.
+    const int wg = (warp - 4) >> 3;
+    const int ch = ((warp - 4) >> 2) & 1;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     if (wg < halves) {
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-      const uint32_t tS = tmem + wg * kAttnBN + lane_off;
-      const uint32_t tO = tmem + tO0 + wg * dh + lane_off;
+      const uint32_t tS = tmem + wg * kAttnBN + lane_off + ch * 64;
+      const int dh2 = dh / 2;
+      const uint32_t tO = tmem + tO0 + wg * dh + lane_off + ch * dh2;
+      uint16_t* xch = reinterpret_cast<uint16_t*>(base + SL.xchg) + (wg * 4 + q) * 64;
+      uint64_t* xb = &xbar[wg * 4 + q];
       const float c = a.scale_log2;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
       for (int t = 0; t < n_tiles; ++t) {
-        // The two groups take turns (0 on tile t, then 1 on tile t, then 0
+        // The two halves take turns (0 on tile t, then 1 on tile t, then 0
         // on t+1): the tensor core runs one half's P.V and next S while the
         // other half's softmax runs, instead of both halves contending for
         // MUFU and then both waiting for their MMAs.  p_full[other] marks
-        // the other group's tile done.
+        // the other half's tile done.
         if (halves == 2 && (wg == 1 || t > 0) &&
             !mbar_wait(&p_full[wg ^ 1], (uint32_t)(wg == 1 ? t : t - 1) & 1u, a.err, abort_flag,
                        WHERE_ATTN_SOFTMAX)) {
@@ -359,27 +370,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           ok = false;
           break;
         }
-        TT_TRACE_POINT(lane == 0 && q == 0, 5 + 5 * wg, t);
+        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 5 + 5 * wg, t);
         tc_fence_after();
-        const int nvalid = tile_info(t, has_blk, k0, k1, a.S).nvalid;
-        const bool full = nvalid == kAttnBN;
-        // pass 1: row max over 128 columns, 64 at a time, eight chains
-        float mc[8];
+        // Columns past the valid keys (the block's own tile, or the last
+        // tile of a split) are overwritten with -inf: nothing to the max,
+        // exp2 gives 0 on both exponential paths.
+        const int nv = tile_info(t, has_blk, k0, k1, a.S).nvalid - ch * 64;
+        if (nv < 64) {
+          for (int c0 = max(nv, 0) & ~31; c0 < 64; c0 += 32) {
+            uint32_t v[32];
+            if (c0 < nv) {
+              tmem_ld32(tS + c0, v);
+              tmem_wait_ld();
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mc[k] = -INFINITY;
+              for (int j = 0; j < 32; ++j) v[j] = c0 + j < nv ? v[j] : __float_as_uint(-INFINITY);
+            } else {
 #pragma unroll
-        for (int c0 = 0; c0 < kAttnBN; c0 += 64) {
-          uint32_t sr[64];
-          tmem_ld64(tS + c0, sr);
+              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(-INFINITY);
+            }
+            tmem_st32(tS + c0, v);
+          }
+          tmem_wait_st();
+        }
+        float mc[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mc[k] = -INFINITY;
+        uint32_t sa[32];
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          tmem_ld32(tS + c0, sa);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 64; ++j)
-            mc[j & 7] = (full || c0 + j < nvalid) ? fmaxf(mc[j & 7], __uint_as_float(sr[j]))
-                                                   : mc[j & 7];
+          for (int j = 0; j < 32; j += 2)
+            mc[(j >> 1) & 3] = fmax3(mc[(j >> 1) & 3], __uint_as_float(sa[j]), __uint_as_float(sa[j + 1]));
         }
-        const float mx = fmaxf(fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3])),
-                               fmaxf(fmaxf(mc[4], mc[5]), fmaxf(mc[6], mc[7])));
-        TT_TRACE_POINT(lane == 0 && q == 0, 6 + 5 * wg, t);
+        const float part = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
+        // The first exponential slice is read while the maxima are swapped.
+        tmem_ld32(tS, sa);
+        // One buffer suffices: a warp writes tile t+1's value only after
+        // S(t+1), which needs its partner's P(t), written after the read.
+        xch[ch * 32 + lane] = bf16_bits(part);
+        mbar_arrive(xb);
+        if (!mbar_wait(xb, (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
+          tmem_wait_ld();
+          ok = false;
+          break;
+        }
+        const float mx = fmaxf(bf16_value(xch[lane]), bf16_value(xch[32 + lane]));
+        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 6 + 5 * wg, t);
         const float mxs = mx * c;
         const bool need = mxs > m + kRescaleThreshold;
         float alpha = 1.f;
@@ -388,9 +426,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           m = mxs;
         }
         l *= alpha;
-        // s_full also covers P_h(t-1).V, so O_h is settled here.
+        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 7 + 5 * wg, t);
+        // P = exp2(S*c - m) as bf16 pairs, written into this warp's own S
+        // columns (slice i's 16 pair columns over slice i's first half, read
+        // already); one pair in eight on the FMA pipe.
+        float s0 = 0.f, s1 = 0.f;
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          if (c0 > 0) {
+            tmem_ld32(tS + c0, sa);
+            tmem_wait_ld();
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float x0 = fmaf(__uint_as_float(sa[j]), c, -m);
+            const float x1 = fmaf(__uint_as_float(sa[j + 1]), c, -m);
+            float p0, p1;
+            if ((j & 15) == 14) {
+              p0 = exp2_poly(x0);
+              p1 = exp2_poly(x1);
+            } else {
+              p0 = ex2(x0);
+              p1 = ex2(x1);
+            }
+            s0 += p0;
+            s1 += p1;
+            pk[j >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + c0 / 2, pk);
+        }
+        l += s0 + s1;
+        // O_h to the new max before P_h(t).V adds to it (s_full also
+        // covered P_h(t-1).V, so O_h is settled).
         if (t > 0 && __any_sync(0xffffffffu, need)) {
-          for (int c0 = 0; c0 < dh; c0 += 32) {
+          for (int c0 = 0; c0 < dh2; c0 += 32) {
             uint32_t o[32];
             tmem_ld32(tO + c0, o);
             tmem_wait_ld();
@@ -399,47 +470,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tO + c0, o);
           }
         }
-        TT_TRACE_POINT(lane == 0 && q == 0, 7 + 5 * wg, t);
-        // pass 2: P = exp2(S*c - m) as bf16 pairs over the first 64 columns
-        // (slice 0 is stored before slice 1 is read; slice 1 lands on
-        // columns 32..63, already consumed); one pair in four on the FMA pipe.
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-        for (int c0 = 0; c0 < kAttnBN; c0 += 64) {
-          uint32_t sr[64], pk[32];
-          tmem_ld64(tS + c0, sr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 64; j += 2) {
-            const float x0 = fmaf(__uint_as_float(sr[j]), c, -m);
-            const float x1 = fmaf(__uint_as_float(sr[j + 1]), c, -m);
-            float p0, p1;
-            if ((j & 7) == 6) {
-              p0 = exp2_poly(x0);
-              p1 = exp2_poly(x1);
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
-            }
-            if (!full) {
-              p0 = (c0 + j < nvalid) ? p0 : 0.f;
-              p1 = (c0 + j + 1 < nvalid) ? p1 : 0.f;
-            }
-            s0 += p0;
-            s1 += p1;
-            pk[j >> 1] = pack_bf16x2(p0, p1);
-          }
-          tmem_st32(tS + c0 / 2, pk);
-        }
-        l += s0 + s1;
-        TT_TRACE_POINT(lane == 0 && q == 0, 8 + 5 * wg, t);
+        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 8 + 5 * wg, t);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[wg]);
-        TT_TRACE_POINT(lane == 0 && q == 0, 9 + 5 * wg, t);
+        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 9 + 5 * wg, t);
       }
-      if (ok && mbar_wait(&o_full[wg], 0, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
+      // Column half 1 hands its row sum to column half 0, which writes the
+      // whole row.  o_full (the last P.V done) implies both warps have read
+      // the last tile's maxima, so the buffer is free.
+      if (ok) ok = mbar_wait(&o_full[wg], 0, a.err, abort_flag, WHERE_ATTN_SOFTMAX);
+      if (ok) {
+        if (ch == 1) {
+          const uint32_t lb = __float_as_uint(l);
+          xch[lane] = (uint16_t)(lb & 0xffffu);
+          xch[32 + lane] = (uint16_t)(lb >> 16);
+        }
+        mbar_arrive(xb);
+        ok = mbar_wait(xb, (uint32_t)n_tiles & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX);
+      }
+      if (ok && ch == 0) {
+        l += __uint_as_float((uint32_t)xch[lane] | ((uint32_t)xch[32 + lane] << 16));
         tc_fence_after();
+        const uint32_t tOr = tmem + tO0 + wg * dh + lane_off;  // the whole O row
         const bool valid = r < a.rows_per_half;
         const int s = pos0 + wg * a.s_per_half + r / a.G;
         const int head = g * a.G + r % a.G;
@@ -448,7 +501,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           uint16_t* dst = a.out + (size_t)(b * a.S + s) * a.ldo + head * dh;
           for (int c0 = 0; c0 < dh; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(tO + c0, o);
+            tmem_ld32(tOr + c0, o);
             tmem_wait_ld();
             if (valid) {
 #pragma unroll
@@ -467,7 +520,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           float* po = a.part_o + prow_i * dh;
           for (int c0 = 0; c0 < dh; c0 += 32) {
             uint32_t o[32];
-            tmem_ld32(tO + c0, o);
+            tmem_ld32(tOr + c0, o);
             tmem_wait_ld();
             if (valid) {
 #pragma unroll
@@ -510,27 +563,44 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a) {
   if (h >= a.halves || r >= a.rows_per_half) return;
   const int pair = pq / a.n_qtiles, qt = pq % a.n_qtiles;
   const int b = pair / a.Hkv, g = pair % a.Hkv;
-  float mstar = -INFINITY;
-  for (int sp = 0; sp < a.n_splits; ++sp) {
-    const size_t i = ((size_t)(pq * a.n_splits + sp) * 256 + row256) * 2;
-    if (a.part_ml[i + 1] > 0.f) mstar = fmaxf(mstar, a.part_ml[i]);
-  }
+  // One pass over the splits (running max, rescaled sums), four splits'
+  // loads in flight before any is used; an empty split (l = 0, O never
+  // written) is skipped by selection.
+  const size_t prow0 = (size_t)pq * a.n_splits * 256 + row256;
   const int d0 = lane * 4;
   const bool act = d0 < a.dh;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float den = 0.f;
-  for (int sp = 0; sp < a.n_splits; ++sp) {
-    const size_t prow = (size_t)(pq * a.n_splits + sp) * 256 + row256;
-    const float ms = a.part_ml[prow * 2], ls = a.part_ml[prow * 2 + 1];
-    if (!(ls > 0.f)) continue;
-    const float w = ex2(ms - mstar);
-    den += w * ls;
-    if (act) {
-      const float4 o = *reinterpret_cast<const float4*>(a.part_o + prow * a.dh + d0);
-      acc.x += w * o.x;
-      acc.y += w * o.y;
-      acc.z += w * o.z;
-      acc.w += w * o.w;
+  float den = 0.f, mrun = -INFINITY;
+  for (int sp0 = 0; sp0 < a.n_splits; sp0 += 4) {
+    float2 ml[4];
+    float4 o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const size_t prow = prow0 + (size_t)(sp0 + i) * 256;
+      const bool in = sp0 + i < a.n_splits;
+      ml[i] = in ? *reinterpret_cast<const float2*>(a.part_ml + prow * 2)
+                 : make_float2(-INFINITY, 0.f);
+      o[i] = in && act ? *reinterpret_cast<const float4*>(a.part_o + prow * a.dh + d0)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (!(ml[i].y > 0.f)) continue;
+      if (ml[i].x > mrun) {
+        const float sc = mrun == -INFINITY ? 0.f : ex2(mrun - ml[i].x);
+        den *= sc;
+        acc.x *= sc;
+        acc.y *= sc;
+        acc.z *= sc;
+        acc.w *= sc;
+        mrun = ml[i].x;
+      }
+      const float w = ex2(ml[i].x - mrun);
+      den += w * ml[i].y;
+      acc.x += w * o[i].x;
+      acc.y += w * o[i].y;
+      acc.z += w * o[i].z;
+      acc.w += w * o[i].w;
     }
   }
   if (act) {

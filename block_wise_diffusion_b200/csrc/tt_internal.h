@@ -84,9 +84,9 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int
 
 // ------------------------------------------------------------- attention
 constexpr int kAttnBN = 128;       // keys per tile
-// warp 0 TMA, warps 1-2 MMA (one per 128-row half), warp 3 TMEM allocator,
-// warps 4-7 / 8-11 softmax of half 0 / half 1
-constexpr int kAttnThreads = 384;
+// warp 0 TMA, warps 1-2 MMA (one per 128-row half), warp 3 TMEM owner and
+// V padding, warps 4-11 / 12-19 softmax of half 0 / half 1
+constexpr int kAttnThreads = 640;
 
 struct AttnArgs {
   int B, S, Hq, Hkv, dh, G, L_cap;
@@ -116,7 +116,8 @@ cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t st);
 struct PlanArgs {
   int B, S;
   const uint8_t* masked;
-  int* rowlist;     // [B*S] compact list of masked rows (b*S+s)
+  int* rowlist;     // [2*B*S]: compact list of masked rows (b*S+s), then at
+                    // B*S + row the compact index of each masked row
   float* t;         // [B]   masked fraction at the start of the step
   int* ctrl;        // writes CTRL_M, CTRL_REMAINING, CTRL_ACTIVE, CTRL_STEPS_RUN
   int count_step;   // unused (kept for layout); steps are counted by the commit kernel
@@ -143,12 +144,18 @@ cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_
                          const uint16_t* e_mask, uint16_t* dst, int rows, int H, int V,
                          const int* active, int* err, cudaStream_t st);
 
+// The commit runs as B*S/kCommitRows CTAs (one warp per block row); the
+// last CTA of a sequence to finish (a per-sequence counter) applies the
+// commit rule to the whole sequence.
+constexpr int kCommitRows = 4;
 struct CommitArgs {
   int B, S, n_vt;
+  float2* rowres;       // [B*S] (confidence, token bits) of each row
+  int* seqcnt;          // [B] finished CTAs per sequence; zero before the call, left zero
   const float4* stats;  // [compact row][n_vt] tile statistics of the vocab GEMM
   float scale_log2;
   float gamma;
-  const int* rowlist;   // compact row -> b*S+s
+  const int* rowlist;   // compact row -> b*S+s, then b*S+s -> compact row (at B*S + row)
   const int* M_dev;
   int* tokens;
   uint8_t* masked;

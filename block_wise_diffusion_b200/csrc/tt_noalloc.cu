@@ -73,10 +73,13 @@ extern "C" tt_status tt_vocab_confidence_commit_noalloc(
   const size_t n_vt = (size_t)(d->V + kVocabBN - 1) / kVocabBN;
   size_t off = 0;
   const size_t o_ctrl = off;    off = up256(off + kCtrlBytes);
-  const size_t o_rows = off;    off = up256(off + rows * sizeof(int));
+  const size_t o_seq = off;     off = up256(off + (size_t)d->B * sizeof(int));
+  const size_t clear_bytes = off;  // control block and sequence counters start at zero
+  const size_t o_rows = off;    off = up256(off + 2 * rows * sizeof(int));
   const size_t o_t = off;       off = up256(off + (size_t)d->B * sizeof(float));
   const size_t o_yc = off;      off = up256(off + rows * (size_t)d->H * 2);
   const size_t o_st = off;      off = up256(off + n_vt * rows * sizeof(float4));
+  const size_t o_rr = off;      off = up256(off + rows * sizeof(float2));
   if (off > kNoAllocScratchBytes) {
     char msg[200];
     snprintf(msg, sizeof msg,
@@ -95,12 +98,14 @@ extern "C" tt_status tt_vocab_confidence_commit_noalloc(
   float* tvec = reinterpret_cast<float*>(sb + o_t);
   uint16_t* y_c = reinterpret_cast<uint16_t*>(sb + o_yc);
   float4* stats = reinterpret_cast<float4*>(sb + o_st);
+  int* seqcnt = reinterpret_cast<int*>(sb + o_seq);
+  float2* rowres = reinterpret_cast<float2*>(sb + o_rr);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
 
   // The array keeps the previous call's contents: the control block (row
-  // count, error word) must start from zero; everything else is written
-  // before it is read.
-  e = cudaMemsetAsync(ctrl, 0, kCtrlBytes, st);
+  // count, error word) and the per-sequence counters must start from zero;
+  // everything else is written before it is read.
+  e = cudaMemsetAsync(ctrl, 0, clear_bytes, st);
   if (e != cudaSuccess) return set_error(TT_ERR_CUDA, cudaGetErrorString(e));
 
   PlanArgs p{d->B, d->S, masked, rowlist, tvec, ctrl, 0};
@@ -133,6 +138,8 @@ extern "C" tt_status tt_vocab_confidence_commit_noalloc(
   c.scale_log2 = g.scale_log2;
   c.gamma = gamma;
   c.rowlist = rowlist;
+  c.rowres = rowres;
+  c.seqcnt = seqcnt;
   c.M_dev = ctrl + CTRL_M;
   c.tokens = tokens;
   c.masked = masked;

@@ -37,7 +37,10 @@ __device__ void plan_block(const PlanArgs& a) {
       before_warps += (w < warp) ? c : 0;
       total += c;
     }
-    if (f) a.rowlist[running + before_warps + before_in_warp] = i;
+    if (f) {
+      a.rowlist[running + before_warps + before_in_warp] = i;
+      a.rowlist[n + i] = running + before_warps + before_in_warp;
+    }
     __syncthreads();
     if (tid == 0) running += total;
     __syncthreads();
@@ -64,8 +67,8 @@ __global__ void __launch_bounds__(1024) plan_kernel(const PlanArgs a) {
 // ----------------------------------------------------------------- adaLN
 // One CTA per output row.  y = LN(x) * (1 + E1 + cos(t w)) + E0 + sin(t w),
 // w_i = 10000^(-i/H): the adaLN-single reading of this library.
-constexpr int kAdaThreads = 256;
-constexpr int kAdaMaxVec = 4;  // H <= 256 threads * 4 vectors * 8 = 8192
+constexpr int kAdaThreads = 512;
+constexpr int kAdaMaxVec = 2;  // H <= 512 threads * 2 vectors * 8 = 8192
 
 __device__ __forceinline__ float block_sum(float v, float* red) {
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -84,6 +87,18 @@ __device__ __forceinline__ void adaln_finish(float (&v)[kAdaMaxVec][8], float s,
                                              const uint16_t* __restrict__ ss,
                                              uint16_t* __restrict__ yrow, float* red) {
   const int nvec = H / 8;
+  // shift/scale loads are issued before the two reductions
+  uint4 a0[kAdaMaxVec], a1[kAdaMaxVec];
+  const uint4* e0 = reinterpret_cast<const uint4*>(ss);
+  const uint4* e1 = reinterpret_cast<const uint4*>(ss + H);
+#pragma unroll
+  for (int k = 0; k < kAdaMaxVec; ++k) {
+    const int vi = threadIdx.x + k * kAdaThreads;
+    if (vi < nvec) {
+      a0[k] = e0[vi];
+      a1[k] = e1[vi];
+    }
+  }
   const float mean = block_sum(s, red) / (float)H;
   float q = 0.f;
 #pragma unroll
@@ -101,15 +116,12 @@ __device__ __forceinline__ void adaln_finish(float (&v)[kAdaMaxVec][8], float s,
   const float rstd = rsqrtf(var + 1e-6f);
   const float lw = -13.287712379549449f / (float)H;  // -log2(10000) / H
   uint4* yr = reinterpret_cast<uint4*>(yrow);
-  const uint4* e0 = reinterpret_cast<const uint4*>(ss);
-  const uint4* e1 = reinterpret_cast<const uint4*>(ss + H);
 #pragma unroll
   for (int k = 0; k < kAdaMaxVec; ++k) {
     const int vi = threadIdx.x + k * kAdaThreads;
     if (vi < nvec) {
-      const uint4 a0 = e0[vi], a1 = e1[vi];
-      const uint32_t sh[4] = {a0.x, a0.y, a0.z, a0.w};
-      const uint32_t sc[4] = {a1.x, a1.y, a1.z, a1.w};
+      const uint32_t sh[4] = {a0[k].x, a0[k].y, a0[k].z, a0[k].w};
+      const uint32_t sc[4] = {a1[k].x, a1[k].y, a1[k].z, a1[k].w};
       float out[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -172,6 +184,7 @@ __device__ bool loop_row(const uint8_t* __restrict__ masked, int rows, int S, in
   }
   if (threadIdx.x == 0) {
     rowlist[before] = row;
+    rowlist[rows + row] = before;
     if (before == 0) ctrl[CTRL_M] = total;
   }
   *j_out = before;
@@ -242,40 +255,77 @@ __global__ void __launch_bounds__(kAdaThreads)
   const int qt = s / sq, within = s % sq;
   const int hh = within / a.s_per_half, sl = within % a.s_per_half;
   const int nvec = H / 8;
-  float v[kAdaMaxVec][8];
+  // Each thread merges kAdaMaxVec 8-element vectors of the row in one pass
+  // over the splits (running max, rescaled sums), loading four splits' data
+  // for all its vectors before using any.  An empty split (l = 0, O never
+  // written) is skipped by selection.
+  size_t prow[kAdaMaxVec];  // partial row of split 0
+  int d0[kAdaMaxVec];
+  bool kin[kAdaMaxVec];
+  float mrun[kAdaMaxVec], den[kAdaMaxVec], v[kAdaMaxVec][8];
+#pragma unroll
+  for (int k = 0; k < kAdaMaxVec; ++k) {
+    kin[k] = (int)threadIdx.x + k * kAdaThreads < nvec;
+    const int vi = min((int)threadIdx.x + k * kAdaThreads, nvec - 1);
+    const int e0 = vi * 8, head = e0 / a.dh;
+    const int g = head / a.G, jh = head % a.G;
+    prow[k] = (size_t)((b * a.Hkv + g) * a.n_qtiles + qt) * a.n_splits * 256 + hh * 128 +
+              sl * a.G + jh;
+    d0[k] = e0 % a.dh;
+    mrun[k] = -INFINITY;
+    den[k] = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[k][e] = 0.f;
+  }
+  for (int sp0 = 0; sp0 < a.n_splits; sp0 += 4) {
+    float2 ml[4][kAdaMaxVec];
+    float4 x0[4][kAdaMaxVec], x1[4][kAdaMaxVec];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int k = 0; k < kAdaMaxVec; ++k) {
+        if (sp0 + i < a.n_splits && kin[k]) {
+          const size_t pr = prow[k] + (size_t)(sp0 + i) * 256;
+          ml[i][k] = *reinterpret_cast<const float2*>(a.part_ml + pr * 2);
+          const float4* po = reinterpret_cast<const float4*>(a.part_o + pr * a.dh + d0[k]);
+          x0[i][k] = po[0];
+          x1[i][k] = po[1];
+        } else {
+          ml[i][k] = make_float2(-INFINITY, 0.f);
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+      for (int k = 0; k < kAdaMaxVec; ++k) {
+        if (!(ml[i][k].y > 0.f)) continue;
+        if (ml[i][k].x > mrun[k]) {
+          const float sc = mrun[k] == -INFINITY ? 0.f : ex2(mrun[k] - ml[i][k].x);
+          den[k] *= sc;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[k][e] *= sc;
+          mrun[k] = ml[i][k].x;
+        }
+        const float w = ex2(ml[i][k].x - mrun[k]);
+        den[k] += w * ml[i][k].y;
+        v[k][0] += w * x0[i][k].x; v[k][1] += w * x0[i][k].y;
+        v[k][2] += w * x0[i][k].z; v[k][3] += w * x0[i][k].w;
+        v[k][4] += w * x1[i][k].x; v[k][5] += w * x1[i][k].y;
+        v[k][6] += w * x1[i][k].z; v[k][7] += w * x1[i][k].w;
+      }
+    }
+  }
   float sum = 0.f;
 #pragma unroll
   for (int k = 0; k < kAdaMaxVec; ++k) {
-    const int vi = threadIdx.x + k * kAdaThreads;
-    if (vi < nvec) {
-      const int e0 = vi * 8, head = e0 / a.dh, d0 = e0 % a.dh;
-      const int g = head / a.G, jh = head % a.G;
-      const size_t unit0 = (size_t)((b * a.Hkv + g) * a.n_qtiles + qt) * a.n_splits;
-      const int r256 = hh * 128 + sl * a.G + jh;
-      float mstar = -INFINITY;
-      for (int sp = 0; sp < a.n_splits; ++sp) {
-        const size_t pr = (unit0 + sp) * 256 + r256;
-        if (a.part_ml[pr * 2 + 1] > 0.f) mstar = fmaxf(mstar, a.part_ml[pr * 2]);
-      }
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      float den = 0.f;
-      for (int sp = 0; sp < a.n_splits; ++sp) {
-        const size_t pr = (unit0 + sp) * 256 + r256;
-        const float ls = a.part_ml[pr * 2 + 1];
-        if (!(ls > 0.f)) continue;
-        const float w = ex2(a.part_ml[pr * 2] - mstar);
-        den += w * ls;
-        const float4* po = reinterpret_cast<const float4*>(a.part_o + pr * a.dh + d0);
-        const float4 x0 = po[0], x1 = po[1];
-        acc[0] += w * x0.x; acc[1] += w * x0.y; acc[2] += w * x0.z; acc[3] += w * x0.w;
-        acc[4] += w * x1.x; acc[5] += w * x1.y; acc[6] += w * x1.z; acc[7] += w * x1.w;
-      }
-      const float inv = 1.f / den;
+    if (!kin[k]) continue;
+    const float inv = 1.f / den[k];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        v[k][e] = __uint_as_float(pack_bf16x2(acc[e] * inv, 0.f) << 16);
-        sum += v[k][e];
-      }
+    for (int e = 0; e < 8; ++e) {
+      // the attention output is bf16 in the unfused path: round the same way
+      v[k][e] = __uint_as_float(pack_bf16x2(v[k][e] * inv, 0.f) << 16);
+      sum += v[k][e];
     }
   }
   adaln_finish(v, sum, H, tb, ss, y + (size_t)j * H, red);
@@ -325,92 +375,96 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------- commit
-// One CTA per sequence, one warp per block position.  A masked position's
-// 256-column tile statistics are merged into its confidence
+// One warp per block row, kCommitRows rows per CTA.  A masked position's
+// tile statistics are merged into its confidence
 //   conf = 1 / sum_t z_t 2^(c*(v_t - v*)),  token = argmax column of the
-// tile with the largest v_t (lowest tile on ties, hence lowest id);
-// then warp 0 applies the commit rule across the block.
-__global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
+// tile with the largest v_t (lowest tile on ties, hence lowest id).
+// The last CTA of a sequence to finish then applies the commit rule
+// across the sequence's S positions.
+__global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitArgs a) {
   griddep_launch();
   griddep_wait();
-  __shared__ float s_conf[32];
+  __shared__ int s_last;
   __shared__ int s_tok[32];
-  __shared__ int s_mask[32];
   __shared__ int s_com[32];
   if (a.active != nullptr && *a.active == 0) return;
-  const int b = blockIdx.x;
+  const int S = a.S, per_seq = S / kCommitRows;
+  const int b = blockIdx.x / per_seq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = a.S;
+  const int row = b * S + (blockIdx.x % per_seq) * kCommitRows + warp;
   const int M = a.M_dev != nullptr ? *a.M_dev : a.B * S;
-  if (warp < S) {
-    const int row = b * S + warp;
-    const int is_m = a.masked[row] != 0;
-    float conf = -1.f;
-    int tok = -1;
-    if (is_m) {
-      // compact index of this row: rowlist is sorted, so search it
-      int lo = 0, hi = M - 1, j = -1;
-      while (lo <= hi) {
-        const int mid = (lo + hi) >> 1;
-        const int v = a.rowlist[mid];
-        if (v == row) {
-          j = mid;
-          break;
-        }
-        if (v < row) lo = mid + 1; else hi = mid - 1;
-      }
-      if (j >= 0) {
-        // tiles of row j are contiguous: lane t reads tiles t, t+32, ...
-        const float4* st = a.stats + (size_t)j * a.n_vt;
-        float bv = -INFINITY;
-        int bt = 0x7fffffff;
-        for (int t = lane; t < a.n_vt; t += 32) {
-          const float v = st[t].x;
-          if (v > bv) {  // t increases per lane, so ties keep the lowest tile
-            bv = v;
-            bt = t;
+  float conf = -1.f;
+  int tok = -1;
+  if (a.masked[row] != 0) {
+    const int j = a.rowlist[a.B * S + row];  // this row's compact index
+    if (j >= 0 && j < M) {
+      // One pass over the row's tiles (lane t reads tiles t, t+32, ...):
+      // running best tile maximum v*, its token, and
+      //   Z = sum_t z_t 2^(c (v_t - v*)),
+      // rescaled whenever v* grows.  t increases per lane, so a strict >
+      // keeps the lowest tile on ties.
+      const float4* st = a.stats + (size_t)j * a.n_vt;
+      const float c = a.scale_log2;
+      float bv = -INFINITY, Z = 0.f;
+      int bt = 0x7fffffff, btok = -1;
+      for (int t0 = lane; t0 < a.n_vt; t0 += 32 * 8) {
+        float4 q[8];  // eight loads in flight before any is used
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          q[i] = t0 + 32 * i < a.n_vt ? st[t0 + 32 * i] : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (q[i].x > bv) {
+            Z = (bv == -INFINITY ? 0.f : Z * ex2((bv - q[i].x) * c)) + q[i].y;
+            bv = q[i].x;
+            bt = t0 + 32 * i;
+            btok = __float_as_int(q[i].z);
+          } else if (q[i].x > -INFINITY) {
+            Z += q[i].y * ex2((q[i].x - bv) * c);
           }
         }
-        for (int o = 16; o > 0; o >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-          const int ot = __shfl_xor_sync(0xffffffffu, bt, o);
-          if (ov > bv || (ov == bv && ot < bt)) {
-            bv = ov;
-            bt = ot;
-          }
-        }
-        const float mstar = bv * a.scale_log2;
-        float Z = 0.f;
-        for (int t = lane; t < a.n_vt; t += 32) {
-          const float4 q = st[t];
-          Z += q.y * ex2(q.x * a.scale_log2 - mstar);
-        }
-        for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
-        conf = 1.f / Z;
-        tok = (bt < a.n_vt) ? __float_as_int(st[bt].z) : -1;
       }
-    }
-    if (lane == 0) {
-      s_conf[warp] = conf;
-      s_tok[warp] = tok;
-      s_mask[warp] = is_m;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int ot = __shfl_xor_sync(0xffffffffu, bt, o);
+        const int otok = __shfl_xor_sync(0xffffffffu, btok, o);
+        const float oZ = __shfl_xor_sync(0xffffffffu, Z, o);
+        const float nv = fmaxf(bv, ov);
+        Z = (bv == nv ? Z : Z * ex2((bv - nv) * c)) + (ov == nv ? oZ : oZ * ex2((ov - nv) * c));
+        if (ov > bv || (ov == bv && ot < bt)) {
+          bv = ov;
+          bt = ot;
+          btok = otok;
+        }
+      }
+      conf = 1.f / Z;
+      tok = bt < a.n_vt ? btok : -1;
     }
   }
+  if (lane == 0) a.rowres[row] = make_float2(conf, __int_as_float(tok));
   __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(a.seqcnt + b, 1) == per_seq - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
   if (warp == 0) {
     const int s = lane;
     const bool in = s < S;
-    const int row = b * S + s;
-    const int is_m = in ? s_mask[s] : 0;
-    float cf = in ? s_conf[s] : -1.f;
-    const int tok = in ? s_tok[s] : -1;
+    const int r = b * S + s;
+    const int is_m = in ? a.masked[r] != 0 : 0;
+    const float2 rr = in ? __ldcg(a.rowres + r) : make_float2(-1.f, __int_as_float(-1));
+    float cf = rr.x;
+    const int tk = __float_as_int(rr.y);
     const bool bad = is_m && !(cf >= 0.f && cf <= 1.0001f);  // NaN or impossible value
     if (__any_sync(0xffffffffu, bad) && lane == 0) {
       atomicCAS(a.ctrl + CTRL_ERR, 0, (int)TT_ERR_INTERNAL);
       atomicCAS(a.ctrl + CTRL_ERR_WHERE, 0, (int)WHERE_COMMIT_NAN);
     }
     if (bad) cf = -1.f;
-    const bool qual = is_m && cf >= a.gamma && tok >= 0;
+    const bool qual = is_m && cf >= a.gamma && tk >= 0;
     const unsigned qmask = __ballot_sync(0xffffffffu, qual);
     const unsigned mmask = __ballot_sync(0xffffffffu, is_m != 0);
     bool commit = qual;
@@ -429,36 +483,37 @@ __global__ void __launch_bounds__(1024) commit_kernel(const CommitArgs a) {
       commit = is_m && s == bs;
     }
     s_com[lane] = (in && commit) ? 1 : 0;
+    s_tok[lane] = tk >= 0 ? tk : 0;
     if (in) {
       if (commit) {
-        s_tok[s] = tok >= 0 ? tok : 0;
-        a.tokens[row] = s_tok[s];
-        a.masked[row] = 0;
-        if (a.commit_step != nullptr) a.commit_step[row] = a.step;
+        a.tokens[r] = s_tok[lane];
+        a.masked[r] = 0;
+        if (a.commit_step != nullptr) a.commit_step[r] = a.step;
       }
-      if (a.conf_out != nullptr) a.conf_out[row] = is_m ? s_conf[s] : -1.f;
-      if (a.argmax_out != nullptr) a.argmax_out[row] = is_m ? tok : -1;
+      if (a.conf_out != nullptr) a.conf_out[r] = is_m ? rr.x : -1.f;
+      if (a.argmax_out != nullptr) a.argmax_out[r] = is_m ? tk : -1;
     }
     const unsigned cmask = __ballot_sync(0xffffffffu, commit);
     if (lane == 0) {
+      a.seqcnt[b] = 0;  // ready for the next call
       if (a.n_committed != nullptr) a.n_committed[b] = __popc(cmask);
       if (a.steps_taken != nullptr && mmask != 0) a.steps_taken[b] = a.step + 1;
+      if (a.plan_next) {
+        // Loop: the remaining-masked counter is also the next step's active flag.
+        if (cmask) atomicSub(a.ctrl + CTRL_REMAINING, __popc(cmask));
+        if (b == 0) atomicAdd(a.ctrl + CTRL_STEPS_RUN, 1);
+      }
     }
   }
   __syncthreads();
   // Loop only: a newly committed position's next embedding is Emb[token].
-  if (a.egath != nullptr && warp < S && s_com[warp]) {
-    const uint4* src = reinterpret_cast<const uint4*>(a.emb + (size_t)s_tok[warp] * a.H);
-    uint4* dst = reinterpret_cast<uint4*>(a.egath + (size_t)(b * S + warp) * a.H);
-    for (int i = lane; i < a.H / 8; i += 32) dst[i] = src[i];
-  }
-  if (!a.plan_next) return;
-  // Loop: the remaining-masked counter is also the next step's active flag.
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int i = 0; i < S; ++i) n += s_com[i];
-    if (n) atomicSub(a.ctrl + CTRL_REMAINING, n);
-    if (b == 0) atomicAdd(a.ctrl + CTRL_STEPS_RUN, 1);
+  if (a.egath != nullptr) {
+    for (int s = warp; s < S; s += kCommitRows) {
+      if (!s_com[s]) continue;
+      const uint4* src = reinterpret_cast<const uint4*>(a.emb + (size_t)s_tok[s] * a.H);
+      uint4* dst = reinterpret_cast<uint4*>(a.egath + (size_t)(b * S + s) * a.H);
+      for (int i = lane; i < a.H / 8; i += 32) dst[i] = src[i];
+    }
   }
 }
 
@@ -525,7 +580,8 @@ cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_
 }
 
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
-  return launch_k(commit_kernel, dim3(a.B), dim3(a.S * 32), 0, st, a);
+  return launch_k(commit_kernel, dim3(a.B * (a.S / kCommitRows)), dim3(kCommitRows * 32), 0, st,
+                  a);
 }
 
 cudaError_t launch_selftest_wait(int* ctrl, unsigned long long limit_ns, cudaStream_t st) {

@@ -241,9 +241,10 @@ TT_API tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, c
  * minus the workspace.  Its scratch is one built-in device array of 16 MiB
  * (16777216 bytes) that every GPU which loads this library holds until the
  * process exits.  A problem whose scratch exceeds it - 256 bytes of control
- * words, the masked-row list (B*S*4 bytes), B*4 bytes of timesteps,
- * B*S*H*2 bytes of gathered rows and B*S*ceil(V/224)*16 bytes of tile
- * statistics, each rounded up to 256 bytes - is rejected with
+ * words, B*4 bytes of per-sequence counters, the masked-row list and its
+ * inverse (B*S*8 bytes), B*4 bytes of timesteps, B*S*H*2 bytes of gathered
+ * rows, B*S*ceil(V/224)*16 bytes of tile statistics and B*S*8 bytes of row
+ * results, each rounded up to 256 bytes - is rejected with
  * TT_ERR_WORKSPACE before any launch.  It allocates nothing:
  * no cudaMalloc/cudaFree and no allocating library routine.
  *  - The first call on each device looks up the array's device address
