@@ -182,7 +182,7 @@ static tt_status check_ptr(const void* p, const char* name, bool need16) {
 
 // ------------------------------------------------------------ geometry
 struct AttnGeom {
-  int G, s_per_half, rows_per_half, halves, n_qtiles, n_splits, chunk;
+  int G, s_per_half, rows_per_half, halves, n_qtiles, n_splits, chunk, first;
   size_t part_o_bytes, part_ml_bytes;
 };
 
@@ -194,15 +194,17 @@ static AttnGeom attn_geom(const tt_dims& d) {
   g.halves = std::min(2, d.S / g.s_per_half);
   g.n_qtiles = d.S / (g.halves * g.s_per_half);
   const long long units = (long long)d.B * d.Hkv * g.n_qtiles;
-  const int max_tiles = std::max(1, (d.L_cap + kAttnBN - 1) / kAttnBN);
+  const int ctx_tiles = (d.L_cap + kAttnBN - 1) / kAttnBN;
   const int forced = g_forced_splits.load();
   // one CTA per (unit, split): fill the SMs once
   int n = forced > 0 ? forced : (int)std::max<long long>(1, kNumSMs / units);
-  n = std::min(std::min(n, max_tiles), 64);
-  int per = (d.L_cap + n - 1) / n;
-  g.chunk = std::max(kAttnBN, (per + kAttnBN - 1) / kAttnBN * kAttnBN);
-  // rounding the chunk up to whole tiles can leave trailing splits empty
-  n = std::max(1, (d.L_cap + g.chunk - 1) / g.chunk);
+  n = std::min(std::min(n, ctx_tiles + 1), 64);
+  // Split 0 also runs the block's own key tile, so it gets one context tile
+  // fewer: every split then runs at most c tiles, c = ceil((tiles + 1) / n).
+  const int c = (ctx_tiles + 1 + n - 1) / n;
+  g.chunk = c * kAttnBN;
+  g.first = (c - 1) * kAttnBN;
+  n = 1 + (std::max(0, d.L_cap - g.first) + g.chunk - 1) / g.chunk;
   g.n_splits = n;
   const size_t rows = (size_t)units * n * 256;
   g.part_o_bytes = n > 1 ? rows * d.dh * sizeof(float) : 0;
@@ -282,7 +284,10 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     w.qkv = c.take<uint16_t>(rows * n_qkv * 2);
     w.attn_out = c.take<uint16_t>(rows * d.H * 2);
     const int ks = qkv_ksplit(d);
-    if (ks > 1) w.qkv_partial = c.take<float>((size_t)ks * rows * n_qkv * sizeof(float));
+    // tile-major partials: ks planes of whole 128 x kQkvBN tiles
+    const size_t tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kQkvBN - 1) / kQkvBN);
+    if (ks > 1)
+      w.qkv_partial = c.take<float>((size_t)ks * tiles * kGemmBM * kQkvBN * sizeof(float));
   }
   w.total = (c.off + 255) & ~size_t(255);
   return w;
@@ -340,6 +345,7 @@ static AttnArgs attn_args(const tt_dims& d, const AttnGeom& g, const int32_t* ct
   a.n_qtiles = g.n_qtiles;
   a.n_splits = g.n_splits;
   a.chunk = g.chunk;
+  a.first = g.first;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.dh));
   a.out = out;
   a.ldo = d.H;

@@ -12,22 +12,26 @@
 // an M=128 tcgen05 tile with its own TMEM columns.  Per 128-key tile i and
 // half h:
 //   S_h  = Q_h . K(i)^T       (TMEM, 128 fp32 columns; Q and K from smem)
-//   P_h  = exp2(S_h*c - m)    (bf16, written back over S_h's columns)
+//   P_h  = exp2(S_h*c - m)    (bf16 pairs, written back into S_h's columns)
 //   O_h += P_h . V(i)         (TMEM accumulator; A = P_h read from TMEM)
-// so P never goes through shared memory.  Warp 0 streams K (3-slot ring)
-// and V (2-slot ring) by TMA.  Warps 1 and 2 issue the MMAs of half 0 and
-// half 1: P_h(i).V(i) as soon as softmax h has written P_h(i), then S_h(i+1)
-// into the same columns (tcgen05 MMAs of one thread execute in issue order),
-// so neither half's chain ever queues behind the other's.  Warp 3 owns the
-// TMEM allocation and zeroes the V rows past the last valid key that a
-// 16-key MMA step still reads.  Warps 4-7 and
-// 8-11 are the softmax warpgroups of the two halves (two per SMSP, one
-// thread per row = TMEM lane: row max and row sum need no shuffles).  An
-// eighth of the exponentials run on the FMA pipe (exp2_poly) to offload
-// the MUFU unit.  The running max only moves (and O is rescaled in TMEM)
-// when it grows by more than 2^8; the final O / l is exact for any stale
-// max.  With one split the CTA writes the bf16 output; otherwise
-// (unnormalised O, max, sum) partials for a merge kernel.
+// so P never goes through shared memory.  Roles (20 warps):
+//   warp 0     TMA for Q and K (3-slot ring);
+//   warps 1, 2 MMA issue for half 0 / half 1: P_h(i).V(i) as soon as
+//              softmax h has written P_h(i), then S_h(i+1) into the same
+//              columns (tcgen05 MMAs of one thread execute in issue order);
+//   warp 3     TMEM owner; TMA for V (2-slot ring) and zeroing of the V rows
+//              past the last valid key that a 16-key MMA step still reads;
+//   warps 4-11 / 12-19  softmax of half 0 / half 1.  Warp w serves the 32
+//              rows of its TMEM lane quarter (w % 4) and one 64-key column
+//              half of every tile; the two warps of a row swap partial row
+//              maxima through shared memory.  Thread = row: no shuffles.
+// The two softmax groups take turns tile by tile, so the tensor core runs
+// one half's MMAs during the other half's softmax.  An eighth of the
+// exponentials run on the FMA pipe (exp2_poly) to offload the MUFU unit.
+// The running max only moves (and O is rescaled in TMEM) when it grows by
+// more than 2^8; the final O / l is exact for any stale max.  With one split
+// the CTA writes the bf16 output; otherwise (unnormalised O, max, sum)
+// partials for a merge kernel.
 #include <math.h>
 
 #include "tt_ptx.cuh"
@@ -118,8 +122,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (threadIdx.x == 0) atomicCAS(a.err, 0, (int)TT_ERR_INVALID_ARG);
     L = min(max(L, 0), a.L_cap);
   }
-  const int k0 = split * a.chunk;
-  const int k1 = min(k0 + a.chunk, L);
+  const int k0 = split == 0 ? 0 : a.first + (split - 1) * a.chunk;
+  const int k1 = min(split == 0 ? a.first : k0 + a.chunk, L);
   const int n_ctx_tiles = k1 > k0 ? (k1 - k0 + kAttnBN - 1) / kAttnBN : 0;
   const int has_blk = split == 0 ? 1 : 0;
   const int n_tiles = has_blk + n_ctx_tiles;
@@ -200,11 +204,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (warp < 4) {
     if (warp == 0) {
-      // ------------------------------------------------------ TMA producer
+      // ------------------------------------------------ TMA producer: Q, K
       if (lane == 0) {
         prefetch_tmap(&tmQ);
         prefetch_tmap(&tmKc);
-        prefetch_tmap(&tmVc);
         const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
         mbar_arrive_expect_tx(q_full, (uint32_t)(halves * nsub * a.rows_per_half * 128));
         for (int h = 0; h < halves; ++h)
@@ -229,19 +232,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               tma_load_2d_hint(dk + xh * kKVSub, &tmKc, &k_full[ks], xh * 64, row_base + ti.key0,
                                pol_kv);
           }
-          const int vs = t % kVSlots;
-          if (!mbar_wait(&v_empty[vs], ((uint32_t)(t / kVSlots) & 1u) ^ 1u, a.err, abort_flag,
-                         WHERE_ATTN_PRODUCER))
-            break;
-          uint8_t* dv = sV + vs * nsub * kKVSub;
-          mbar_arrive_expect_tx(&v_full[vs], bytes);
-          for (int xh = 0; xh < nsub; ++xh) {
-            if (ti.is_blk)
-              tma_load_3d(dv + xh * kKVSub, &tmVb, &v_full[vs], xh * 64, g, b * a.S);
-            else
-              tma_load_2d_hint(dv + xh * kKVSub, &tmVc, &v_full[vs], xh * 64, row_base + ti.key0,
-                               pol_kv);
-          }
         }
       }
     } else if (warp == 1 || warp == 2) {
@@ -250,8 +240,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (h < halves) {
         const uint32_t idS = idesc_bf16(128, kAttnBN, false, false);
         const uint32_t idO = idesc_bf16(128, dh, false, true);
-        const uint32_t q0 = smem_u32(sQ), k0s = smem_u32(sK), v0s = smem_u32(sV);
         const uint32_t tS = tmem + h * kAttnBN, tOh = tmem + tO0 + h * dh;
+        // Descriptor bases; each MMA adds a compile-time offset (the start
+        // address field is address >> 4 in the low bits, and no smem address
+        // carries out of it), so an issue costs a few instructions: the
+        // issuing warp shares its SMSP with busy softmax warps.
+        const uint64_t dQ = sdesc_sw128(smem_u32(sQ) + h * nsub * kQSub, 16, 1024);
+        const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+        const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kKVSub, 1024);
         // S_h(t) = Q_h . K(t)^T
         auto scores = [&](int t) -> bool {
           const int ks = t % kKSlots;
@@ -261,12 +257,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (h == 0) TT_TRACE_POINT(lane == 0, 1, t);
           tc_fence_after();
           if (lane == 0) {
-            for (int kk = 0; kk < dh / 16; ++kk) {
-              const int xh = kk >> 2;
-              const uint32_t off = (uint32_t)(kk & 3) * 32;
-              umma_bf16_ss(tS, sdesc_sw128(q0 + (h * nsub + xh) * kQSub + off, 16, 1024),
-                           sdesc_sw128(k0s + (ks * nsub + xh) * kKVSub + off, 16, 1024), idS,
-                           kk > 0);
+            const uint64_t dK = dK0 + (uint64_t)((uint32_t)(ks * nsub) * (kKVSub >> 4));
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              if (kk < dh / 16)
+                umma_bf16_ss(tS, dQ + (uint64_t)(((kk >> 2) * kQSub + (kk & 3) * 32) >> 4),
+                             dK + (uint64_t)(((kk >> 2) * kKVSub + (kk & 3) * 32) >> 4), idS,
+                             kk > 0);
             }
             umma_commit(&s_full[h]);
             umma_commit(&k_empty[ks]);
@@ -287,11 +284,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             return false;
           tc_fence_after();
           if (lane == 0) {
-            for (int kk = 0; kk < ksteps; ++kk) {
-              // V as an MN-major operand: 64-wide dh blocks kKVSub apart, 8-key groups 1 KB apart.
-              const uint64_t bd = sdesc_sw128(v0s + vs * nsub * kKVSub + kk * 2048, kKVSub, 1024);
-              // P of keys 0..63 sits in columns 0..31, of keys 64..127 in 64..95
-            umma_bf16_ts(tOh, tS + kk * 8 + (kk >= 4 ? 32 : 0), bd, idO, (t > 0 || kk > 0) ? 1u : 0u);
+            // V as an MN-major operand: 64-wide dh blocks kKVSub apart, 8-key
+            // groups 1 KB apart, 16 keys (2 KB) per MMA.  P of keys 0..63
+            // sits in columns 0..31, of keys 64..127 in columns 64..95.
+            const uint64_t dV = dV0 + (uint64_t)((uint32_t)(vs * nsub) * (kKVSub >> 4));
+#pragma unroll
+            for (int kk = 0; kk < kAttnBN / 16; ++kk) {
+              if (kk < ksteps)
+                umma_bf16_ts(tOh, tS + kk * 8 + (kk >= 4 ? 32 : 0), dV + (uint64_t)(kk * (2048 >> 4)),
+                             idO, (t > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&v_empty[vs]);
           }
@@ -309,27 +310,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
       }
     } else {
-      // ------------------------------------------------------- V cleaner
-      // The P.V MMA reads V rows up to the next multiple of 16 past the valid
-      // keys.  Those rows hold whatever the cache holds beyond the context
-      // (or an older tile's rows); P is zero there but 0 * NaN is NaN, so they
-      // are zeroed before either half's MMA may read the slot.
-      for (int t = 0; t < n_tiles; ++t) {
-        const int vs = t % kVSlots;
-        if (!mbar_wait(&v_full[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
-                       WHERE_ATTN_MMA))
-          break;
-        const int nvalid = tile_info(t, has_blk, k0, k1, a.S).nvalid;
-        const int pad = ((nvalid + 15) & ~15) - nvalid;
-        if (pad > 0) {
-          for (int xh = 0; xh < nsub; ++xh) {
-            uint4* dst = reinterpret_cast<uint4*>(sV + (vs * nsub + xh) * kKVSub + nvalid * 128);
-            for (int i = lane; i < pad * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+      // ------------------------------------------- TMA producer: V; V padding
+      // Lane 0 streams V (own loop, so K never waits for a V slot).  The
+      // P.V MMA reads V rows up to the next multiple of 16 past the valid
+      // keys; those rows hold whatever the cache holds beyond the context (or
+      // an older tile's rows), and P is zero there but 0 * NaN is NaN, so the
+      // warp zeroes them before either half's MMA may read the slot.  V(t) is
+      // issued before V(t-1) is cleaned, keeping two loads in flight.
+      if (lane == 0) prefetch_tmap(&tmVc);
+      const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
+      const int row_base = (b * a.Hkv + g) * a.L_cap;
+      for (int t = 0; t <= n_tiles; ++t) {
+        if (t < n_tiles) {
+          int good = 1;
+          if (lane == 0) {
+            const TileInfo ti = tile_info(t, has_blk, k0, k1, a.S);
+            const uint32_t bytes =
+                ti.is_blk ? (uint32_t)(nsub * a.S * 128) : (uint32_t)(nsub * kKVSub);
+            const int vs = t % kVSlots;
+            good = mbar_wait(&v_empty[vs], ((uint32_t)(t / kVSlots) & 1u) ^ 1u, a.err,
+                             abort_flag, WHERE_ATTN_PRODUCER);
+            if (good) {
+              uint8_t* dv = sV + vs * nsub * kKVSub;
+              mbar_arrive_expect_tx(&v_full[vs], bytes);
+              for (int xh = 0; xh < nsub; ++xh) {
+                if (ti.is_blk)
+                  tma_load_3d(dv + xh * kKVSub, &tmVb, &v_full[vs], xh * 64, g, b * a.S);
+                else
+                  tma_load_2d_hint(dv + xh * kKVSub, &tmVc, &v_full[vs], xh * 64,
+                                   row_base + ti.key0, pol_kv);
+              }
+            }
           }
-          fence_proxy_async_smem();
+          if (__shfl_sync(0xffffffffu, good, 0) == 0) break;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&v_ready[vs]);
+        if (t >= 1) {
+          const int tc = t - 1, vs = tc % kVSlots;
+          const bool landed = mbar_wait(&v_full[vs], (uint32_t)(tc / kVSlots) & 1u, a.err,
+                                        abort_flag, WHERE_ATTN_MMA);
+          if (!__all_sync(0xffffffffu, landed)) break;
+          const int nvalid = tile_info(tc, has_blk, k0, k1, a.S).nvalid;
+          const int pad = ((nvalid + 15) & ~15) - nvalid;
+          if (pad > 0) {
+            for (int xh = 0; xh < nsub; ++xh) {
+              uint4* dst = reinterpret_cast<uint4*>(sV + (vs * nsub + xh) * kKVSub + nvalid * 128);
+              for (int i = lane; i < pad * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&v_ready[vs]);
+        }
       }
     }
   } else {
@@ -516,8 +547,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
           }
         } else {
-          const size_t prow_i = (size_t)unit * 256 + wg * 128 + r;
-          float* po = a.part_o + prow_i * dh;
+          // Partial O is tile-major, [unit][dh/4][256 rows][4]: a warp's
+          // float4 store covers 32 consecutive rows, 512 contiguous bytes.
+          const int r256 = wg * 128 + r;
+          const size_t prow_i = (size_t)unit * 256 + r256;
+          float* po = a.part_o + (size_t)unit * dh * 256 + (size_t)r256 * 4;
           for (int c0 = 0; c0 < dh; c0 += 32) {
             uint32_t o[32];
             tmem_ld32(tOr + c0, o);
@@ -525,7 +559,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (valid) {
 #pragma unroll
               for (int v = 0; v < 8; ++v)
-                *reinterpret_cast<float4*>(po + c0 + 4 * v) =
+                *reinterpret_cast<float4*>(po + (size_t)(c0 / 4 + v) * 1024) =
                     make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
                                 __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
             }
@@ -547,72 +581,68 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-// One warp per query row: combine the splits' partials,
-//   O = sum_i 2^(m_i - m*) O_i / sum_i 2^(m_i - m*) l_i.
+// Thread per (query row, 4-column group): combine the splits' partials,
+//   O = sum_i 2^(m_i - m*) O_i / sum_i 2^(m_i - m*) l_i,
+// in one pass over the splits (running max, rescaled sums), four splits'
+// loads in flight before any is used.  Consecutive threads take consecutive
+// rows, so the tile-major partial reads are coalesced.  An empty split
+// (l = 0, O never written) is skipped by selection.
 __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a) {
   griddep_launch();
   griddep_wait();
   if (a.active != nullptr && *a.active == 0) return;
-  const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int total = a.B * a.Hkv * a.n_qtiles * 256;
-  if (gw >= total) return;
-  const int row256 = gw & 255;
-  const int pq = gw >> 8;  // pair * n_qtiles + qt
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int ngrp = a.dh / 4;
+  const int row256 = (int)(i & 255);
+  const int grp = (int)((i >> 8) % ngrp);
+  const int pq = (int)((i >> 8) / ngrp);  // pair * n_qtiles + qt
+  if (pq >= a.B * a.Hkv * a.n_qtiles) return;
   const int h = row256 >> 7, r = row256 & 127;
   if (h >= a.halves || r >= a.rows_per_half) return;
   const int pair = pq / a.n_qtiles, qt = pq % a.n_qtiles;
   const int b = pair / a.Hkv, g = pair % a.Hkv;
-  // One pass over the splits (running max, rescaled sums), four splits'
-  // loads in flight before any is used; an empty split (l = 0, O never
-  // written) is skipped by selection.
-  const size_t prow0 = (size_t)pq * a.n_splits * 256 + row256;
-  const int d0 = lane * 4;
-  const bool act = d0 < a.dh;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f, mrun = -INFINITY;
   for (int sp0 = 0; sp0 < a.n_splits; sp0 += 4) {
     float2 ml[4];
     float4 o[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const size_t prow = prow0 + (size_t)(sp0 + i) * 256;
-      const bool in = sp0 + i < a.n_splits;
-      ml[i] = in ? *reinterpret_cast<const float2*>(a.part_ml + prow * 2)
+    for (int k = 0; k < 4; ++k) {
+      const size_t pt = (size_t)pq * a.n_splits + sp0 + k;
+      const bool in = sp0 + k < a.n_splits;
+      ml[k] = in ? *reinterpret_cast<const float2*>(a.part_ml + (pt * 256 + row256) * 2)
                  : make_float2(-INFINITY, 0.f);
-      o[i] = in && act ? *reinterpret_cast<const float4*>(a.part_o + prow * a.dh + d0)
-                       : make_float4(0.f, 0.f, 0.f, 0.f);
+      o[k] = in ? *reinterpret_cast<const float4*>(a.part_o + ((pt * ngrp + grp) * 256 + row256) * 4)
+                : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (!(ml[i].y > 0.f)) continue;
-      if (ml[i].x > mrun) {
-        const float sc = mrun == -INFINITY ? 0.f : ex2(mrun - ml[i].x);
+    for (int k = 0; k < 4; ++k) {
+      if (!(ml[k].y > 0.f)) continue;
+      if (ml[k].x > mrun) {
+        const float sc = mrun == -INFINITY ? 0.f : ex2(mrun - ml[k].x);
         den *= sc;
         acc.x *= sc;
         acc.y *= sc;
         acc.z *= sc;
         acc.w *= sc;
-        mrun = ml[i].x;
+        mrun = ml[k].x;
       }
-      const float w = ex2(ml[i].x - mrun);
-      den += w * ml[i].y;
-      acc.x += w * o[i].x;
-      acc.y += w * o[i].y;
-      acc.z += w * o[i].z;
-      acc.w += w * o[i].w;
+      const float w = ex2(ml[k].x - mrun);
+      den += w * ml[k].y;
+      acc.x += w * o[k].x;
+      acc.y += w * o[k].y;
+      acc.z += w * o[k].z;
+      acc.w += w * o[k].w;
     }
   }
-  if (act) {
-    const float inv = 1.f / den;
-    const int s = qt * a.halves * a.s_per_half + h * a.s_per_half + r / a.G;
-    const int head = g * a.G + r % a.G;
-    uint16_t* dst = a.out + (size_t)(b * a.S + s) * a.ldo + head * a.dh + d0;
-    uint2 wv;
-    wv.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    wv.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(dst) = wv;
-  }
+  const float inv = 1.f / den;
+  const int s = qt * a.halves * a.s_per_half + h * a.s_per_half + r / a.G;
+  const int head = g * a.G + r % a.G;
+  uint16_t* dst = a.out + (size_t)(b * a.S + s) * a.ldo + head * a.dh + grp * 4;
+  uint2 wv;
+  wv.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+  wv.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+  *reinterpret_cast<uint2*>(dst) = wv;
 }
 
 }  // namespace
@@ -631,8 +661,8 @@ cudaError_t launch_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKc, const C
 }
 
 cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t st) {
-  const long long warps = (long long)a.B * a.Hkv * a.n_qtiles * 256;
-  const int blocks = (int)((warps * 32 + 255) / 256);
+  const long long threads = (long long)a.B * a.Hkv * a.n_qtiles * 256 * (a.dh / 4);
+  const int blocks = (int)((threads + 255) / 256);
   return launch_k(attn_merge_kernel, dim3(blocks), dim3(256), 0, st, a);
 }
 

@@ -8,11 +8,14 @@
 //  * the linear update [q|k|v] = e . U of the block loop, plain bf16 store.
 //
 // Layout: A [M, K] and B [N, K] are K-major bf16, loaded by TMA in 128-byte
-// swizzled 64-column boxes (A: 128 rows, B: 256 rows per stage).  One CTA per
-// SM walks tiles m-fastest, so the CTAs that share a W tile run together and
-// W crosses HBM once.  Warp 0 issues TMA, warp 1 issues tcgen05.mma
-// (M=128, N=256, K=16) into one of two 256-column TMEM accumulators, warps
-// 2..5 drain the other accumulator (TMEM lane = tile row).
+// swizzled 64-column boxes (A: 128 rows, B: BN rows per stage; BN = 224 for
+// the vocabulary, 128 for the linear update).  One CTA per SM walks tiles
+// m-fastest, so the CTAs that share a W tile run together and W crosses HBM
+// once.  Warp 0 issues TMA, warp 1 issues tcgen05.mma (M=128, N=BN, K=16)
+// into one of two BN-column TMEM accumulators, warps 2..5 drain the other
+// accumulator (TMEM lane = tile row).  With few rows the linear update is
+// split over K so every SM streams part of U; the fp32 partial tiles are
+// summed by splitk_reduce_kernel.
 #include <math.h>
 
 #include "tt_ptx.cuh"
@@ -230,23 +233,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&acce[acc]);
       } else {
-        // split-K: store this K range's fp32 partial tile
+        // split-K: store this K range's fp32 partial tile in tile-major
+        // order [chunk][4-column group][row][4], so each warp store covers
+        // 32 consecutive rows = 512 contiguous bytes.
         const int ks = u - tile * ksplit;
-        float* prow = a.partial + ((size_t)ks * a.M_alloc + row) * a.N + n * BN;
+        float* ptile = a.partial + (((size_t)ks * num_m + m) * num_n + n) * (size_t)(BN * kGemmBM);
+        const int r = q * 32 + lane;
         for (int ch = 0; ch < nchunks; ++ch) {
-          uint32_t r[32];
-          tmem_ld32(tbase + ch * 32, r);
+          uint32_t rr[32];
+          tmem_ld32(tbase + ch * 32, rr);
           tmem_wait_ld();
-          if (row < M) {
-            const int lim = ncols - ch * 32;
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              if (v * 4 < lim)
-                __stcg(reinterpret_cast<float4*>(prow + ch * 32 + 4 * v),
-                       make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3])));
-            }
-          }
+          for (int v = 0; v < 8; ++v)
+            __stcg(reinterpret_cast<float4*>(ptile + ((size_t)(ch * 8 + v) * kGemmBM + r) * 4),
+                   make_float4(__uint_as_float(rr[4 * v]), __uint_as_float(rr[4 * v + 1]),
+                               __uint_as_float(rr[4 * v + 2]), __uint_as_float(rr[4 * v + 3])));
         }
         tc_fence_before();
         __syncwarp();
@@ -265,23 +266,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// Sum of the split-K partials (tile-major, as the split-K epilogue stores
+// them) to bf16 C.  Thread = (tile, 32-column chunk, 8-column group, row):
+// its reads are coalesced across the warp's consecutive rows.
+template <int BN>
 __global__ void __launch_bounds__(256)
     splitk_reduce_kernel(const float* __restrict__ partial, int ksplit, int rows, int N,
                          uint16_t* __restrict__ C, int ldc, const int* active) {
   griddep_launch();
   griddep_wait();
   if (active != nullptr && *active == 0) return;
-  const int per_row = N / 8;
+  const int num_m = (rows + kGemmBM - 1) / kGemmBM, num_n = (N + BN - 1) / BN;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= (long long)rows * per_row) return;
-  const int row = (int)(i / per_row), c8 = (int)(i % per_row) * 8;
-  const size_t plane = (size_t)rows * N;
-  const float* p = partial + (size_t)row * N + c8;
+  const int r = (int)(i % kGemmBM);
+  long long rest = i / kGemmBM;
+  const int g8 = (int)(rest % (BN / 8));  // 8-column group within the tile
+  rest /= BN / 8;
+  const int n = (int)(rest % num_n), m = (int)(rest / num_n);
+  if (m >= num_m) return;
+  const int row = m * kGemmBM + r, col = n * BN + g8 * 8;
+  if (row >= rows || col >= N) return;
+  const size_t plane = (size_t)num_m * num_n * BN * kGemmBM;
+  // columns g8*8 .. +7 are the 4-column groups 2*g8 and 2*g8+1 of the tile
+  const float* p = partial + ((size_t)m * num_n + n) * (size_t)(BN * kGemmBM) +
+                   ((size_t)(2 * g8) * kGemmBM + r) * 4;
   float4 x0 = __ldcg(reinterpret_cast<const float4*>(p));
-  float4 x1 = __ldcg(reinterpret_cast<const float4*>(p + 4));
+  float4 x1 = __ldcg(reinterpret_cast<const float4*>(p + kGemmBM * 4));
   for (int k = 1; k < ksplit; ++k) {
     const float4 y0 = __ldcg(reinterpret_cast<const float4*>(p + k * plane));
-    const float4 y1 = __ldcg(reinterpret_cast<const float4*>(p + k * plane + 4));
+    const float4 y1 = __ldcg(reinterpret_cast<const float4*>(p + k * plane + kGemmBM * 4));
     x0.x += y0.x; x0.y += y0.y; x0.z += y0.z; x0.w += y0.w;
     x1.x += y1.x; x1.y += y1.y; x1.z += y1.z; x1.w += y1.w;
   }
@@ -290,7 +303,7 @@ __global__ void __launch_bounds__(256)
   w.y = pack_bf16x2(x0.z, x0.w);
   w.z = pack_bf16x2(x1.x, x1.y);
   w.w = pack_bf16x2(x1.z, x1.w);
-  *reinterpret_cast<uint4*>(C + (size_t)row * ldc + c8) = w;
+  *reinterpret_cast<uint4*>(C + (size_t)row * ldc + col) = w;
 }
 
 template <int EPI, int BN, int STAGES>
@@ -319,9 +332,10 @@ cudaError_t launch_gemm_bf16(const CUtensorMap& tmA, const CUtensorMap& tmB, con
 
 cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int N, uint16_t* C,
                                  int ldc, const int* active, cudaStream_t st) {
-  const long long threads = (long long)rows * (N / 8);
-  return launch_k(splitk_reduce_kernel, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st,
-                  partial, ksplit, rows, N, C, ldc, active);
+  const long long tiles = (long long)((rows + kGemmBM - 1) / kGemmBM) * ((N + kQkvBN - 1) / kQkvBN);
+  const long long threads = tiles * (kQkvBN / 8) * kGemmBM;
+  return launch_k(splitk_reduce_kernel<kQkvBN>, dim3((unsigned)((threads + 255) / 256)), dim3(256),
+                  0, st, partial, ksplit, rows, N, C, ldc, active);
 }
 
 }  // namespace tt

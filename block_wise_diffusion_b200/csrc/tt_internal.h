@@ -45,7 +45,7 @@ enum WhereTag {
 // a 5-deep ring; the linear update uses 256-column tiles with a 4-deep ring.
 constexpr int kGemmBM = 128, kGemmBK = 64;
 constexpr int kVocabBN = 224, kVocabStages = 5;
-constexpr int kQkvBN = 256, kQkvStages = 4;
+constexpr int kQkvBN = 128, kQkvStages = 6;
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr size_t gemm_smem_bytes(int bn, int stages) {
   return (size_t)stages * (kGemmBM + bn) * kGemmBK * 2 + 1024 + 256;
@@ -97,12 +97,13 @@ struct AttnArgs {
   int halves;           // 128-row halves per query tile and CTA (1 or 2)
   int n_qtiles;         // CTAs along the query axis per (b, g)
   int n_splits;         // key splits
-  int chunk;            // context keys per split (multiple of kAttnBN)
+  int chunk;            // context keys per split > 0 (multiple of kAttnBN)
+  int first;            // context keys of split 0, which also runs the block's own tile
   float scale_log2;     // log2(e) / sqrt(dh)
   uint16_t* out;        // bf16 [B*S, ldo]
   int ldo;
   int kv_keep;          // 1: load K/V with evict-last (small cache re-read every step)
-  float* part_o;        // [units][256][dh] unnormalised partial outputs
+  float* part_o;        // [units][dh/4][256 rows][4] unnormalised partial outputs
   float* part_ml;       // [units][256][2] (running max in log2 units, sum)
   int* err;
 };

@@ -145,6 +145,59 @@ __device__ __forceinline__ void adaln_finish(float (&v)[kAdaMaxVec][8], float s,
   }
 }
 
+// As adaln_finish, for rows held as 4-column groups: group k of this thread
+// covers columns i0[k]..i0[k]+3 (gin[k] false: no group).
+template <int KG>
+__device__ __forceinline__ void adaln_finish_groups(float (&v)[KG][4], const bool (&gin)[KG],
+                                                    const int (&i0)[KG], float s, int H, float tb,
+                                                    const uint16_t* __restrict__ ss,
+                                                    uint16_t* __restrict__ yrow, float* red) {
+  uint2 a0[KG], a1[KG];  // shift/scale loads are issued before the reductions
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    if (gin[k]) {
+      a0[k] = *reinterpret_cast<const uint2*>(ss + i0[k]);
+      a1[k] = *reinterpret_cast<const uint2*>(ss + H + i0[k]);
+    }
+  }
+  const float mean = block_sum(s, red) / (float)H;
+  float q = 0.f;
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    if (gin[k]) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float d = v[k][e] - mean;
+        q += d * d;
+      }
+    }
+  }
+  const float var = block_sum(q, red) / (float)H;
+  const float rstd = rsqrtf(var + 1e-6f);
+  const float lw = -13.287712379549449f / (float)H;  // -log2(10000) / H
+#pragma unroll
+  for (int k = 0; k < KG; ++k) {
+    if (!gin[k]) continue;
+    const uint32_t sh[2] = {a0[k].x, a0[k].y};
+    const uint32_t sc[2] = {a1[k].x, a1[k].y};
+    float out[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = i0[k] + e;
+      const float w = ex2((float)i * lw);
+      float sn, cs;
+      __sincosf(tb * w, &sn, &cs);  // |t w| <= 1: abs error ~1e-6, far below bf16 output
+      const uint32_t hs = (e & 1) ? (sh[e >> 1] & 0xffff0000u) : (sh[e >> 1] << 16);
+      const uint32_t hc = (e & 1) ? (sc[e >> 1] & 0xffff0000u) : (sc[e >> 1] << 16);
+      out[e] = (v[k][e] - mean) * rstd * (1.f + __uint_as_float(hc) + cs) + __uint_as_float(hs) + sn;
+    }
+    uint2 o;
+    o.x = pack_bf16x2(out[0], out[1]);
+    o.y = pack_bf16x2(out[2], out[3]);
+    *reinterpret_cast<uint2*>(yrow + i0[k]) = o;
+  }
+}
+
 // Block loop, one CTA per block row (all B*S rows are launched): decides
 // whether this CTA's row is still masked and, if so, its index j in the
 // compact list of masked rows (masked rows before it) and its sequence's
@@ -237,6 +290,9 @@ __global__ void __launch_bounds__(kAdaThreads)
 //   o = sum_i 2^(m_i - m*) O_i / sum_i 2^(m_i - m*) l_i,
 // rounded to bf16 (the attention output's storage precision), and the whole
 // row then goes through adaln_finish.
+// KG four-column groups per thread (H <= KG * 4 * kAdaThreads); NB splits'
+// loads in flight per round.
+template <int KG, int NB>
 __global__ void __launch_bounds__(kAdaThreads)
     merge_adaln_kernel(const AttnArgs a, const uint16_t* __restrict__ ss,
                        uint16_t* __restrict__ y, const uint8_t* __restrict__ masked,
@@ -254,81 +310,85 @@ __global__ void __launch_bounds__(kAdaThreads)
   const int sq = a.halves * a.s_per_half;
   const int qt = s / sq, within = s % sq;
   const int hh = within / a.s_per_half, sl = within % a.s_per_half;
-  const int nvec = H / 8;
-  // Each thread merges kAdaMaxVec 8-element vectors of the row in one pass
-  // over the splits (running max, rescaled sums), loading four splits' data
-  // for all its vectors before using any.  An empty split (l = 0, O never
-  // written) is skipped by selection.
-  size_t prow[kAdaMaxVec];  // partial row of split 0
-  int d0[kAdaMaxVec];
-  bool kin[kAdaMaxVec];
-  float mrun[kAdaMaxVec], den[kAdaMaxVec], v[kAdaMaxVec][8];
+  // Each thread merges up to KG four-column groups of the row in one pass
+  // over the splits (running max, rescaled sums), loading NB splits' data
+  // for all its groups before using any.  Group gi covers head
+  // gi % Hq, columns 4*(gi / Hq)..+3: consecutive threads take consecutive
+  // heads, i.e. consecutive rows of the tile-major partials (coalesced).  An
+  // empty split (l = 0, O never written) is skipped by selection.
+  constexpr int kG = KG;
+  const int ngrp = a.dh / 4, ng = a.Hq * ngrp;
+  size_t pt0[kG];  // partial tile of split 0
+  int r256[kG], grp[kG], i0[kG];
+  bool gin[kG];
+  float mrun[kG], den[kG], v[kG][4];
 #pragma unroll
-  for (int k = 0; k < kAdaMaxVec; ++k) {
-    kin[k] = (int)threadIdx.x + k * kAdaThreads < nvec;
-    const int vi = min((int)threadIdx.x + k * kAdaThreads, nvec - 1);
-    const int e0 = vi * 8, head = e0 / a.dh;
+  for (int k = 0; k < kG; ++k) {
+    const int gi = (int)threadIdx.x + k * kAdaThreads;
+    gin[k] = gi < ng;
+    const int gc = min(gi, ng - 1);
+    const int head = gc % a.Hq;
+    grp[k] = gc / a.Hq;
+    i0[k] = head * a.dh + grp[k] * 4;
     const int g = head / a.G, jh = head % a.G;
-    prow[k] = (size_t)((b * a.Hkv + g) * a.n_qtiles + qt) * a.n_splits * 256 + hh * 128 +
-              sl * a.G + jh;
-    d0[k] = e0 % a.dh;
+    pt0[k] = (size_t)((b * a.Hkv + g) * a.n_qtiles + qt) * a.n_splits;
+    r256[k] = hh * 128 + sl * a.G + jh;
     mrun[k] = -INFINITY;
     den[k] = 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[k][e] = 0.f;
+    for (int e = 0; e < 4; ++e) v[k][e] = 0.f;
   }
-  for (int sp0 = 0; sp0 < a.n_splits; sp0 += 4) {
-    float2 ml[4][kAdaMaxVec];
-    float4 x0[4][kAdaMaxVec], x1[4][kAdaMaxVec];
+  for (int sp0 = 0; sp0 < a.n_splits; sp0 += NB) {
+    float2 ml[NB][kG];
+    float4 x[NB][kG];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < NB; ++i) {
 #pragma unroll
-      for (int k = 0; k < kAdaMaxVec; ++k) {
-        if (sp0 + i < a.n_splits && kin[k]) {
-          const size_t pr = prow[k] + (size_t)(sp0 + i) * 256;
-          ml[i][k] = *reinterpret_cast<const float2*>(a.part_ml + pr * 2);
-          const float4* po = reinterpret_cast<const float4*>(a.part_o + pr * a.dh + d0[k]);
-          x0[i][k] = po[0];
-          x1[i][k] = po[1];
+      for (int k = 0; k < kG; ++k) {
+        if (sp0 + i < a.n_splits && gin[k]) {
+          const size_t pt = pt0[k] + sp0 + i;
+          ml[i][k] = *reinterpret_cast<const float2*>(a.part_ml + (pt * 256 + r256[k]) * 2);
+          x[i][k] = *reinterpret_cast<const float4*>(
+              a.part_o + ((pt * ngrp + grp[k]) * 256 + r256[k]) * 4);
         } else {
           ml[i][k] = make_float2(-INFINITY, 0.f);
         }
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < NB; ++i) {
 #pragma unroll
-      for (int k = 0; k < kAdaMaxVec; ++k) {
+      for (int k = 0; k < kG; ++k) {
         if (!(ml[i][k].y > 0.f)) continue;
         if (ml[i][k].x > mrun[k]) {
           const float sc = mrun[k] == -INFINITY ? 0.f : ex2(mrun[k] - ml[i][k].x);
           den[k] *= sc;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[k][e] *= sc;
+          for (int e = 0; e < 4; ++e) v[k][e] *= sc;
           mrun[k] = ml[i][k].x;
         }
         const float w = ex2(ml[i][k].x - mrun[k]);
         den[k] += w * ml[i][k].y;
-        v[k][0] += w * x0[i][k].x; v[k][1] += w * x0[i][k].y;
-        v[k][2] += w * x0[i][k].z; v[k][3] += w * x0[i][k].w;
-        v[k][4] += w * x1[i][k].x; v[k][5] += w * x1[i][k].y;
-        v[k][6] += w * x1[i][k].z; v[k][7] += w * x1[i][k].w;
+        v[k][0] += w * x[i][k].x;
+        v[k][1] += w * x[i][k].y;
+        v[k][2] += w * x[i][k].z;
+        v[k][3] += w * x[i][k].w;
       }
     }
   }
   float sum = 0.f;
 #pragma unroll
-  for (int k = 0; k < kAdaMaxVec; ++k) {
-    if (!kin[k]) continue;
+  for (int k = 0; k < kG; ++k) {
+    if (!gin[k]) continue;
     const float inv = 1.f / den[k];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
+    for (int e = 0; e < 4; ++e) {
       // the attention output is bf16 in the unfused path: round the same way
       v[k][e] = __uint_as_float(pack_bf16x2(v[k][e] * inv, 0.f) << 16);
       sum += v[k][e];
     }
   }
-  adaln_finish(v, sum, H, tb, ss, y + (size_t)j * H, red);
+  adaln_finish_groups<kG>(v, gin, i0, sum, H, tb, ss, y + (size_t)j * H, red);
 }
 
 // ---------------------------------------------------------------- gathers
@@ -507,12 +567,33 @@ __global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitAr
   }
   __syncthreads();
   // Loop only: a newly committed position's next embedding is Emb[token].
+  // All threads copy the committed rows together, eight 16-byte loads in
+  // flight per thread before any store.
   if (a.egath != nullptr) {
-    for (int s = warp; s < S; s += kCommitRows) {
-      if (!s_com[s]) continue;
-      const uint4* src = reinterpret_cast<const uint4*>(a.emb + (size_t)s_tok[s] * a.H);
-      uint4* dst = reinterpret_cast<uint4*>(a.egath + (size_t)(b * S + s) * a.H);
-      for (int i = lane; i < a.H / 8; i += 32) dst[i] = src[i];
+    const int nv = a.H / 8;  // 16-byte vectors per row
+    int nc = 0;
+    for (int s = 0; s < S; ++s) nc += s_com[s];
+    const long long total = (long long)nc * nv;
+    for (long long v0 = threadIdx.x; v0 < total; v0 += 8 * kCommitRows * 32) {
+      uint4 buf[8];
+      uint4* dst[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const long long v = v0 + (long long)k * kCommitRows * 32;
+        dst[k] = nullptr;
+        if (v < total) {
+          int c = (int)(v / nv), s = 0;
+          for (;; ++s) {  // the c-th committed position
+            if (s_com[s] && c-- == 0) break;
+          }
+          const int i = (int)(v % nv);
+          buf[k] = __ldg(reinterpret_cast<const uint4*>(a.emb + (size_t)s_tok[s] * a.H) + i);
+          dst[k] = reinterpret_cast<uint4*>(a.egath + (size_t)(b * S + s) * a.H) + i;
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (dst[k] != nullptr) *dst[k] = buf[k];
     }
   }
 }
@@ -559,7 +640,10 @@ cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const f
 cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, uint16_t* y,
                                const uint8_t* masked, int* rowlist, int* ctrl, cudaStream_t st) {
   const int rows = a.B * a.S;
-  return launch_k(merge_adaln_kernel, dim3(rows), dim3(kAdaThreads), 0, st, a, shift_scale, y,
+  if (a.Hq * a.dh <= 2 * 4 * kAdaThreads)
+    return launch_k(merge_adaln_kernel<2, 4>, dim3(rows), dim3(kAdaThreads), 0, st, a, shift_scale,
+                    y, masked, rowlist, ctrl);
+  return launch_k(merge_adaln_kernel<4, 2>, dim3(rows), dim3(kAdaThreads), 0, st, a, shift_scale, y,
                   masked, rowlist, ctrl);
 }
 

@@ -50,6 +50,17 @@ TIE_CONF_REL = 1e-3   # |conf - gamma| / gamma below this: threshold decision ex
 TIE_FALLBACK_REL = 1e-4  # fallback between confidences this close (relative): excluded
 
 
+# End-to-end loop comparison (teacher-forced on tokens and mask only): the
+# oracle recomputes attention and y in float64, so its logits differ from the
+# kernel's by the attention difference the parity bar allows, carried through
+# LayerNorm (unit-variance rows) and a W row of unit norm.  Measured attention
+# differences are a few 1e-3 relative, i.e. logit differences of order
+# 1e-3..1e-2 per unit of logit_scale.  A committed token may therefore be the
+# oracle's runner-up when the oracle's top-2 gap is below this (times
+# logit_scale); it must still be one of the oracle's two best tokens.
+LOOP_TIE_LOGIT = 2e-2
+
+
 def spec_excluded(conf, gap_p, gamma):
     return (np.abs(conf - gamma) < 1e-3) | (gap_p < 1e-3)
 

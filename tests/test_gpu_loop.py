@@ -58,6 +58,7 @@ def compare_teacher_forced(inp, g, gamma, logit_scale, bsel=None):
 
     r = O.denoise_block_loop(inp, gamma, logit_scale, max_steps=int(cs.max()) + 1, teacher=state)
     n_cmp = n_ex = 0
+    n_flip = [0]
     for k, st in enumerate(r["trace"]):
         tok_k, m_k = state(k)
         for b in range(m_k.shape[0]):
@@ -76,8 +77,19 @@ def compare_teacher_forced(inp, g, gamma, logit_scale, bsel=None):
                 continue
             n_cmp += 1
             np.testing.assert_array_equal(gpu_c, ora_c, err_msg=f"step {k} seq {b}")
-            np.testing.assert_array_equal(g["tokens"][b][gpu_c], st["tok"][b][ora_c],
-                                          err_msg=f"step {k} seq {b} tokens")
+            for s in np.flatnonzero(ora_c):
+                got, want = int(g["tokens"][b][s]), int(st["tok"][b][s])
+                if got == want:
+                    continue
+                # a flip between the oracle's two best tokens at a near tie
+                lg = O.logits(st["y"][b, s][None], O.from_bf16(inp["w"]), logit_scale)[0]
+                top2 = np.argsort(-lg, kind="stable")[:2]
+                gap = lg[top2[0]] - lg[top2[1]]
+                assert got in top2 and gap < G.LOOP_TIE_LOGIT * logit_scale, (
+                    f"step {k} seq {b} pos {s}: token {got}, oracle top-2 {top2} gap {gap:.3g}")
+                n_flip[0] += 1
+    if n_flip[0]:
+        print(f"near-tie top-2 flips: {n_flip[0]} of {n_cmp} compared sequence-steps")
     return n_cmp, n_ex
 
 
