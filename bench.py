@@ -258,20 +258,42 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------ GPU arm
-def algorithmic(kind, d, inp, m_rows_total, launches):
-    """(bound, algorithmic bytes or flops per launch, unit) of a kernel kind."""
-    n_vt = -(-d.V // 256)
+def algorithmic(kind, d, inp, m_per_launch, launches, peaks):
+    """(bound, algorithmic bytes or FLOPs per launch, unit, roofline time s) of a
+    kernel kind over its launches.
+
+    Each launch has algorithmic bytes and FLOPs; its floor is the larger of
+    bytes / HBM peak and FLOPs / sustained bf16 peak.  The bound reported is
+    the one whose floors dominate the sum over launches (the vocabulary GEMM
+    is HBM-bound at a few hundred rows and tensor-bound above; attention sits
+    at the ridge).  ``m_per_launch`` lists the vocabulary GEMM's rows per
+    launch (the still-masked positions of each step).
+    """
+    hbm = peaks["hbm_gbs"] * 1e9
+    tc = peaks["bf16_tflops_sustained"] * 1e12
     if kind == "gemm_vocab":
-        m_avg = m_rows_total / max(1, launches)
-        return "hbm", d.V * d.H * 2 + m_avg * (d.H * 2 + n_vt * 12), "GB/s"
-    if kind == "attn":
-        kv = 2 * d.Hkv * d.dh * 2 * float(np.sum(inp["ctx_len"]))
+        n_vt = -(-d.V // 224)
+        ms = list(m_per_launch)[:launches] or [0]
+        by = [d.V * d.H * 2 + m * (d.H * 2 + n_vt * 16) for m in ms]
+        fl = [2.0 * m * d.V * d.H for m in ms]
+    elif kind == "attn":
+        L = np.asarray(inp["ctx_len"], dtype=np.float64)
+        kv = 2 * d.Hkv * d.dh * 2 * float(L.sum())
         blk = d.B * d.S * (d.Hq + 2 * d.Hkv) * d.dh * 2 + d.B * d.S * d.H * 2
-        return "hbm", kv + blk, "GB/s"
-    if kind == "gemm_qkv":
+        by = [kv + blk] * launches
+        fl = [4.0 * d.S * d.Hq * d.dh * float((L + d.S).sum())] * launches
+    elif kind == "gemm_qkv":
         n_qkv = d.H + 2 * d.Hkv * d.dh
-        return "tensor", 2.0 * d.B * d.S * d.H * n_qkv, "TFLOP/s"
-    return None, None, None
+        by = [n_qkv * d.H * 2 + d.B * d.S * (d.H + n_qkv) * 2] * launches
+        fl = [2.0 * d.B * d.S * d.H * n_qkv] * launches
+    else:
+        return None, None, None, None
+    t_h = sum(b / hbm for b in by)
+    t_t = sum(f / tc for f in fl)
+    t_roof = sum(max(b / hbm, f / tc) for b, f in zip(by, fl))
+    if t_t > t_h:
+        return "tensor", sum(fl) / len(fl), "TFLOP/s", t_roof
+    return "hbm", sum(by) / len(by), "GB/s", t_roof
 
 
 def run_ours(args, rank, world, local):
@@ -395,19 +417,22 @@ def run_ours(args, rank, world, local):
     table = tt.profile_table()
     tt.tt_profile_enable(False)
     cs = commit_step.cpu().numpy()
-    m_rows_total = float((cs[inp["masked"].astype(bool)] + 1).sum())
+    m0 = inp["masked"].astype(bool)
+    # rows of the vocabulary GEMM at step k: positions still masked at its start
+    m_per_step = [int((m0 & (cs >= k)).sum()) for k in range(int(cs.max()) + 1)]
     peaks, peak_src = load_peaks()
     kernels = {}
     for kind, (kms, n) in sorted(table.items(), key=lambda kv: -kv[1][0]):
         e = {"launches": n, "total_ms": round(kms, 4), "avg_us": round(1e3 * kms / n, 2)}
-        bound, per, unit = algorithmic(kind, d, inp, m_rows_total, n)
+        bound, per, unit, t_roof = algorithmic(kind, d, inp, m_per_step, n, peaks)
         if bound is not None:
             ach = per / (kms / n / 1e3) / (1e9 if unit == "GB/s" else 1e12)
             pk = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops_sustained"]
-            e.update(bound=bound, achieved=round(ach, 2), unit=unit, frac=round(ach / pk, 4))
+            e.update(bound=bound, achieved=round(ach, 2), unit=unit, frac=round(ach / pk, 4),
+                     roofline_time_frac=round(t_roof / (kms / 1e3), 4))
         kernels[kind] = e
     dom = max(table, key=lambda k: table[k][0])
-    bound, per, unit = algorithmic(dom, d, inp, m_rows_total, table[dom][1])
+    bound, per, unit, t_roof = algorithmic(dom, d, inp, m_per_step, table[dom][1], peaks)
     roofline = None
     if bound is not None:
         avg_s = table[dom][0] / table[dom][1] / 1e3
@@ -417,7 +442,8 @@ def run_ours(args, rank, world, local):
                     "unit": unit, "frac": round(ach / pk, 4),
                     "traffic": committed_traffic(dom, args.workload),
                     "peak_source": f"{peak_src} ({'hbm_gbs' if bound == 'hbm' else 'bf16_tflops_sustained'})",
-                    "algorithmic_per_launch": per}
+                    "algorithmic_per_launch": per,
+                    "roofline_time_frac": round(t_roof / (table[dom][0] / 1e3), 4)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

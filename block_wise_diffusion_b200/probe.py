@@ -5,8 +5,9 @@ For profilers (ncu) and quick timing of a single stage outside the block loop:
     python -m block_wise_diffusion_b200.probe attn --workload long --B 2
     python -m block_wise_diffusion_b200.probe vocab --workload mid --V 65536
 
-Each call runs ``--calls`` times on the current stream, then checks the
-device status word.  Inputs come from ``tt_inputs`` (the same seeded
+The entry point runs once, then ``--calls`` more times on the current stream
+(``--time`` reports their mean with CUDA events), then the device status word
+is checked.  Inputs come from ``tt_inputs`` (the same seeded
 generator the tests and the benchmark use); nothing here computes a reference.
 """
 from __future__ import annotations
@@ -27,7 +28,8 @@ def _dev(bits):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
 
 
-def run_attn(d, calls: int) -> None:
+def setup_attn(d):
+    """Upload seeded inputs; return (call, check) for tt_block_denoise_attn."""
     import torch
     import tt_inputs
     import block_wise_diffusion_b200 as tt
@@ -37,13 +39,16 @@ def run_attn(d, calls: int) -> None:
     D = tt.dims(d)
     out = torch.empty((d.B, d.S, d.Hq, d.dh), dtype=torch.bfloat16, device="cuda")
     ws = tt.workspace(D, tt.TT_WS_ATTN)
-    for _ in range(calls):
+
+    def call():
         tt.tt_block_denoise_attn(D, q, kb, vb, kc, vc, cl, out, ws)
-    if tt.tt_device_status(ws) != 0:
-        raise RuntimeError("device reported an error")
+
+    return call, lambda: tt.tt_device_status(ws)
 
 
-def run_vocab(d, calls: int) -> None:
+def setup_vocab(d):
+    """Upload seeded inputs; return (call, check) for tt_vocab_confidence_commit
+    with every position masked (all B*S rows go through the GEMM)."""
     import torch
     import tt_inputs
     import block_wise_diffusion_b200 as tt
@@ -53,15 +58,18 @@ def run_vocab(d, calls: int) -> None:
     w = _dev(inp["w"])
     D = tt.dims(d)
     ws = tt.workspace(D, tt.TT_WS_VOCAB)
-    for _ in range(calls):
-        tok = torch.full((d.B, d.S), -1, dtype=torch.int32, device="cuda")
-        msk = torch.ones((d.B, d.S), dtype=torch.uint8, device="cuda")
-        conf = torch.empty((d.B, d.S), dtype=torch.float32, device="cuda")
-        am = torch.empty((d.B, d.S), dtype=torch.int32, device="cuda")
-        nc = torch.empty((d.B,), dtype=torch.int32, device="cuda")
+    tok = torch.full((d.B, d.S), -1, dtype=torch.int32, device="cuda")
+    msk0 = torch.ones((d.B, d.S), dtype=torch.uint8, device="cuda")
+    msk = msk0.clone()
+    conf = torch.empty((d.B, d.S), dtype=torch.float32, device="cuda")
+    am = torch.empty((d.B, d.S), dtype=torch.int32, device="cuda")
+    nc = torch.empty((d.B,), dtype=torch.int32, device="cuda")
+
+    def call():
+        msk.copy_(msk0)  # the call commits positions: start every call fully masked
         tt.tt_vocab_confidence_commit(D, y, w, 0.8, 1.0, tok, msk, conf, am, nc, ws)
-    if tt.tt_device_status(ws) != 0:
-        raise RuntimeError("device reported an error")
+
+    return call, lambda: tt.tt_device_status(ws)
 
 
 def main(argv=None) -> int:
@@ -73,6 +81,8 @@ def main(argv=None) -> int:
     p.add_argument("--B", type=int, default=None, help="override the batch")
     p.add_argument("--V", type=int, default=None, help="override the vocabulary (vocab stage)")
     p.add_argument("--calls", type=int, default=2)
+    p.add_argument("--time", action="store_true",
+                   help="report the mean time of the calls after the first (CUDA events)")
     a = p.parse_args(argv)
     over = {}
     if a.B is not None:
@@ -80,11 +90,21 @@ def main(argv=None) -> int:
     if a.V is not None:
         over["V"] = a.V
     d = tt_inputs.workload(a.workload, **over)
-    (run_attn if a.stage == "attn" else run_vocab)(d, a.calls)
+    call, check = (setup_attn if a.stage == "attn" else setup_vocab)(d)
+    call()  # warm-up
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(a.calls):
+        call()
+    ev[1].record()
     torch.cuda.synchronize()
-    print(f"ok {a.stage} {d}")
+    if check() != 0:
+        raise RuntimeError("device reported an error")
+    msg = f"ok {a.stage} {d}"
+    if a.time:
+        msg += f": {ev[0].elapsed_time(ev[1]) * 1e3 / a.calls:.1f} us per call (no L2 flush)"
+    print(msg)
     return 0
-
 
 if __name__ == "__main__":
     sys.exit(main())
