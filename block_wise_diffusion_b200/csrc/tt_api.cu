@@ -201,7 +201,15 @@ static AttnGeom attn_geom(const tt_dims& d) {
   n = std::min(std::min(n, ctx_tiles + 1), 64);
   // Split 0 also runs the block's own key tile, so it gets one context tile
   // fewer: every split then runs at most c tiles, c = ceil((tiles + 1) / n).
-  const int c = (ctx_tiles + 1 + n - 1) / n;
+  int c = (ctx_tiles + 1 + n - 1) / n;
+  if (forced <= 0 && units > kNumSMs) {
+    // More units than SMs: several waves whatever the split.  Context lengths
+    // differ per sequence (and live on the device), so cap a split at about
+    // an eighth of an SM's share of the largest possible work; the splits of
+    // short sequences that fall past their context exit at once.
+    const long long per_sm = units * (long long)(ctx_tiles + 1) / kNumSMs;
+    c = (int)std::min<long long>(c, std::max<long long>(8, (per_sm + 7) / 8));
+  }
   g.chunk = c * kAttnBN;
   g.first = (c - 1) * kAttnBN;
   n = 1 + (std::max(0, d.L_cap - g.first) + g.chunk - 1) / g.chunk;
