@@ -151,7 +151,9 @@ static tt_status check_dims(const tt_dims* d) {
   if (d->B < 1 || d->Hq < 1 || d->Hkv < 1 || d->V < 2 || d->L_cap < 0)
     return fail(TT_ERR_INVALID_ARG, "bad sizes: B=%d Hq=%d Hkv=%d V=%d L_cap=%d", d->B, d->Hq,
                 d->Hkv, d->V, d->L_cap);
-  if (d->S != 16 && d->S != 32) return fail(TT_ERR_UNSUPPORTED, "S=%d not in {16,32}", d->S);
+  // S = 1 is the autoregressive baseline step (one position per block)
+  if (d->S != 1 && d->S != 16 && d->S != 32)
+    return fail(TT_ERR_UNSUPPORTED, "S=%d not in {1,16,32}", d->S);
   if (d->dh != 64 && d->dh != 128)
     return fail(TT_ERR_UNSUPPORTED, "dh=%d not in {64,128}", d->dh);
   if (d->Hq % d->Hkv != 0)

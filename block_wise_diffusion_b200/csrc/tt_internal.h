@@ -145,7 +145,7 @@ cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_
                          const uint16_t* e_mask, uint16_t* dst, int rows, int H, int V,
                          const int* active, int* err, cudaStream_t st);
 
-// The commit runs as B*S/kCommitRows CTAs (one warp per block row); the
+// The commit runs as B*ceil(S/kCommitRows) CTAs (one warp per block row); the
 // last CTA of a sequence to finish (a per-sequence counter) applies the
 // commit rule to the whole sequence.
 constexpr int kCommitRows = 4;

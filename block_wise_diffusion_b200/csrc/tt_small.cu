@@ -448,14 +448,16 @@ __global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitAr
   __shared__ int s_tok[32];
   __shared__ int s_com[32];
   if (a.active != nullptr && *a.active == 0) return;
-  const int S = a.S, per_seq = S / kCommitRows;
+  const int S = a.S, per_seq = (S + kCommitRows - 1) / kCommitRows;
   const int b = blockIdx.x / per_seq;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = b * S + (blockIdx.x % per_seq) * kCommitRows + warp;
+  const int s_row = (blockIdx.x % per_seq) * kCommitRows + warp;
+  const bool row_ok = s_row < S;  // S < kCommitRows leaves warps without a row
+  const int row = b * S + min(s_row, S - 1);
   const int M = a.M_dev != nullptr ? *a.M_dev : a.B * S;
   float conf = -1.f;
   int tok = -1;
-  if (a.masked[row] != 0) {
+  if (row_ok && a.masked[row] != 0) {
     const int j = a.rowlist[a.B * S + row];  // this row's compact index
     if (j >= 0 && j < M) {
       // One pass over the row's tiles (lane t reads tiles t, t+32, ...):
@@ -501,7 +503,7 @@ __global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitAr
       tok = bt < a.n_vt ? btok : -1;
     }
   }
-  if (lane == 0) a.rowres[row] = make_float2(conf, __int_as_float(tok));
+  if (lane == 0 && row_ok) a.rowres[row] = make_float2(conf, __int_as_float(tok));
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
@@ -664,8 +666,8 @@ cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_
 }
 
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
-  return launch_k(commit_kernel, dim3(a.B * (a.S / kCommitRows)), dim3(kCommitRows * 32), 0, st,
-                  a);
+  const int per_seq = (a.S + kCommitRows - 1) / kCommitRows;
+  return launch_k(commit_kernel, dim3(a.B * per_seq), dim3(kCommitRows * 32), 0, st, a);
 }
 
 cudaError_t launch_selftest_wait(int* ctrl, unsigned long long limit_ns, cudaStream_t st) {

@@ -70,7 +70,7 @@ def test_workspace_sizes(L):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(S=8), 2), (dict(dh=96), 2), (dict(Hkv=3), 1), (dict(Hq=24, Hkv=2), 2),
+    (dict(S=8), 2), (dict(S=2), 2), (dict(dh=96), 2), (dict(Hkv=3), 1), (dict(Hq=24, Hkv=2), 2),
     (dict(H=1000), 1), (dict(B=0), 1), (dict(V=1), 1), (dict(L_cap=-1), 1),
 ])
 def test_bad_dims_rejected(L, kw, code):

@@ -58,6 +58,9 @@ CASES = [
                                  ctx=("fixed", 513)), np.array([513, 129]), True),
     ("mha-like-g2", tt_inputs.Dims(B=2, S=16, Hq=4, Hkv=2, dh=128, V=512, L_cap=200,
                                    ctx=("fixed", 200)), np.array([1, 200]), False),
+    # autoregressive baseline step: one block position, M = G query rows
+    ("ar-S1", tt_inputs.workload("mid", B=3, S=1, L_cap=700, ctx=("fixed", 700), V=1024),
+     np.array([700, 129, 0]), True),
 ]
 
 

@@ -121,6 +121,18 @@ def test_loop_tiny(gamma, logit_scale):
     assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
 
 
+@pytest.mark.parametrize("logit_scale", [1.0, 12.0])
+def test_loop_autoregressive_step_s1(logit_scale):
+    """S = 1: every call commits the block's single position in one step."""
+    d = tt_inputs.workload("mid", B=4, S=1, L_cap=300, ctx=("fixed", 300), V=1024)
+    inp = tt_inputs.generate(d, seed=41)
+    g = run_loop_gpu(d, inp, 0.8, logit_scale)
+    check_invariants(d, inp, g)
+    assert g["steps_run"] == 1 and np.all(g["steps_taken"] == 1)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale)
+    assert n_cmp + n_ex == d.B and n_ex <= 1, (n_cmp, n_ex)
+
+
 def test_loop_canonical_scale_commits_in_position_order():
     d = tt_inputs.workload("tiny", B=2)
     inp = tt_inputs.generate(d, seed=32)

@@ -339,3 +339,33 @@ def test_loop_multi_commit_and_resume():
     inp2 = dict(inp, tokens=r1["tokens"], masked=r1["masked"].astype(np.uint8))
     r2 = O.denoise_block_loop(inp2, gamma=0.5, logit_scale=40.0)
     np.testing.assert_array_equal(r2["tokens"], r["tokens"])
+
+
+def test_loop_autoregressive_s1_single_step():
+    """S = 1 (the autoregressive baseline): the loop takes exactly one step,
+    t = 1, and commits the argmax of that step's logits, whose attention is
+    one softmax over the context keys and the position's own key."""
+    d = tt_inputs.Dims(B=3, S=1, Hq=4, Hkv=1, dh=64, V=1024, L_cap=64, ctx=("fixed", 64))
+    inp = tt_inputs.generate(d, seed=5)
+    r = O.denoise_block_loop(inp, gamma=0.8)
+    assert len(r["trace"]) == 1
+    st = r["trace"][0]
+    np.testing.assert_array_equal(r["steps_taken"], [1, 1, 1])
+    np.testing.assert_array_equal(r["commit_step"], np.zeros((3, 1), dtype=r["commit_step"].dtype))
+    np.testing.assert_array_equal(st["t"], [1.0, 1.0, 1.0])
+    np.testing.assert_array_equal(r["tokens"][:, 0], st["tok"][:, 0])
+    # the attention of that step, by explicit loops over the L + 1 keys
+    f = O.from_bf16
+    e = O.embed_block(inp["tokens"], inp["masked"], inp["emb"], inp["e_mask"])
+    q, k, v = O.linear_update(e, f(inp["u_t"]), d.Hq, d.Hkv, d.dh)
+    kc, vc = f(inp["k_ctx"]), f(inp["v_ctx"])
+    for b in range(d.B):
+        for h in range(d.Hq):
+            keys = [kc[b, 0, j] for j in range(d.L_cap)] + [k[b, 0, 0]]
+            vals = [vc[b, 0, j] for j in range(d.L_cap)] + [v[b, 0, 0]]
+            sc = [float(np.dot(q[b, 0, h], kk)) / np.sqrt(d.dh) for kk in keys]
+            mx = max(sc)
+            w = [np.exp(x - mx) for x in sc]
+            o = sum(wi * vi for wi, vi in zip(w, vals)) / sum(w)
+            np.testing.assert_allclose(st["o"][b, 0, h * d.dh:(h + 1) * d.dh],
+                                       O.round_bf16(o), rtol=0, atol=2 ** -8 * np.abs(o).max())

@@ -99,6 +99,9 @@ WORKLOADS = {
                      ctx=("uniform", 512, 32768), precommit=("uniform", 0.0, 0.75)),
     "ragged32": Dims(B=128, S=32, Hq=32, Hkv=2, dh=128, V=131072, L_cap=32768,
                      ctx=("uniform", 512, 32768), precommit=("uniform", 0.0, 0.75)),
+    # autoregressive baseline at the mid shapes: one position per block (S = 1),
+    # the same denoiser step; the denominator of a block-vs-AR throughput ratio
+    "mid_ar": _fixed(8, 1, 32, 2, 128, 131072, 4096),
 }
 
 
