@@ -152,8 +152,8 @@ static tt_status check_dims(const tt_dims* d) {
     return fail(TT_ERR_INVALID_ARG, "bad sizes: B=%d Hq=%d Hkv=%d V=%d L_cap=%d", d->B, d->Hq,
                 d->Hkv, d->V, d->L_cap);
   // S = 1 is the autoregressive baseline step (one position per block)
-  if (d->S != 1 && d->S != 16 && d->S != 32)
-    return fail(TT_ERR_UNSUPPORTED, "S=%d not in {1,16,32}", d->S);
+  if (d->S != 1 && d->S != 16 && d->S != 32 && d->S != 64 && d->S != 128)
+    return fail(TT_ERR_UNSUPPORTED, "S=%d not in {1,16,32,64,128}", d->S);
   if (d->dh != 64 && d->dh != 128)
     return fail(TT_ERR_UNSUPPORTED, "dh=%d not in {64,128}", d->dh);
   if (d->Hq % d->Hkv != 0)

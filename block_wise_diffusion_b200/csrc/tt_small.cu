@@ -445,8 +445,10 @@ __global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitAr
   griddep_launch();
   griddep_wait();
   __shared__ int s_last;
-  __shared__ int s_tok[32];
-  __shared__ int s_com[32];
+  __shared__ int s_tok[kCommitRows * 32];
+  __shared__ int s_com[kCommitRows * 32];
+  __shared__ float s_bc[kCommitRows];
+  __shared__ int s_bs[kCommitRows];
   if (a.active != nullptr && *a.active == 0) return;
   const int S = a.S, per_seq = (S + kCommitRows - 1) / kCommitRows;
   const int b = blockIdx.x / per_seq;
@@ -512,25 +514,26 @@ __global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitAr
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  if (warp == 0) {
-    const int s = lane;
+  {
+    // One thread per position of sequence b (S <= kCommitRows * 32).
+    const int s = threadIdx.x;
     const bool in = s < S;
-    const int r = b * S + s;
+    const int r = b * S + min(s, S - 1);
     const int is_m = in ? a.masked[r] != 0 : 0;
     const float2 rr = in ? __ldcg(a.rowres + r) : make_float2(-1.f, __int_as_float(-1));
     float cf = rr.x;
     const int tk = __float_as_int(rr.y);
     const bool bad = is_m && !(cf >= 0.f && cf <= 1.0001f);  // NaN or impossible value
-    if (__any_sync(0xffffffffu, bad) && lane == 0) {
+    if (__syncthreads_or(bad) && threadIdx.x == 0) {
       atomicCAS(a.ctrl + CTRL_ERR, 0, (int)TT_ERR_INTERNAL);
       atomicCAS(a.ctrl + CTRL_ERR_WHERE, 0, (int)WHERE_COMMIT_NAN);
     }
     if (bad) cf = -1.f;
     const bool qual = is_m && cf >= a.gamma && tk >= 0;
-    const unsigned qmask = __ballot_sync(0xffffffffu, qual);
-    const unsigned mmask = __ballot_sync(0xffffffffu, is_m != 0);
+    const int nqual = __syncthreads_count(qual);
+    const int nmask = __syncthreads_count(is_m != 0);
     bool commit = qual;
-    if (qmask == 0 && mmask != 0) {
+    if (nqual == 0 && nmask != 0) {  // uniform over the CTA
       // fallback: the most confident masked position, lowest s on ties
       float bc = is_m ? cf : -INFINITY;
       int bs = is_m ? s : 0x7fffffff;
@@ -542,27 +545,38 @@ __global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitAr
           bs = os;
         }
       }
+      if (lane == 0) {
+        s_bc[warp] = bc;
+        s_bs[warp] = bs;
+      }
+      __syncthreads();
+      for (int w = 0; w < kCommitRows; ++w) {
+        if (s_bc[w] > bc || (s_bc[w] == bc && s_bs[w] < bs)) {
+          bc = s_bc[w];
+          bs = s_bs[w];
+        }
+      }
       commit = is_m && s == bs;
     }
-    s_com[lane] = (in && commit) ? 1 : 0;
-    s_tok[lane] = tk >= 0 ? tk : 0;
+    s_com[s] = (in && commit) ? 1 : 0;
+    s_tok[s] = tk >= 0 ? tk : 0;
     if (in) {
       if (commit) {
-        a.tokens[r] = s_tok[lane];
+        a.tokens[r] = s_tok[s];
         a.masked[r] = 0;
         if (a.commit_step != nullptr) a.commit_step[r] = a.step;
       }
       if (a.conf_out != nullptr) a.conf_out[r] = is_m ? rr.x : -1.f;
       if (a.argmax_out != nullptr) a.argmax_out[r] = is_m ? tk : -1;
     }
-    const unsigned cmask = __ballot_sync(0xffffffffu, commit);
-    if (lane == 0) {
+    const int ncom = __syncthreads_count(in && commit);
+    if (threadIdx.x == 0) {
       a.seqcnt[b] = 0;  // ready for the next call
-      if (a.n_committed != nullptr) a.n_committed[b] = __popc(cmask);
-      if (a.steps_taken != nullptr && mmask != 0) a.steps_taken[b] = a.step + 1;
+      if (a.n_committed != nullptr) a.n_committed[b] = ncom;
+      if (a.steps_taken != nullptr && nmask != 0) a.steps_taken[b] = a.step + 1;
       if (a.plan_next) {
         // Loop: the remaining-masked counter is also the next step's active flag.
-        if (cmask) atomicSub(a.ctrl + CTRL_REMAINING, __popc(cmask));
+        if (ncom) atomicSub(a.ctrl + CTRL_REMAINING, ncom);
         if (b == 0) atomicAdd(a.ctrl + CTRL_STEPS_RUN, 1);
       }
     }

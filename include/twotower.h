@@ -27,8 +27,8 @@
  *  - Inputs are never modified, except `tokens` and `masked`, which are
  *    in/out state of the commit step and of the loop.
  *
- * Supported shapes: dh in {64, 128}; S in {1, 16, 32} (S = 1 is the
- * autoregressive baseline: one position per block); H == Hq*dh with H a
+ * Supported shapes: dh in {64, 128}; S in {1, 16, 32, 64, 128} (S = 1 is
+ * the autoregressive baseline: one position per block); H == Hq*dh with H a
  * multiple of 64, at most 8192; G = Hq/Hkv a power of two, at most 128; V >= 2;
  * B >= 1; 0 <= ctx_len[b] <= L_cap.  Other shapes return TT_ERR_UNSUPPORTED.
  */

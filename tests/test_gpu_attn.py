@@ -61,6 +61,11 @@ CASES = [
     # autoregressive baseline step: one block position, M = G query rows
     ("ar-S1", tt_inputs.workload("mid", B=3, S=1, L_cap=700, ctx=("fixed", 700), V=1024),
      np.array([700, 129, 0]), True),
+    # larger blocks: S = 128 is a whole key tile of block keys and 8 query tiles
+    ("block-S128", tt_inputs.workload("mid", B=2, S=128, L_cap=500, ctx=("fixed", 500), V=1024),
+     np.array([500, 77]), True),
+    ("block-S64-g4", tt_inputs.Dims(B=2, S=64, Hq=8, Hkv=2, dh=64, V=512, L_cap=300,
+                                    ctx=("fixed", 300)), np.array([300, 0]), True),
 ]
 
 

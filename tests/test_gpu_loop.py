@@ -133,6 +133,16 @@ def test_loop_autoregressive_step_s1(logit_scale):
     assert n_cmp + n_ex == d.B and n_ex <= 1, (n_cmp, n_ex)
 
 
+@pytest.mark.parametrize("S,logit_scale", [(128, 1.0), (128, 40.0), (64, 12.0)])
+def test_loop_larger_blocks(S, logit_scale):
+    d = tt_inputs.workload("tiny", B=2, S=S, precommit=("uniform", 0.0, 0.75))
+    inp = tt_inputs.generate(d, seed=43)
+    g = run_loop_gpu(d, inp, 0.8, logit_scale)
+    check_invariants(d, inp, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale)
+    assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
+
+
 def test_loop_canonical_scale_commits_in_position_order():
     d = tt_inputs.workload("tiny", B=2)
     inp = tt_inputs.generate(d, seed=32)
