@@ -342,6 +342,22 @@ def denoise_step(q, k, v, k_ctx, v_ctx, ctx_len, shift_scale, w_bits, tokens, ma
                 tokens=tokens2, masked=masked2, committed=committed, fallback=fallback)
 
 
+def denoiser_layers(x, layers, ctx_len, t, Hq, Hkv, dh):
+    """Every denoiser layer but the last, on all block rows (reading of the
+    layer-aligned attention of the Architecture section: each denoiser layer
+    attends to the context tower's KV of the same layer, with its own
+    adaLN-single table).  Layer l: [q|k|v] = x.U_l, o = attention over
+    [Kctx_l ; k], x <- adaLN_l(o, t), every stored tensor rounded to bf16.
+    ``layers`` is a list of (u_t, k_ctx, v_ctx, E) float64 tuples; x is
+    float64 [B,S,H]; t [B].  Returns the input of the last layer."""
+    B, S, H = x.shape
+    for u_t, kc, vc, E in layers:
+        q, k, v = linear_update(x, u_t, Hq, Hkv, dh)
+        o = round_bf16(block_attention(q, k, v, kc, vc, ctx_len)).reshape(B * S, H)
+        x = round_bf16(adaln_modulate(o, E, np.repeat(t, S))).reshape(B, S, H)
+    return x
+
+
 def denoise_block_loop(inp: dict, gamma: float, logit_scale: float = 1.0,
                        max_steps: int | None = None, teacher=None):
     """Refine one block until every position is committed (Generation Process).
@@ -349,9 +365,12 @@ def denoise_block_loop(inp: dict, gamma: float, logit_scale: float = 1.0,
     ``inp`` holds the bf16 bit arrays of tt_inputs (k_ctx, v_ctx, shift_scale,
     w, emb, e_mask, u_t) plus ctx_len, tokens, masked.  Each step: embed ->
     linear update -> attention -> adaLN -> vocab confidence -> commit, with
-    t_b recomputed from the mask.  ``teacher`` (optional callable step ->
-    (tokens, masked) or None) replaces the state at the start of a step, which
-    lets a test follow another implementation's trajectory step by step.
+    t_b recomputed from the mask.  With ``<name>_l`` arrays (several
+    denoiser layers, tt_inputs.generate(n_layers=...)) the layers before the
+    last run first (denoiser_layers) and the last one feeds the vocabulary.
+    ``teacher`` (optional callable step -> (tokens, masked) or None) replaces
+    the state at the start of a step, which lets a test follow another
+    implementation's trajectory step by step.
     Returns dict(tokens, masked, steps_taken [B], commit_step [B,S], trace).
     """
     tokens = np.array(inp["tokens"], dtype=np.int64, copy=True)
@@ -360,10 +379,17 @@ def denoise_block_loop(inp: dict, gamma: float, logit_scale: float = 1.0,
     Hkv, dh = inp["k_ctx"].shape[1], inp["k_ctx"].shape[3]
     H = inp["e_mask"].shape[0]
     Hq = H // dh
-    k_ctx = from_bf16(inp["k_ctx"])
-    v_ctx = from_bf16(inp["v_ctx"])
-    E = from_bf16(inp["shift_scale"])
-    u_t = from_bf16(inp["u_t"])
+    if "k_ctx_l" in inp:
+        n_layers = inp["k_ctx_l"].shape[0]
+        per = [tuple(from_bf16(inp[n + "_l"][i]) for n in ("u_t", "k_ctx", "v_ctx", "shift_scale"))
+               for i in range(n_layers)]
+        early, (u_t, k_ctx, v_ctx, E) = per[:-1], per[-1]
+    else:
+        early = []
+        k_ctx = from_bf16(inp["k_ctx"])
+        v_ctx = from_bf16(inp["v_ctx"])
+        E = from_bf16(inp["shift_scale"])
+        u_t = from_bf16(inp["u_t"])
     w = from_bf16(inp["w"])
     steps_taken = np.zeros(B, dtype=np.int64)
     commit_step = np.full((B, S), -1, dtype=np.int64)
@@ -379,6 +405,8 @@ def denoise_block_loop(inp: dict, gamma: float, logit_scale: float = 1.0,
             break
         active = masked.any(axis=1)
         e = embed_block(tokens, masked, inp["emb"], inp["e_mask"])
+        if early:
+            e = denoiser_layers(e, early, inp["ctx_len"], masked.sum(axis=1) / S, Hq, Hkv, dh)
         q, k, v = linear_update(e, u_t, Hq, Hkv, dh)
         r = denoise_step(q, k, v, k_ctx, v_ctx, inp["ctx_len"], E, w, tokens, masked,
                          gamma, logit_scale)

@@ -369,3 +369,87 @@ def test_loop_autoregressive_s1_single_step():
             o = sum(wi * vi for wi, vi in zip(w, vals)) / sum(w)
             np.testing.assert_allclose(st["o"][b, 0, h * d.dh:(h + 1) * d.dh],
                                        O.round_bf16(o), rtol=0, atol=2 ** -8 * np.abs(o).max())
+
+
+def _stack_one_layer(inp):
+    out = dict(inp)
+    for n in tt_inputs.LAYER_NAMES:
+        out[n + "_l"] = inp[n][None]
+    return out
+
+
+def test_layers_one_layer_stack_equals_single_layer_loop():
+    d, inp = _tiny_loop_inputs(B=2, precommit=("uniform", 0.0, 0.75))
+    a = O.denoise_block_loop(inp, 0.5, 40.0)
+    b = O.denoise_block_loop(_stack_one_layer(inp), 0.5, 40.0)
+    np.testing.assert_array_equal(a["tokens"], b["tokens"])
+    np.testing.assert_array_equal(a["commit_step"], b["commit_step"])
+
+
+def test_layers_depend_only_on_their_own_context():
+    d = tt_inputs.workload("tiny", B=2)
+    inp = tt_inputs.generate(d, seed=7, n_layers=2)
+    f = O.from_bf16
+    layers = [tuple(f(inp[n + "_l"][i]) for n in ("u_t", "k_ctx", "v_ctx", "shift_scale"))
+              for i in range(2)]
+    e = O.embed_block(inp["tokens"], inp["masked"], inp["emb"], inp["e_mask"])
+    t = inp["masked"].sum(axis=1) / d.S
+    x1 = O.denoiser_layers(e, layers[:1], inp["ctx_len"], t, d.Hq, d.Hkv, d.dh)
+    # layer 1's context has no effect on layer 0's output ...
+    bumped = list(layers)
+    bumped[1] = (layers[1][0], layers[1][1] + 1.0, layers[1][2] - 1.0, layers[1][3])
+    np.testing.assert_array_equal(
+        x1, O.denoiser_layers(e, bumped[:1], inp["ctx_len"], t, d.Hq, d.Hkv, d.dh))
+    # ... and layer 0's context beyond ctx_len has none either
+    kc = layers[0][1].copy()
+    kc[:, :, d.L_cap // 2:] = 0.0
+    short = np.full(d.B, d.L_cap // 2, dtype=np.int32)
+    half = [(layers[0][0], kc, layers[0][2], layers[0][3])]
+    np.testing.assert_array_equal(
+        O.denoiser_layers(e, layers[:1], short, t, d.Hq, d.Hkv, d.dh),
+        O.denoiser_layers(e, half, short, t, d.Hq, d.Hkv, d.dh))
+    # while the last layer's context does move the final confidences
+    r = O.denoise_block_loop(inp, 0.8, max_steps=1)
+    inp2 = dict(inp, v_ctx_l=inp["v_ctx_l"].copy())
+    inp2["v_ctx_l"][1] = tt_inputs.bf16_bits(-O.from_bf16(inp["v_ctx_l"][1]).astype(np.float32))
+    r2 = O.denoise_block_loop(inp2, 0.8, max_steps=1)
+    assert not np.allclose(r["trace"][0]["conf"], r2["trace"][0]["conf"])
+
+
+def test_layer_by_explicit_loops():
+    """One denoiser layer (all rows) against explicit loops: scores, softmax,
+    LayerNorm and the sinusoidal modulation written out element by element."""
+    d = tt_inputs.Dims(B=1, S=2, Hq=2, Hkv=1, dh=4, V=8, L_cap=3, ctx=("fixed", 3))
+    inp = tt_inputs.generate(d, seed=9, n_layers=2)
+    f = O.from_bf16
+    u, kc, vc, E = (f(inp[n + "_l"][0]) for n in ("u_t", "k_ctx", "v_ctx", "shift_scale"))
+    inp["masked"][0, 1] = 0
+    inp["tokens"][0, 1] = 5
+    e = O.embed_block(inp["tokens"], inp["masked"], inp["emb"], inp["e_mask"])
+    t = np.array([0.5])
+    got = O.denoiser_layers(e, [(u, kc, vc, E)], inp["ctx_len"], t, d.Hq, d.Hkv, d.dh)
+    H, dh = d.H, d.dh
+    for s in range(d.S):
+        row = [O.round_bf16(sum(e[0, s, i] * u[j, i] for i in range(H))) for j in range(u.shape[0])]
+        o = []
+        for h in range(d.Hq):
+            q = row[h * dh:(h + 1) * dh]
+            keys = [list(kc[0, 0, j]) for j in range(3)]
+            vals = [list(vc[0, 0, j]) for j in range(3)]
+            for s2 in range(d.S):
+                r2 = [O.round_bf16(sum(e[0, s2, i] * u[jj, i] for i in range(H)))
+                      for jj in range(u.shape[0])]
+                keys.append(r2[H:H + dh])
+                vals.append(r2[H + dh:H + 2 * dh])
+            sc = [sum(q[c] * kv[c] for c in range(dh)) / np.sqrt(dh) for kv in keys]
+            mx = max(sc)
+            w = [np.exp(x - mx) for x in sc]
+            o += [O.round_bf16(sum(w[j] * vals[j][c] for j in range(len(w))) / sum(w))
+                  for c in range(dh)]
+        mean = sum(o) / H
+        var = sum((x - mean) ** 2 for x in o) / H
+        for i in range(H):
+            om = 10000.0 ** (-i / H)
+            y = (o[i] - mean) / np.sqrt(var + 1e-6) * (1 + E[1, i] + np.cos(0.5 * om)) \
+                + E[0, i] + np.sin(0.5 * om)
+            assert abs(got[0, s, i] - O.round_bf16(y)) <= 2 ** -7 * max(1.0, abs(y)), (s, i)

@@ -146,14 +146,22 @@ def _normal_bf16(ss: np.random.SeedSequence, shape, scale: float, threads: int) 
     return out.reshape(shape)
 
 
+LAYER_NAMES = ("k_ctx", "v_ctx", "shift_scale", "u_t")
+
+
 def generate(d: Dims, seed: int = 0, *, sharp: bool = False, names=None,
-             threads: int | None = None) -> dict:
+             threads: int | None = None, n_layers: int = 1) -> dict:
     """Draw the inputs of one denoise-step problem.
 
     ``names`` restricts which large tensors are produced (the others are
     skipped but still consume their seed slot, so the bytes of every tensor
     are the same whatever subset is asked for).  ``sharp`` draws Q and K
     (block and context) unscaled, which makes attention far from uniform.
+
+    ``n_layers`` > 1 adds ``<name>_l`` arrays for the per-layer tensors
+    (context K/V, adaLN table, linear update) with a leading layer dimension;
+    layer 0 is the single-layer draw, layer i > 0 comes from its own
+    ``SeedSequence([seed, i])``.
     """
     if d.Hq % d.Hkv:
         raise ValueError("Hq must be a multiple of Hkv")
@@ -204,4 +212,15 @@ def generate(d: Dims, seed: int = 0, *, sharp: bool = False, names=None,
             masked[b, pos] = 0
     out["tokens"] = tokens
     out["masked"] = masked
+    if n_layers > 1:
+        for name in LAYER_NAMES:
+            if name not in want:
+                continue
+            shape, scale = shapes[name]
+            stack = np.empty((n_layers,) + shape, dtype=np.uint16)
+            stack[0] = out[name]
+            for i in range(1, n_layers):
+                lk = dict(zip(_STREAMS, np.random.SeedSequence([seed, i]).spawn(len(_STREAMS))))
+                stack[i] = _normal_bf16(lk[name], shape, float(scale), threads)
+            out[name + "_l"] = stack
     return out
