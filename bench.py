@@ -60,6 +60,8 @@ def parse_args(argv=None):
     p.add_argument("--logit-scale", type=float, default=1.0)
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--n-layers", type=int, default=1,
+                   help="denoiser layers per step (each with its own context KV)")
     a = p.parse_args(argv)
     if a.warmup < 3:
         p.error("--warmup must be >= 3")
@@ -101,7 +103,8 @@ def workload_config(d, args, world):
     return {
         "workload": (f"{args.workload}-block-loop: B={d.B} S={d.S} Hq={d.Hq} Hkv={d.Hkv} "
                      f"dh={d.dh} H={d.H} V={d.V} ctx={d.ctx} gamma={args.gamma} "
-                     f"logit_scale={args.logit_scale}"),
+                     f"logit_scale={args.logit_scale}"
+                     + (f" layers={args.n_layers}" if args.n_layers > 1 else "")),
         "global_batch": d.B * world,
         "seq_len": d.L_cap,
         "block_size": d.S,
@@ -207,6 +210,9 @@ def oracle_sample(d, inp, gamma, logit_scale, n_seq=3):
     one = dict(inp)
     for k in ("k_ctx", "v_ctx", "ctx_len", "tokens", "masked"):
         one[k] = inp[k][:n_seq]
+    for k in ("k_ctx_l", "v_ctx_l"):
+        if k in inp:
+            one[k] = inp[k][:, :n_seq]
     t0 = time.perf_counter()
     r = O.denoise_block_loop(one, gamma, logit_scale)
     dt = time.perf_counter() - t0
@@ -230,7 +236,7 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     d = tt_inputs.workload(args.workload)
-    inp = tt_inputs.generate(d, seed=rank_seed(args.seed, 0))
+    inp = tt_inputs.generate(d, seed=rank_seed(args.seed, 0), n_layers=args.n_layers)
     times, tokens, steps = [], 0, 0
     for i in range(args.warmup + args.steps):
         dt, c, s, _ = oracle_sample(d, inp, args.gamma, args.logit_scale, n_seq=1)
@@ -313,14 +319,16 @@ def run_ours(args, rank, world, local):
     d = tt_inputs.workload(args.workload)
     D = tt.dims(d)
     t0 = time.time()
-    inp = tt_inputs.generate(d, seed=rank_seed(args.seed, rank))
+    nl = args.n_layers
+    inp = tt_inputs.generate(d, seed=rank_seed(args.seed, rank), n_layers=nl)
     log(f"[rank {rank}] inputs generated in {time.time() - t0:.1f}s")
 
     def bf(k):
         return torch.from_numpy(inp[k].view(np.int16)).to(dev).view(torch.bfloat16)
 
     names = ["k_ctx", "v_ctx", "emb", "e_mask", "u_t", "shift_scale", "w"]
-    X = {k: bf(k) for k in names}
+    # with several layers the per-layer tensors are the stacked ones
+    X = {k: bf(k + "_l" if nl > 1 and k in tt_inputs.LAYER_NAMES else k) for k in names}
     ctx_len = torch.from_numpy(inp["ctx_len"]).to(dev)
     tokens0 = torch.from_numpy(inp["tokens"]).to(dev)
     masked0 = torch.from_numpy(inp["masked"]).to(dev)
@@ -333,12 +341,14 @@ def run_ours(args, rank, world, local):
     n_masked0 = int(inp["masked"].sum())
 
     def call(kc=None, vc=None, cl=None, tk=None, mk=None):
-        return tt.tt_denoise_block_loop(
-            D, kc if kc is not None else X["k_ctx"], vc if vc is not None else X["v_ctx"],
-            cl if cl is not None else ctx_len, X["emb"], X["e_mask"], X["u_t"],
-            X["shift_scale"], X["w"], args.gamma, args.logit_scale, d.S,
-            tk if tk is not None else tokens, mk if mk is not None else masked,
-            steps_taken, commit_step, ws, stream)
+        a = (kc if kc is not None else X["k_ctx"], vc if vc is not None else X["v_ctx"],
+             cl if cl is not None else ctx_len, X["emb"], X["e_mask"], X["u_t"],
+             X["shift_scale"], X["w"], args.gamma, args.logit_scale, d.S,
+             tk if tk is not None else tokens, mk if mk is not None else masked,
+             steps_taken, commit_step, ws, stream)
+        if nl > 1:
+            return tt.tt_denoise_block_loop_layers(D, nl, *a)
+        return tt.tt_denoise_block_loop(D, *a)
 
     def reset():
         tokens.copy_(tokens0)

@@ -258,6 +258,7 @@ struct Ws {
   float* part_ml = nullptr;
   float4* stats = nullptr;
   float* qkv_partial = nullptr;
+  uint16_t* xrows = nullptr;  // loop: one layer's modulated rows for the next layer
   int* seqcnt = nullptr;     // follows ctrl directly: cleared together
   float2* rowres = nullptr;
   size_t ctrl_clear = kCtrlBytes;  // bytes from ctrl to clear at the start of a call
@@ -291,6 +292,7 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
   if (which == TT_WS_LOOP) {
     const size_t n_qkv = (size_t)d.H + 2 * (size_t)d.Hkv * d.dh;
     w.egath = c.take<uint16_t>(rows * d.H * 2);
+    w.xrows = c.take<uint16_t>(rows * d.H * 2);
     w.qkv = c.take<uint16_t>(rows * n_qkv * 2);
     w.attn_out = c.take<uint16_t>(rows * d.H * 2);
     const int ks = qkv_ksplit(d);
@@ -588,13 +590,16 @@ tt_status tt_vocab_confidence_commit(const tt_dims* d, const tt_bf16* y, const t
   return TT_OK;
 }
 
-tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt_bf16* v_ctx,
-                                const int32_t* ctx_len, const tt_bf16* emb,
-                                const tt_bf16* e_mask, const tt_bf16* u_t,
-                                const tt_bf16* shift_scale, const tt_bf16* W, float gamma,
-                                float logit_scale, int32_t max_steps, int32_t* tokens,
-                                uint8_t* masked, int32_t* steps_taken, int32_t* commit_step,
-                                int32_t* steps_run, void* ws, size_t ws_bytes, void* stream) {
+// The block loop over n_layers denoiser layers (n_layers = 1: the
+// single-layer step).  Per-layer tensors are stacked with the layer index
+// outermost: k_ctx/v_ctx [n_layers][B,Hkv,L_cap,dh], u_t [n_layers][n_qkv,H],
+// shift_scale [n_layers][2,H].
+static tt_status denoise_block_loop_impl(
+    const tt_dims* d, int32_t n_layers, const tt_bf16* k_ctx, const tt_bf16* v_ctx,
+    const int32_t* ctx_len, const tt_bf16* emb, const tt_bf16* e_mask, const tt_bf16* u_t,
+    const tt_bf16* shift_scale, const tt_bf16* W, float gamma, float logit_scale,
+    int32_t max_steps, int32_t* tokens, uint8_t* masked, int32_t* steps_taken,
+    int32_t* commit_step, int32_t* steps_run, void* ws, size_t ws_bytes, void* stream) {
   TT_CHECK(check_dims(d));
   TT_CHECK(check_ptr(k_ctx, "k_ctx", true));
   TT_CHECK(check_ptr(v_ctx, "v_ctx", true));
@@ -608,6 +613,8 @@ tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt
   TT_CHECK(check_ptr(masked, "masked", false));
   TT_CHECK(check_ptr(steps_taken, "steps_taken", false));
   TT_CHECK(check_ptr(commit_step, "commit_step", false));
+  if (n_layers < 1 || n_layers > 64)
+    return fail(TT_ERR_INVALID_ARG, "n_layers=%d not in [1, 64]", n_layers);
   if (!(gamma > 0.f && gamma <= 1.f))
     return fail(TT_ERR_INVALID_ARG, "gamma=%g not in (0, 1]", (double)gamma);
   if (!(logit_scale > 0.f) || !std::isfinite(logit_scale))
@@ -620,14 +627,24 @@ tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt
   const int rows = d->B * d->S;
   const int n_qkv = d->H + 2 * d->Hkv * d->dh;
   const AttnGeom g = attn_geom(*d);
+  const size_t ctx_elems = (size_t)d->B * d->Hkv * d->L_cap * d->dh;
 
-  CUtensorMap tmE, tmU;
+  // Layer 0 reads the gathered embeddings, later layers the previous
+  // layer's modulated rows (every position of the block).
+  CUtensorMap tmE, tmX;
   if (!make_tmap_2d(&tmE, w.egath, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM) ||
-      !make_tmap_2d(&tmU, u_t, d->H, n_qkv, (uint64_t)d->H * 2, kGemmBK, kQkvBN))
+      !make_tmap_2d(&tmX, w.xrows, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM))
     return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
-  AttnMaps m;
-  TT_CHECK(build_attn_maps(*d, g, w.qkv, n_qkv, w.qkv + d->H, w.qkv + d->H + d->Hkv * d->dh,
-                           n_qkv, k_ctx, v_ctx, &m));
+  std::vector<CUtensorMap> tmU(n_layers);
+  std::vector<AttnMaps> maps(n_layers);
+  for (int l = 0; l < n_layers; ++l) {
+    if (!make_tmap_2d(&tmU[l], u_t + (size_t)l * n_qkv * d->H, d->H, n_qkv, (uint64_t)d->H * 2,
+                      kGemmBK, kQkvBN))
+      return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
+    TT_CHECK(build_attn_maps(*d, g, w.qkv, n_qkv, w.qkv + d->H, w.qkv + d->H + d->Hkv * d->dh,
+                             n_qkv, k_ctx + (size_t)l * ctx_elems, v_ctx + (size_t)l * ctx_elems,
+                             &maps[l]));
+  }
 
   TT_CUDA(cudaMemsetAsync(w.ctrl, 0, w.ctrl_clear, st));
   TT_LAUNCH(TT_K_INIT, st, launch_loop_init(d->B, d->S, steps_taken, commit_step, w.ctrl, st));
@@ -656,18 +673,27 @@ tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt
   TT_LAUNCH(TT_K_EMBED, st, launch_embed(tokens, masked, emb, e_mask, w.egath, rows, d->H, d->V,
                                          active, w.ctrl, st));
   for (int step = 0; step < max_steps; ++step) {
-    TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(tmE, tmU, ga, std::min(qkv_tiles, kNumSMs), st));
-    if (ga.ksplit > 1)
-      TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
-                                                        w.qkv, n_qkv, active, st));
-    TT_CHECK(run_attn(*d, g, m, ctx_len, w.attn_out, w, active, false, st));
-    if (g.n_splits > 1) {
-      const AttnArgs aa = attn_args(*d, g, ctx_len, w.attn_out, w, active);
-      TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, shift_scale, w.y_c, masked, w.rowlist,
-                                                   w.ctrl, st));
-    } else {
-      TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, shift_scale, nullptr, w.y_c, rows, d->S,
-                                             d->H, masked, w.rowlist, w.ctrl, active, st));
+    for (int l = 0; l < n_layers; ++l) {
+      const bool last = l == n_layers - 1;
+      const tt_bf16* ss = shift_scale + (size_t)l * 2 * d->H;
+      TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(l == 0 ? tmE : tmX, tmU[l], ga,
+                                                    std::min(qkv_tiles, kNumSMs), st));
+      if (ga.ksplit > 1)
+        TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
+                                                          w.qkv, n_qkv, active, st));
+      TT_CHECK(run_attn(*d, g, maps[l], ctx_len, w.attn_out, w, active, false, st));
+      // The last layer keeps the masked rows, compacted, for the vocabulary;
+      // earlier layers modulate every row (all positions are keys of the
+      // next layer).  A null row list selects the latter.
+      uint16_t* y = last ? w.y_c : w.xrows;
+      int* rl = last ? w.rowlist : nullptr;
+      if (g.n_splits > 1) {
+        const AttnArgs aa = attn_args(*d, g, ctx_len, w.attn_out, w, active);
+        TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, ss, y, masked, rl, w.ctrl, st));
+      } else {
+        TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, ss, nullptr, y, rows, d->S, d->H,
+                                               masked, rl, w.ctrl, active, st));
+      }
     }
     TT_CHECK(run_vocab_gemm(*d, w, W, logit_scale, w.ctrl + CTRL_M, active, w_keep_tiles, st));
     CommitArgs c = commit_args(*d, w, gamma, logit_scale, tokens, masked);
@@ -689,6 +715,32 @@ tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt
     return fail((tt_status)h[CTRL_ERR], "device reported %s at tag 0x%x",
                 tt_status_string((tt_status)h[CTRL_ERR]), h[CTRL_ERR_WHERE]);
   return TT_OK;
+}
+
+tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt_bf16* v_ctx,
+                                const int32_t* ctx_len, const tt_bf16* emb,
+                                const tt_bf16* e_mask, const tt_bf16* u_t,
+                                const tt_bf16* shift_scale, const tt_bf16* W, float gamma,
+                                float logit_scale, int32_t max_steps, int32_t* tokens,
+                                uint8_t* masked, int32_t* steps_taken, int32_t* commit_step,
+                                int32_t* steps_run, void* ws, size_t ws_bytes, void* stream) {
+  return denoise_block_loop_impl(d, 1, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale, W,
+                                 gamma, logit_scale, max_steps, tokens, masked, steps_taken,
+                                 commit_step, steps_run, ws, ws_bytes, stream);
+}
+
+tt_status tt_denoise_block_loop_layers(const tt_dims* d, int32_t n_layers, const tt_bf16* k_ctx,
+                                       const tt_bf16* v_ctx, const int32_t* ctx_len,
+                                       const tt_bf16* emb, const tt_bf16* e_mask,
+                                       const tt_bf16* u_t, const tt_bf16* shift_scale,
+                                       const tt_bf16* W, float gamma, float logit_scale,
+                                       int32_t max_steps, int32_t* tokens, uint8_t* masked,
+                                       int32_t* steps_taken, int32_t* commit_step,
+                                       int32_t* steps_run, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  return denoise_block_loop_impl(d, n_layers, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t,
+                                 shift_scale, W, gamma, logit_scale, max_steps, tokens, masked,
+                                 steps_taken, commit_step, steps_run, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

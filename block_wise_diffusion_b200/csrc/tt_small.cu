@@ -208,7 +208,10 @@ __device__ bool loop_row(const uint8_t* __restrict__ masked, int rows, int S, in
                          int* __restrict__ rowlist, int* __restrict__ ctrl, int* j_out,
                          float* tb_out) {
   __shared__ int cnt[3][kAdaThreads / 32];
-  if (masked[row] == 0) return false;
+  // rowlist == nullptr: every row (a denoiser layer before the last), at its
+  // own index, with nothing recorded
+  const bool all_rows = rowlist == nullptr;
+  if (!all_rows && masked[row] == 0) return false;
   const int b0 = (row / S) * S;
   int before = 0, total = 0, seq = 0;
   for (int i = threadIdx.x; i < rows; i += blockDim.x) {
@@ -235,12 +238,12 @@ __device__ bool loop_row(const uint8_t* __restrict__ masked, int rows, int S, in
     total += cnt[1][w];
     seq += cnt[2][w];
   }
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && !all_rows) {
     rowlist[before] = row;
     rowlist[rows + row] = before;
     if (before == 0) ctrl[CTRL_M] = total;
   }
-  *j_out = before;
+  *j_out = all_rows ? row : before;
   *tb_out = (float)seq / (float)S;
   return true;
 }

@@ -231,6 +231,37 @@ TT_API tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, c
                                 int32_t* steps_run, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The block loop over n_layers denoiser layers ("Architecture" of the
+ * gist.science summary: each denoiser layer attends to the frozen context
+ * tower's KV of the same layer; each has its own adaLN-single table).  One
+ * step: x_0 = the block's embeddings (every position); for each layer l,
+ * [q|k|v] = x_l.U_l, o = attention over [Kctx_l ; k] (as
+ * tt_block_denoise_attn), x_{l+1} = adaLN_l(o, t_b) for every position
+ * (bf16); the last layer's masked rows feed the vocabulary and the commit
+ * (as tt_denoise_block_loop).  n_layers = 1 is tt_denoise_block_loop.
+ *
+ *   n_layers    1 .. 64
+ *   k_ctx/v_ctx bf16 [n_layers][B, Hkv, L_cap, dh]   layer outermost
+ *   u_t         bf16 [n_layers][H + 2*Hkv*dh, H]
+ *   shift_scale bf16 [n_layers][2, H]
+ *   other arguments, ownership, workspace (TT_WS_LOOP) and errors as
+ *   tt_denoise_block_loop; n_layers outside 1..64 is TT_ERR_INVALID_ARG.
+ * The pages fix only the layer alignment; the composition
+ * x_{l+1} = adaLN_l(attention_l(x_l)) without a residual is this library's
+ * reading (one layer reduces to the single-layer step).
+ */
+TT_API tt_status tt_denoise_block_loop_layers(const tt_dims* d, int32_t n_layers,
+                                              const tt_bf16* k_ctx, const tt_bf16* v_ctx,
+                                              const int32_t* ctx_len, const tt_bf16* emb,
+                                              const tt_bf16* e_mask, const tt_bf16* u_t,
+                                              const tt_bf16* shift_scale, const tt_bf16* w,
+                                              float gamma, float logit_scale, int32_t max_steps,
+                                              int32_t* tokens, uint8_t* masked,
+                                              int32_t* steps_taken, int32_t* commit_step,
+                                              int32_t* steps_run, void* ws, size_t ws_bytes,
+                                              void* stream);
+
+/*
  * Allocation-free variant of tt_vocab_confidence_commit.
  * The paper has no counterpart: this entry point exists for callers that
  * cannot provide a workspace - code running inside another runtime's

@@ -114,6 +114,11 @@ def test_commit_and_loop_argument_checks(L):
         *([FAKE] * 4), None, FAKE, wsl, None)
     assert loop(0) == 1
     assert loop(2000) == 1
+    layers = lambda n: L.tt_denoise_block_loop_layers(
+        ctypes.byref(d), n, *([FAKE] * 8), ctypes.c_float(0.8), ctypes.c_float(1.0), 4,
+        *([FAKE] * 4), None, FAKE, wsl, None)
+    assert layers(0) == 1 and "n_layers" in tt.tt_last_error()
+    assert layers(65) == 1
 
 
 def test_split_knob(L):

@@ -36,10 +36,32 @@ def run_loop_gpu(d, inp, gamma, logit_scale, max_steps=None):
                 steps_run=n)
 
 
+def run_loop_layers_gpu(d, inp, n_layers, gamma, logit_scale, max_steps=None):
+    D = tt.dims(d)
+    dv = {k: G.dev_bf16(inp[k + "_l"] if n_layers > 1 else inp[k][None])
+          for k in ("k_ctx", "v_ctx", "shift_scale", "u_t")}
+    dv.update({k: G.dev_bf16(inp[k]) for k in ("w", "emb", "e_mask")})
+    tokens = G.dev(inp["tokens"])
+    masked = G.dev(inp["masked"])
+    steps_taken = torch.full((d.B,), -7, dtype=torch.int32, device="cuda")
+    commit_step = torch.full((d.B, d.S), -7, dtype=torch.int32, device="cuda")
+    ws = G.workspace(D, tt.TT_WS_LOOP)
+    n = tt.tt_denoise_block_loop_layers(
+        D, n_layers, dv["k_ctx"], dv["v_ctx"], G.dev(inp["ctx_len"]), dv["emb"], dv["e_mask"],
+        dv["u_t"], dv["shift_scale"], dv["w"], gamma, logit_scale, max_steps or d.S, tokens,
+        masked, steps_taken, commit_step, ws)
+    return dict(tokens=tokens.cpu().numpy(), masked=masked.cpu().numpy(),
+                steps_taken=steps_taken.cpu().numpy(), commit_step=commit_step.cpu().numpy(),
+                steps_run=n)
+
+
 def slice_batch(inp, bsel):
     out = dict(inp)
     for k in ("k_ctx", "v_ctx", "ctx_len", "tokens", "masked"):
         out[k] = inp[k][bsel]
+    for k in ("k_ctx_l", "v_ctx_l"):
+        if k in inp:
+            out[k] = inp[k][:, bsel]
     return out
 
 
@@ -177,4 +199,33 @@ def test_loop_full_mid_shape_sampled_sequences(logit_scale):
         assert g["steps_run"] == 16
     n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, bsel=np.array([0, 5]))
     print(f"mid loop scale={logit_scale}: compared {n_cmp} sequence-steps, excluded {n_ex}")
+    assert n_cmp > 0 and n_ex <= 2
+
+
+@pytest.mark.parametrize("n_layers,logit_scale", [(2, 1.0), (3, 40.0), (2, 12.0)])
+def test_loop_layers_tiny(n_layers, logit_scale):
+    d = tt_inputs.workload("tiny", B=3, precommit=("uniform", 0.0, 0.75))
+    inp = tt_inputs.generate(d, seed=47, n_layers=n_layers)
+    g = run_loop_layers_gpu(d, inp, n_layers, 0.8, logit_scale)
+    check_invariants(d, inp, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale)
+    assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
+
+
+def test_loop_layers_one_layer_is_the_single_layer_call():
+    d = tt_inputs.workload("tiny", B=2, precommit=("uniform", 0.0, 0.75))
+    inp = tt_inputs.generate(d, seed=48)
+    a = run_loop_gpu(d, inp, 0.5, 40.0)
+    b = run_loop_layers_gpu(d, inp, 1, 0.5, 40.0)
+    for k in ("tokens", "masked", "steps_taken", "commit_step"):
+        np.testing.assert_array_equal(a[k], b[k])
+
+
+def test_loop_layers_mid_shape_sampled_sequences():
+    d = tt_inputs.workload("mid")
+    inp = tt_inputs.generate(d, seed=2, n_layers=2)
+    g = run_loop_layers_gpu(d, inp, 2, 0.8, 8.0)
+    check_invariants(d, inp, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, 8.0, bsel=np.array([1, 6]))
+    print(f"mid 2-layer loop: compared {n_cmp} sequence-steps, excluded {n_ex}")
     assert n_cmp > 0 and n_ex <= 2
