@@ -1,5 +1,5 @@
 // Thin inline-PTX wrappers for the sm_100a features the kernels use:
-// mbarriers, TMA tensor loads (no multicast), tcgen05 MMA / TMEM and the
+// mbarriers, TMA tensor loads (each to its own CTA), tcgen05 MMA / TMEM and the
 // proxy fences between them.  Every wait is bounded: after ~2 s of global
 // time a wait gives up, records TT_ERR_TIMEOUT in the caller's error word,
 // raises the CTA's abort flag and returns false, so a wrong byte count or a

@@ -417,3 +417,67 @@ def denoise_block_loop(inp: dict, gamma: float, logit_scale: float = 1.0,
         trace.append(r)
     return dict(tokens=tokens, masked=masked, steps_taken=steps_taken,
                 commit_step=commit_step, trace=trace)
+
+
+# ---- outer block loop (Generation Process: the context tower updates after
+# each block commits, then the next block starts) ---------------------------
+def append_block(k_ctx, v_ctx, ctx_len, tokens, emb_bits, u_ctx):
+    """The committed block joins the context.  The frozen context tower is not
+    modelled: a seeded projection stands in for it (reading), [k | v] of
+    position s = Emb[token_s] . U_ctx^T, rounded to bf16 (stored), written at
+    context positions ctx_len[b] + s.  k_ctx/v_ctx float64 [B,Hkv,L_cap,dh]
+    (modified in place), u_ctx float64 [2*Hkv*dh, H].  Returns the new lengths.
+    """
+    B, S = tokens.shape
+    Hkv, dh = k_ctx.shape[1], k_ctx.shape[3]
+    e = np.stack([from_bf16(emb_bits[tokens[b]]) for b in range(B)])  # [B,S,H]
+    kv = round_bf16(e @ u_ctx.T)                                       # [B,S,2*Hkv*dh]
+    new_len = np.array(ctx_len, dtype=np.int64, copy=True)
+    for b in range(B):
+        L = int(ctx_len[b])
+        if L + S > k_ctx.shape[2]:
+            raise ValueError("context cache full")
+        for s in range(S):
+            k_ctx[b, :, L + s] = kv[b, s, :Hkv * dh].reshape(Hkv, dh)
+            v_ctx[b, :, L + s] = kv[b, s, Hkv * dh:].reshape(Hkv, dh)
+        new_len[b] = L + S
+    return new_len
+
+
+def decode_blocks(inp: dict, n_blocks: int, gamma: float, logit_scale: float = 1.0,
+                  teacher=None):
+    """n_blocks blocks one after the other (Generation Process): each block
+    starts fully masked, is refined to completion by denoise_block_loop, then
+    joins the context (append_block).  ``teacher`` (optional callable
+    block -> tokens [B,S] or None) replaces a block's committed tokens before
+    it joins the context, so a test can follow another implementation.
+    Returns dict(tokens [n_blocks,B,S], ctx_len, k_ctx, v_ctx (float64),
+    blocks: the per-block loop results)."""
+    B, S = inp["tokens"].shape
+    k_ctx = from_bf16(inp["k_ctx"])
+    v_ctx = from_bf16(inp["v_ctx"])
+    u_ctx = from_bf16(inp["u_ctx"])
+    ctx_len = np.array(inp["ctx_len"], dtype=np.int64, copy=True)
+    out_tokens, blocks = [], []
+    for j in range(n_blocks):
+        blk = dict(inp, k_ctx=_to_bits(k_ctx), v_ctx=_to_bits(v_ctx),
+                   ctx_len=ctx_len.astype(np.int32),
+                   tokens=np.full((B, S), -1, dtype=np.int32),
+                   masked=np.ones((B, S), dtype=np.uint8))
+        r = denoise_block_loop(blk, gamma, logit_scale)
+        tok = r["tokens"]
+        if teacher is not None:
+            t = teacher(j)
+            if t is not None:
+                tok = np.asarray(t, dtype=np.int64)
+        ctx_len = append_block(k_ctx, v_ctx, ctx_len, tok, inp["emb"], u_ctx)
+        out_tokens.append(tok)
+        blocks.append(r)
+    return dict(tokens=np.stack(out_tokens), ctx_len=ctx_len, k_ctx=k_ctx, v_ctx=v_ctx,
+                blocks=blocks)
+
+
+def _to_bits(x: np.ndarray) -> np.ndarray:
+    """float64 values that are exactly bf16 -> their bf16 bit patterns."""
+    u = x.astype(np.float32).view(np.uint32)
+    return (u >> 16).astype(np.uint16)

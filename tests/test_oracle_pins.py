@@ -453,3 +453,51 @@ def test_layer_by_explicit_loops():
             y = (o[i] - mean) / np.sqrt(var + 1e-6) * (1 + E[1, i] + np.cos(0.5 * om)) \
                 + E[0, i] + np.sin(0.5 * om)
             assert abs(got[0, s, i] - O.round_bf16(y)) <= 2 ** -7 * max(1.0, abs(y)), (s, i)
+
+
+def _blocks_inputs(seed=3, B=2, n_room=3):
+    d = tt_inputs.Dims(B=B, S=16, Hq=4, Hkv=1, dh=64, V=1024, L_cap=256 + 16 * n_room,
+                       ctx=("fixed", 256))
+    return d, tt_inputs.generate(d, seed=seed)
+
+
+def test_append_block_writes_the_projection_and_nothing_else():
+    d, inp = _blocks_inputs()
+    f = O.from_bf16
+    kc, vc, u = f(inp["k_ctx"]), f(inp["v_ctx"]), f(inp["u_ctx"])
+    kc0, vc0 = kc.copy(), vc.copy()
+    L = np.array([256, 100])
+    tok = np.arange(d.B * d.S).reshape(d.B, d.S) * 7 % d.V
+    new = O.append_block(kc, vc, L, tok, inp["emb"], u)
+    np.testing.assert_array_equal(new, L + d.S)
+    for b in range(d.B):
+        for s in (0, d.S - 1):
+            e = f(inp["emb"][tok[b, s]])
+            for c in (0, 17, d.dh - 1):
+                kk = sum(e[i] * u[c, i] for i in range(d.H))
+                vv = sum(e[i] * u[d.Hkv * d.dh + c, i] for i in range(d.H))
+                assert kc[b, 0, L[b] + s, c] == O.round_bf16(kk)
+                assert vc[b, 0, L[b] + s, c] == O.round_bf16(vv)
+    # outside [L_b, L_b + S) the cache is untouched
+    for b in range(d.B):
+        keep = np.ones(d.L_cap, bool)
+        keep[L[b]:L[b] + d.S] = False
+        np.testing.assert_array_equal(kc[b, :, keep], kc0[b, :, keep])
+        np.testing.assert_array_equal(vc[b, :, keep], vc0[b, :, keep])
+    with pytest.raises(ValueError):
+        O.append_block(kc, vc, np.array([d.L_cap - 3, 0]), tok, inp["emb"], u)
+
+
+def test_decode_blocks_first_block_is_the_block_loop_and_contexts_grow():
+    d, inp = _blocks_inputs()
+    r = O.decode_blocks(inp, 3, 0.8)
+    single = O.denoise_block_loop(inp, 0.8)
+    np.testing.assert_array_equal(r["tokens"][0], single["tokens"])
+    np.testing.assert_array_equal(r["ctx_len"], [256 + 3 * 16] * 2)
+    # block 1 saw block 0: its first step's attention over the grown context
+    b1 = r["blocks"][1]["trace"][0]
+    kc = O.from_bf16(inp["k_ctx"]).copy()
+    vc = O.from_bf16(inp["v_ctx"]).copy()
+    L = O.append_block(kc, vc, inp["ctx_len"], r["tokens"][0], inp["emb"], O.from_bf16(inp["u_ctx"]))
+    o = O.round_bf16(O.block_attention(b1["q"], b1["k"], b1["v"], kc, vc, L))
+    np.testing.assert_array_equal(b1["o"], o.reshape(b1["o"].shape))

@@ -44,9 +44,9 @@ __all__ = [
 # bytes of every stored expectation depend on it.
 _STREAMS = (
     "q_blk", "k_blk", "v_blk", "k_ctx", "v_ctx", "shift_scale", "w", "emb",
-    "e_mask", "u_t", "ctx_len", "precommit",
+    "e_mask", "u_t", "ctx_len", "precommit", "u_ctx",
 )
-INPUT_NAMES = _STREAMS[:-2]
+INPUT_NAMES = tuple(n for n in _STREAMS if n not in ("ctx_len", "precommit"))
 
 _CHUNK = 1 << 22  # elements per independently seeded chunk
 
@@ -182,6 +182,9 @@ def generate(d: Dims, seed: int = 0, *, sharp: bool = False, names=None,
         "emb": ((d.V, d.H), s_h),
         "e_mask": ((d.H,), s_h),
         "u_t": ((d.n_qkv, d.H), s_h),
+        # stand-in for the frozen context tower when a committed block joins
+        # the context: [k | v] = Emb[token] . U_ctx^T
+        "u_ctx": ((2 * d.Hkv * d.dh, d.H), s_h),
     }
     out = {}
     for name, (shape, scale) in shapes.items():
