@@ -15,7 +15,8 @@ import os
 __all__ = [
     "TTError", "Dims", "lib", "lib_path", "dims", "workspace", "tt_workspace_bytes",
     "tt_block_denoise_attn", "tt_adaln_modulate", "tt_vocab_confidence_commit",
-    "tt_denoise_block_loop", "tt_denoise_block_loop_layers", "tt_vocab_confidence_commit_noalloc",
+    "tt_denoise_block_loop", "tt_denoise_block_loop_layers", "tt_decode_blocks",
+    "tt_vocab_confidence_commit_noalloc",
     "tt_device_status", "tt_launch_count", "tt_set_attn_splits",
     "tt_status_string", "tt_last_error", "EXPORTS", "tt_profile_enable", "tt_profile_read",
     "tt_selftest_timeout",
@@ -36,9 +37,10 @@ EXPORTS = (
     "tt_launch_count", "tt_set_attn_splits", "tt_block_denoise_attn", "tt_adaln_modulate",
     "tt_vocab_confidence_commit", "tt_denoise_block_loop", "tt_profile_enable", "tt_profile_read",
     "tt_vocab_confidence_commit_noalloc", "tt_selftest_timeout", "tt_denoise_block_loop_layers",
+    "tt_decode_blocks",
 )
 KERNEL_KINDS = ("plan", "embed", "gemm_qkv", "attn", "merge", "adaln", "gemm_vocab", "commit",
-                "gather", "init", "splitk_reduce")
+                "gather", "init", "splitk_reduce", "append")
 
 
 class TTError(RuntimeError):
@@ -97,6 +99,10 @@ def lib() -> ctypes.CDLL:
         L.tt_denoise_block_loop.argtypes = (
             [ctypes.POINTER(Dims)] + [_P] * 8 + [ctypes.c_float, ctypes.c_float, ctypes.c_int32]
             + [_P] * 5 + [_P, ctypes.c_size_t, _P])
+        L.tt_decode_blocks.restype = ctypes.c_int
+        L.tt_decode_blocks.argtypes = (
+            [ctypes.POINTER(Dims), ctypes.c_int32] + [_P] * 9
+            + [ctypes.c_float, ctypes.c_float] + [_P] * 4 + [_P, ctypes.c_size_t, _P])
         L.tt_denoise_block_loop_layers.restype = ctypes.c_int
         L.tt_denoise_block_loop_layers.argtypes = (
             [ctypes.POINTER(Dims), ctypes.c_int32] + [_P] * 8
@@ -242,6 +248,22 @@ def tt_denoise_block_loop(d: Dims, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shif
         _ptr(tokens), _ptr(masked), _ptr(steps_taken), _ptr(commit_step),
         ctypes.addressof(steps_run), _ptr(ws), ws.numel(), _stream(stream)),
         "tt_denoise_block_loop")
+    return int(steps_run.value)
+
+
+def tt_decode_blocks(d: Dims, n_blocks: int, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t,
+                     shift_scale, w, u_ctx, gamma: float, logit_scale: float, tokens,
+                     steps_taken, commit_step, ws, stream=None) -> int:
+    """n_blocks blocks one after the other, each joining the context once
+    committed (k_ctx, v_ctx and ctx_len are updated in place); returns the
+    total number of steps that did work."""
+    steps_run = ctypes.c_int32(0)
+    _check(lib().tt_decode_blocks(
+        ctypes.byref(d), int(n_blocks), _ptr(k_ctx), _ptr(v_ctx), _ptr(ctx_len), _ptr(emb),
+        _ptr(e_mask), _ptr(u_t), _ptr(shift_scale), _ptr(w), _ptr(u_ctx), float(gamma),
+        float(logit_scale), _ptr(tokens), _ptr(steps_taken), _ptr(commit_step),
+        ctypes.addressof(steps_run), _ptr(ws), ws.numel(), _stream(stream)),
+        "tt_decode_blocks")
     return int(steps_run.value)
 
 

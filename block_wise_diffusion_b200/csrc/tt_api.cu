@@ -224,14 +224,21 @@ static AttnGeom attn_geom(const tt_dims& d) {
 
 // K splits of the linear-update GEMM: enough (tile, K range) units to fill
 // the SMs when the block has few rows; a power of two dividing H/64.
-static int qkv_ksplit(const tt_dims& d) {
+static int ksplit_for(const tt_dims& d, int n_out) {
   const int rows = d.B * d.S;
-  const int n_qkv = d.H + 2 * d.Hkv * d.dh;
-  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kQkvBN - 1) / kQkvBN);
+  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_out + kQkvBN - 1) / kQkvBN);
   const int kb = d.H / kGemmBK;
   int k = 1;
   while (2 * k <= kb && kb % (2 * k) == 0 && tiles * 2 * k <= kNumSMs) k *= 2;
   return k;
+}
+static int qkv_ksplit(const tt_dims& d) { return ksplit_for(d, d.H + 2 * d.Hkv * d.dh); }
+// the projection of a committed block into the context: [k | v] per position
+static int ctx_ksplit(const tt_dims& d) { return ksplit_for(d, 2 * d.Hkv * d.dh); }
+static size_t splitk_bytes(const tt_dims& d, int n_out, int ks) {
+  const size_t rows = (size_t)d.B * d.S;
+  const size_t tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_out + kQkvBN - 1) / kQkvBN);
+  return ks > 1 ? (size_t)ks * tiles * kGemmBM * kQkvBN * sizeof(float) : 0;
 }
 
 struct Carver {
@@ -259,6 +266,7 @@ struct Ws {
   float4* stats = nullptr;
   float* qkv_partial = nullptr;
   uint16_t* xrows = nullptr;  // loop: one layer's modulated rows for the next layer
+  uint8_t* blk_masked = nullptr;  // block after block: the current block's mask
   int* seqcnt = nullptr;     // follows ctrl directly: cleared together
   float2* rowres = nullptr;
   size_t ctrl_clear = kCtrlBytes;  // bytes from ctrl to clear at the start of a call
@@ -295,11 +303,12 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     w.xrows = c.take<uint16_t>(rows * d.H * 2);
     w.qkv = c.take<uint16_t>(rows * n_qkv * 2);
     w.attn_out = c.take<uint16_t>(rows * d.H * 2);
-    const int ks = qkv_ksplit(d);
-    // tile-major partials: ks planes of whole 128 x kQkvBN tiles
-    const size_t tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kQkvBN - 1) / kQkvBN);
-    if (ks > 1)
-      w.qkv_partial = c.take<float>((size_t)ks * tiles * kGemmBM * kQkvBN * sizeof(float));
+    // tile-major partials: ks planes of whole 128 x kQkvBN tiles, for the
+    // linear update or the context projection, whichever needs more
+    const size_t pb = std::max(splitk_bytes(d, (int)n_qkv, qkv_ksplit(d)),
+                               splitk_bytes(d, 2 * d.Hkv * d.dh, ctx_ksplit(d)));
+    if (pb) w.qkv_partial = c.take<float>(pb);
+    w.blk_masked = c.take<uint8_t>(rows);
   }
   w.total = (c.off + 255) & ~size_t(255);
   return w;
@@ -741,6 +750,73 @@ tt_status tt_denoise_block_loop_layers(const tt_dims* d, int32_t n_layers, const
   return denoise_block_loop_impl(d, n_layers, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t,
                                  shift_scale, W, gamma, logit_scale, max_steps, tokens, masked,
                                  steps_taken, commit_step, steps_run, ws, ws_bytes, stream);
+}
+
+tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx, tt_bf16* v_ctx,
+                           int32_t* ctx_len, const tt_bf16* emb, const tt_bf16* e_mask,
+                           const tt_bf16* u_t, const tt_bf16* shift_scale, const tt_bf16* W,
+                           const tt_bf16* u_ctx, float gamma, float logit_scale,
+                           int32_t* tokens, int32_t* steps_taken, int32_t* commit_step,
+                           int32_t* steps_run, void* ws, size_t ws_bytes, void* stream) {
+  TT_CHECK(check_dims(d));
+  TT_CHECK(check_ptr(u_ctx, "u_ctx", true));
+  TT_CHECK(check_ptr(tokens, "tokens", false));
+  TT_CHECK(check_ptr(steps_taken, "steps_taken", false));
+  TT_CHECK(check_ptr(commit_step, "commit_step", false));
+  if (n_blocks < 1 || n_blocks > 4096)
+    return fail(TT_ERR_INVALID_ARG, "n_blocks=%d not in [1, 4096]", n_blocks);
+  Ws w;
+  TT_CHECK(check_ws(*d, TT_WS_LOOP, ws, ws_bytes, &w));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int rows = d->B * d->S;
+  const int n_kv = 2 * d->Hkv * d->dh;
+  CUtensorMap tmE, tmC;
+  if (!make_tmap_2d(&tmE, w.egath, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM) ||
+      !make_tmap_2d(&tmC, u_ctx, d->H, n_kv, (uint64_t)d->H * 2, kGemmBK, kQkvBN))
+    return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the context projection");
+  GemmArgs ga{};
+  ga.M_alloc = rows;
+  ga.N = n_kv;
+  ga.K = d->H;
+  ga.C = w.qkv;  // free between blocks
+  ga.ldc = n_kv;
+  ga.err = w.ctrl;
+  ga.ksplit = ctx_ksplit(*d);
+  ga.partial = w.qkv_partial;
+  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_kv + kQkvBN - 1) / kQkvBN) * ga.ksplit;
+  int total_steps = 0;
+  for (int j = 0; j < n_blocks; ++j) {
+    int32_t* tok = tokens + (size_t)j * rows;
+    // a new block: every position masked, no token yet
+    TT_CUDA(cudaMemsetAsync(tok, 0xff, (size_t)rows * sizeof(int32_t), st));
+    TT_CUDA(cudaMemsetAsync(w.blk_masked, 1, (size_t)rows, st));
+    int32_t n = 0;
+    TT_CHECK(denoise_block_loop_impl(d, 1, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale,
+                                     W, gamma, logit_scale, d->S, tok, w.blk_masked,
+                                     steps_taken + (size_t)j * d->B,
+                                     commit_step + (size_t)j * rows, &n, ws, ws_bytes, stream));
+    total_steps += n;
+    // The committed block joins the context: its rows of the workspace's
+    // embeddings are Emb[token] (the commit re-embeds what it commits), so
+    // [k | v] = Emb[token] . U_ctx^T, appended at each sequence's end.
+    TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(tmE, tmC, ga, std::min(tiles, kNumSMs), st));
+    if (ga.ksplit > 1)
+      TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_kv,
+                                                        w.qkv, n_kv, nullptr, st));
+    TT_LAUNCH(TT_K_APPEND, st, launch_append_kv(w.qkv, n_kv, k_ctx, v_ctx, ctx_len, d->B, d->S,
+                                                d->Hkv, d->dh, d->L_cap, w.ctrl, st));
+    // the next block's loop clears the control block: check this append now
+    int h[8];
+    TT_CHECK(read_ctrl(w, st, h));
+    if (h[CTRL_ERR] != 0) {
+      if (steps_run != nullptr) *steps_run = total_steps;
+      return fail((tt_status)h[CTRL_ERR], "block %d: device reported %s at tag 0x%x", j,
+                  tt_status_string((tt_status)h[CTRL_ERR]), h[CTRL_ERR_WHERE]);
+    }
+  }
+  if (g_prof_on.load()) prof_harvest();
+  if (steps_run != nullptr) *steps_run = total_steps;
+  return TT_OK;
 }
 
 }  // extern "C"

@@ -178,6 +178,9 @@ cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st);
 
 cudaError_t launch_selftest_wait(int* ctrl, unsigned long long limit_ns, cudaStream_t st);
 
+cudaError_t launch_append_kv(const uint16_t* kv, int ld, uint16_t* k_ctx, uint16_t* v_ctx,
+                             int* ctx_len, int B, int S, int Hkv, int dh, int L_cap, int* err,
+                             cudaStream_t st);
 cudaError_t launch_loop_init(int B, int S, int* steps_taken, int* commit_step, int* ctrl,
                              cudaStream_t st);
 

@@ -642,7 +642,44 @@ __global__ void loop_init_kernel(int B, int S, int* steps_taken, int* commit_ste
   if (i < B * S) commit_step[i] = -1;
 }
 
+// A committed block joins the context: CTA b copies the block's projected
+// rows kv [B*S, ld] (k of head g at columns g*dh.., v at Hkv*dh + g*dh..) to
+// context positions ctx_len[b] .. ctx_len[b] + S - 1 of every KV head, then
+// advances ctx_len[b].  A sequence without room records TT_ERR_INVALID_ARG
+// and is left unchanged.
+__global__ void __launch_bounds__(256)
+    append_kv_kernel(const uint16_t* __restrict__ kv, int ld, uint16_t* __restrict__ k_ctx,
+                     uint16_t* __restrict__ v_ctx, int* __restrict__ ctx_len, int S, int Hkv,
+                     int dh, int L_cap, int* err) {
+  griddep_launch();
+  griddep_wait();
+  const int b = blockIdx.x;
+  const int L = ctx_len[b];
+  if (L < 0 || L + S > L_cap) {
+    if (threadIdx.x == 0) atomicCAS(err, 0, (int)TT_ERR_INVALID_ARG);
+    return;
+  }
+  const int nv = dh / 8;  // 16-byte vectors per head row
+  const int total = S * Hkv * nv;
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    const int c = i % nv, g = (i / nv) % Hkv, s = i / (nv * Hkv);
+    const uint4* src = reinterpret_cast<const uint4*>(kv + (size_t)(b * S + s) * ld + g * dh);
+    const size_t dst = ((size_t)(b * Hkv + g) * L_cap + L + s) * dh;
+    reinterpret_cast<uint4*>(k_ctx + dst)[c] = src[c];
+    reinterpret_cast<uint4*>(v_ctx + dst)[c] = src[(Hkv * dh) / 8 + c];
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) ctx_len[b] = L + S;
+}
+
 }  // namespace
+
+cudaError_t launch_append_kv(const uint16_t* kv, int ld, uint16_t* k_ctx, uint16_t* v_ctx,
+                             int* ctx_len, int B, int S, int Hkv, int dh, int L_cap, int* err,
+                             cudaStream_t st) {
+  return launch_k(append_kv_kernel, dim3(B), dim3(256), 0, st, kv, ld, k_ctx, v_ctx, ctx_len, S,
+                  Hkv, dh, L_cap, err);
+}
 
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st) {
   return launch_k(plan_kernel, dim3(1), dim3(1024), 0, st, a);

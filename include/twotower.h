@@ -105,7 +105,7 @@ TT_API tt_status tt_set_attn_splits(int32_t n_splits);
 enum {
   TT_K_PLAN = 0, TT_K_EMBED = 1, TT_K_GEMM_QKV = 2, TT_K_ATTN = 3, TT_K_MERGE = 4,
   TT_K_ADALN = 5, TT_K_GEMM_VOCAB = 6, TT_K_COMMIT = 7, TT_K_GATHER = 8, TT_K_INIT = 9,
-  TT_K_REDUCE = 10, TT_K_COUNT = 11
+  TT_K_REDUCE = 10, TT_K_APPEND = 11, TT_K_COUNT = 12
 };
 
 /* Per-kernel profiler: while enabled, every kernel this library launches is
@@ -229,6 +229,40 @@ TT_API tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, c
                                 float logit_scale, int32_t max_steps, int32_t* tokens,
                                 uint8_t* masked, int32_t* steps_taken, int32_t* commit_step,
                                 int32_t* steps_run, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Blocks one after the other ("Generation Process" of the gist.science
+ * summary: a block of S masked tokens is refined until committed, then the
+ * context tower updates and the next block starts).  For j = 0 .. n_blocks-1:
+ * tokens_j = -1 and every position masked; the block loop of
+ * tt_denoise_block_loop (up to S steps) commits it; then the block joins the
+ * context: for each position, [k | v] = Emb[token] . U_ctx^T (bf16) is written
+ * at context position ctx_len[b] + s of every KV head and ctx_len[b] += S.
+ * The frozen context tower itself is not modelled: U_ctx is a seeded
+ * projection standing in for it (this library's reading).
+ *
+ *   k_ctx, v_ctx   bf16 [B, Hkv, L_cap, dh]   IN/OUT: the rows
+ *                  ctx_len[b] .. ctx_len[b] + n_blocks*S - 1 are written
+ *   ctx_len        int32 [B] device            IN/OUT: grows by S per block
+ *   u_ctx          bf16 [2*Hkv*dh, H]          rows 0..Hkv*dh-1 give k (head g
+ *                  at rows g*dh..), the rest give v
+ *   tokens         int32 [n_blocks, B, S]      OUT
+ *   steps_taken    int32 [n_blocks, B]         OUT (as tt_denoise_block_loop)
+ *   commit_step    int32 [n_blocks, B, S]      OUT
+ *   steps_run      host int32, may be NULL     total steps that did work
+ *   other arguments, workspace (TT_WS_LOOP) and errors as
+ *   tt_denoise_block_loop; one host synchronisation per block.
+ * n_blocks outside 1..4096 is TT_ERR_INVALID_ARG.  A sequence whose cache has
+ * no room for a block (ctx_len[b] + S > L_cap) is left unchanged and the call
+ * returns TT_ERR_INVALID_ARG (recorded on the device).
+ */
+TT_API tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx,
+                                  tt_bf16* v_ctx, int32_t* ctx_len, const tt_bf16* emb,
+                                  const tt_bf16* e_mask, const tt_bf16* u_t,
+                                  const tt_bf16* shift_scale, const tt_bf16* w,
+                                  const tt_bf16* u_ctx, float gamma, float logit_scale,
+                                  int32_t* tokens, int32_t* steps_taken, int32_t* commit_step,
+                                  int32_t* steps_run, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * The block loop over n_layers denoiser layers ("Architecture" of the

@@ -229,3 +229,47 @@ def test_loop_layers_mid_shape_sampled_sequences():
     n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, 8.0, bsel=np.array([1, 6]))
     print(f"mid 2-layer loop: compared {n_cmp} sequence-steps, excluded {n_ex}")
     assert n_cmp > 0 and n_ex <= 2
+
+
+@pytest.mark.parametrize("logit_scale", [1.0, 12.0])
+def test_decode_blocks_block_after_block(logit_scale):
+    """Three blocks one after the other: each committed block joins the
+    context.  The oracle follows the GPU's committed tokens block by block;
+    appended K/V rows agree within one bf16 unit, each block's steps are
+    compared teacher-forced as in the single-block loop."""
+    nb = 3
+    d = tt_inputs.Dims(B=2, S=16, Hq=4, Hkv=1, dh=64, V=1024, L_cap=256 + nb * 16,
+                       ctx=("fixed", 256))
+    inp = tt_inputs.generate(d, seed=51)
+    D = tt.dims(d)
+    kc, vc = G.dev_bf16(inp["k_ctx"]), G.dev_bf16(inp["v_ctx"])
+    cl = G.dev(inp["ctx_len"])
+    dv = {k: G.dev_bf16(inp[k]) for k in ("emb", "e_mask", "u_t", "shift_scale", "w", "u_ctx")}
+    tokens = torch.empty((nb, d.B, d.S), dtype=torch.int32, device="cuda")
+    steps = torch.empty((nb, d.B), dtype=torch.int32, device="cuda")
+    cstep = torch.empty((nb, d.B, d.S), dtype=torch.int32, device="cuda")
+    ws = G.workspace(D, tt.TT_WS_LOOP)
+    n = tt.tt_decode_blocks(D, nb, kc, vc, cl, dv["emb"], dv["e_mask"], dv["u_t"],
+                            dv["shift_scale"], dv["w"], dv["u_ctx"], 0.8, logit_scale, tokens,
+                            steps, cstep, ws)
+    np.testing.assert_array_equal(cl.cpu().numpy(), [256 + nb * 16] * d.B)
+    gt, gs, gc = tokens.cpu().numpy(), steps.cpu().numpy(), cstep.cpu().numpy()
+    assert n == int(gs.max(axis=1).sum())
+    f = O.from_bf16
+    k64, v64, u = f(inp["k_ctx"]), f(inp["v_ctx"]), f(inp["u_ctx"])
+    L = np.array(inp["ctx_len"], dtype=np.int64)
+    n_cmp = n_ex = 0
+    for j in range(nb):
+        blk = dict(inp, k_ctx=O._to_bits(k64), v_ctx=O._to_bits(v64), ctx_len=L.astype(np.int32),
+                   tokens=np.full((d.B, d.S), -1, np.int32), masked=np.ones((d.B, d.S), np.uint8))
+        g = dict(tokens=gt[j], masked=np.zeros((d.B, d.S), np.uint8), steps_taken=gs[j],
+                 commit_step=gc[j], steps_run=int(gs[j].max()))
+        check_invariants(d, blk, g)
+        c, e = compare_teacher_forced(blk, g, 0.8, logit_scale)
+        n_cmp, n_ex = n_cmp + c, n_ex + e
+        L = O.append_block(k64, v64, L, gt[j].astype(np.int64), inp["emb"], u)
+    assert n_cmp > 0 and n_ex <= 3, (n_cmp, n_ex)
+    for got, ref in ((G.host_f64(kc), k64), (G.host_f64(vc), v64)):
+        new = got[:, :, 256:], ref[:, :, 256:]
+        np.testing.assert_allclose(new[0], new[1], rtol=2 ** -8, atol=1e-6)
+        np.testing.assert_array_equal(got[:, :, :256], ref[:, :, :256])
