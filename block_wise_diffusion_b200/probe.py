@@ -13,6 +13,7 @@ generator the tests and the benchmark use); nothing here computes a reference.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import os
 import sys
 
@@ -72,11 +73,43 @@ def setup_vocab(d):
     return call, lambda: tt.tt_device_status(ws)
 
 
+def setup_blocks(d, n_blocks: int, logit_scale: float):
+    """Upload seeded inputs; return (call, check) for tt_decode_blocks over
+    n_blocks blocks (the context is reset before each call)."""
+    import torch
+    import tt_inputs
+    import block_wise_diffusion_b200 as tt
+    inp = tt_inputs.generate(d, seed=0)
+    kc0, vc0 = _dev(inp["k_ctx"]), _dev(inp["v_ctx"])
+    kc, vc = kc0.clone(), vc0.clone()
+    cl0 = torch.from_numpy(inp["ctx_len"]).cuda()
+    cl = cl0.clone()
+    X = {k: _dev(inp[k]) for k in ("emb", "e_mask", "u_t", "shift_scale", "w", "u_ctx")}
+    D = tt.dims(d)
+    tok = torch.empty((n_blocks, d.B, d.S), dtype=torch.int32, device="cuda")
+    steps = torch.empty((n_blocks, d.B), dtype=torch.int32, device="cuda")
+    cs = torch.empty((n_blocks, d.B, d.S), dtype=torch.int32, device="cuda")
+    ws = tt.workspace(D, tt.TT_WS_LOOP)
+
+    def call():
+        kc.copy_(kc0)
+        vc.copy_(vc0)
+        cl.copy_(cl0)
+        tt.tt_decode_blocks(D, n_blocks, kc, vc, cl, X["emb"], X["e_mask"], X["u_t"],
+                            X["shift_scale"], X["w"], X["u_ctx"], 0.8, logit_scale, tok, steps,
+                            cs, ws)
+
+    return call, lambda: tt.tt_device_status(ws)
+
+
 def main(argv=None) -> int:
     import torch
     import tt_inputs
     p = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    p.add_argument("stage", choices=["attn", "vocab"])
+    p.add_argument("stage", choices=["attn", "vocab", "blocks"])
+    p.add_argument("--n-blocks", type=int, default=4,
+                   help="blocks stage: blocks per call (the cache grows to hold them)")
+    p.add_argument("--logit-scale", type=float, default=1.0)
     p.add_argument("--workload", default="mid", choices=sorted(tt_inputs.WORKLOADS))
     p.add_argument("--B", type=int, default=None, help="override the batch")
     p.add_argument("--V", type=int, default=None, help="override the vocabulary (vocab stage)")
@@ -90,7 +123,12 @@ def main(argv=None) -> int:
     if a.V is not None:
         over["V"] = a.V
     d = tt_inputs.workload(a.workload, **over)
-    call, check = (setup_attn if a.stage == "attn" else setup_vocab)(d)
+    if a.stage == "blocks":
+        # room for the blocks behind the context
+        d = dataclasses.replace(d, L_cap=d.L_cap + a.n_blocks * d.S)
+        call, check = setup_blocks(d, a.n_blocks, a.logit_scale)
+    else:
+        call, check = (setup_attn if a.stage == "attn" else setup_vocab)(d)
     call()  # warm-up
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     ev[0].record()
@@ -102,7 +140,10 @@ def main(argv=None) -> int:
         raise RuntimeError("device reported an error")
     msg = f"ok {a.stage} {d}"
     if a.time:
-        msg += f": {ev[0].elapsed_time(ev[1]) * 1e3 / a.calls:.1f} us per call (no L2 flush)"
+        us = ev[0].elapsed_time(ev[1]) * 1e3 / a.calls
+        msg += f": {us:.1f} us per call (no L2 flush)"
+        if a.stage == "blocks":
+            msg += f", {a.n_blocks * d.B * d.S / (us * 1e-6):.0f} committed tokens/s"
     print(msg)
     return 0
 
