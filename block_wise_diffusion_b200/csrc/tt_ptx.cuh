@@ -59,21 +59,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// As above, but a thread whose phase is not yet complete is suspended for up
-// to `hint_ns` (it resumes as soon as the phase completes), so waiting warps
-// leave their SMSP's issue slots to the warps doing work.
-__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-constexpr uint32_t kWaitHintNs = 0;
 
 // Bounded wait for the phase with the given parity.  `abort_flag` is a CTA
 // shared word: once any thread has timed out, later waits return at once.
@@ -84,8 +69,7 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
   for (uint32_t i = 0;; ++i) {
     // A completed phase wins over the abort flag, so threads waiting on the
     // same phase all see the same outcome.
-    if (kWaitHintNs ? mbar_try_wait_for(bar, parity, kWaitHintNs) : mbar_try_wait(bar, parity))
-      return true;
+    if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
     if ((i & 255u) == 255u && global_ns() - t0 > limit_ns) {
       if (err) {
