@@ -34,6 +34,13 @@ def test_round_bf16_ties_and_specials():
     assert O.round_bf16(np.array([0.0]))[0] == 0.0
     assert O.round_bf16(np.array([1e39]))[0] == np.inf
     assert O.round_bf16(np.array([2.0 ** -130]))[0] == 2.0 ** -130          # subnormal, exact
+    # bf16 subnormals are spaced 2^-133 (7 stored bits below 2^-126): ties go to even
+    sub = 2.0 ** -133
+    assert O.round_bf16(np.array([1.5 * sub]))[0] == 2 * sub
+    assert O.round_bf16(np.array([2.5 * sub]))[0] == 2 * sub
+    assert O.round_bf16(np.array([0.75 * sub]))[0] == sub
+    assert O.round_bf16(np.array([0.5 * sub]))[0] == 0.0                   # tie -> even (0)
+    assert O.round_bf16(np.array([2.0 ** -126 + 0.5 * sub]))[0] == 2.0 ** -126
 
 
 def test_round_bf16_matches_torch_and_input_module():
@@ -43,6 +50,11 @@ def test_round_bf16_matches_torch_and_input_module():
     ref_inputs = O.from_bf16(tt_inputs.bf16_bits(x32))
     np.testing.assert_array_equal(mine, ref_torch)
     np.testing.assert_array_equal(mine, ref_inputs)
+    # float32 values around and below the smallest normal bf16 (2^-126)
+    tiny = (np.sign(rnd(20000, 3)) * 2.0 ** (-150 + 30 * np.random.default_rng(4).random(20000))
+            ).astype(np.float32)
+    ref_tiny = torch.from_numpy(tiny).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_bf16(tiny.astype(np.float64)), ref_tiny)
 
 
 def test_from_bf16_exact():
@@ -204,6 +216,9 @@ def test_logits_orientation_and_scale():
     np.testing.assert_allclose(conf, p.max(axis=-1), rtol=1e-12)
     ps = np.sort(p, axis=-1)
     np.testing.assert_allclose(gp, ps[:, -1] - ps[:, -2], rtol=1e-9, atol=1e-15)
+    ls = np.sort(3.0 * yr @ O.from_bf16(wb).T, axis=-1)
+    np.testing.assert_allclose(gl, ls[:, -1] - ls[:, -2], rtol=1e-12, atol=1e-15)
+    assert (gl >= 0).all()
 
 
 # --------------------------------------------------------------------- commit
@@ -263,6 +278,8 @@ def test_commit_invariants_random():
             conf[:, :4] = conf[:, :1]                     # planted ties
         tok = rng.integers(0, 100, (B, S))
         gamma = rng.choice([0.5, 0.8, 0.95])
+        if trial % 4 == 1:
+            conf[:, 4:6] = gamma                          # exactly at the threshold: commits
         t2, m2, c, fb = O.commit(conf, tok, tokens, masked, gamma)
         assert not np.any(c & ~masked)                      # only masked positions commit
         np.testing.assert_array_equal(t2[~masked], tokens[~masked])   # committed never change
@@ -414,6 +431,81 @@ def test_layers_depend_only_on_their_own_context():
     inp2["v_ctx_l"][1] = tt_inputs.bf16_bits(-O.from_bf16(inp["v_ctx_l"][1]).astype(np.float32))
     r2 = O.denoise_block_loop(inp2, 0.8, max_steps=1)
     assert not np.allclose(r["trace"][0]["conf"], r2["trace"][0]["conf"])
+
+
+def test_step_sequences_are_independent():
+    """One step over a batch whose sequences differ in mask (hence t), context
+    length and tokens gives, per sequence, what that sequence gives alone."""
+    d = tt_inputs.workload("tiny", B=3)
+    inp = tt_inputs.generate(d, seed=6)
+    f = O.from_bf16
+    masked = np.ones((d.B, d.S), dtype=bool)
+    masked[1, :5] = False
+    masked[2, 3:15] = False
+    tokens = np.where(masked, -1, 9)
+    cl = np.array([256, 100, 17])
+    e = O.embed_block(tokens, masked, inp["emb"], inp["e_mask"])
+    q, k, v = O.linear_update(e, f(inp["u_t"]), d.Hq, d.Hkv, d.dh)
+    kc, vc, E, w = f(inp["k_ctx"]), f(inp["v_ctx"]), f(inp["shift_scale"]), f(inp["w"])
+    args = (E, w)
+    both = O.denoise_step(q, k, v, kc, vc, cl, *args, tokens, masked, 0.8, 12.0)
+    for b in range(d.B):
+        sl = slice(b, b + 1)
+        one = O.denoise_step(q[sl], k[sl], v[sl], kc[sl], vc[sl], cl[sl], *args, tokens[sl],
+                             masked[sl], 0.8, 12.0)
+        for key in ("o", "y", "conf", "tok", "tokens", "masked", "committed"):
+            np.testing.assert_array_equal(both[key][sl], one[key], err_msg=f"{key} of {b}")
+
+
+def test_layers_sequences_are_independent():
+    """A batch of sequences with different times t gives, row for row, what
+    each sequence gives alone: a row is modulated by its own sequence's t."""
+    d = tt_inputs.workload("tiny", B=3)
+    inp = tt_inputs.generate(d, seed=5, n_layers=2)
+    f = O.from_bf16
+    layers = [tuple(f(inp[n + "_l"][i]) for n in ("u_t", "k_ctx", "v_ctx", "shift_scale"))
+              for i in range(1)]
+    masked = np.ones((d.B, d.S), dtype=bool)
+    masked[1, :5] = False
+    masked[2, :12] = False
+    tokens = np.where(masked, -1, 3)
+    e = O.embed_block(tokens, masked, inp["emb"], inp["e_mask"])
+    t = masked.sum(axis=1) / d.S
+    assert len(set(t)) == 3
+    cl = np.array([256, 100, 17])
+    both = O.denoiser_layers(e, layers, cl, t, d.Hq, d.Hkv, d.dh)
+    for b in range(d.B):
+        one = [(u, kc[b:b + 1], vc[b:b + 1], E) for u, kc, vc, E in layers]
+        np.testing.assert_array_equal(
+            both[b:b + 1], O.denoiser_layers(e[b:b + 1], one, cl[b:b + 1], t[b:b + 1],
+                                             d.Hq, d.Hkv, d.dh))
+
+
+def test_loop_wires_each_layer_to_its_own_tables():
+    """Step 0 of a two-layer loop is layer 0 (its own U, context and adaLN
+    table) followed by the single-layer step on layer 1's tables; layer 0's
+    context moves the result."""
+    d = tt_inputs.workload("tiny", B=2)
+    inp = tt_inputs.generate(d, seed=11, n_layers=2)
+    f = O.from_bf16
+    per = [{n: f(inp[n + "_l"][i]) for n in ("u_t", "k_ctx", "v_ctx", "shift_scale")}
+           for i in range(2)]
+    r = O.denoise_block_loop(inp, 0.8, 8.0, max_steps=1)
+    e = O.embed_block(inp["tokens"], inp["masked"], inp["emb"], inp["e_mask"])
+    t = inp["masked"].sum(axis=1) / d.S
+    l0 = per[0]
+    x = O.denoiser_layers(e, [(l0["u_t"], l0["k_ctx"], l0["v_ctx"], l0["shift_scale"])],
+                          inp["ctx_len"], t, d.Hq, d.Hkv, d.dh)
+    l1 = per[1]
+    q, k, v = O.linear_update(x, l1["u_t"], d.Hq, d.Hkv, d.dh)
+    st = O.denoise_step(q, k, v, l1["k_ctx"], l1["v_ctx"], inp["ctx_len"], l1["shift_scale"],
+                        f(inp["w"]), inp["tokens"], inp["masked"], 0.8, 8.0)
+    np.testing.assert_array_equal(r["trace"][0]["conf"], st["conf"])
+    np.testing.assert_array_equal(r["tokens"], st["tokens"])
+    inp2 = dict(inp, v_ctx_l=inp["v_ctx_l"].copy())
+    inp2["v_ctx_l"][0] = tt_inputs.bf16_bits(-f(inp["v_ctx_l"][0]).astype(np.float32))
+    r2 = O.denoise_block_loop(inp2, 0.8, 8.0, max_steps=1)
+    assert not np.allclose(r["trace"][0]["conf"], r2["trace"][0]["conf"], equal_nan=True)
 
 
 def test_layer_by_explicit_loops():
