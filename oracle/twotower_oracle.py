@@ -88,12 +88,6 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     return out
 
 
-def to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """float64 values that are exactly bf16 -> their bit patterns."""
-    f = np.asarray(x, dtype=np.float64).astype(np.float32)
-    return (f.view(np.uint32) >> np.uint32(16)).astype(np.uint16)
-
-
 # ---- a1: block-denoise attention -------------------------------------------
 def block_attention(q_blk, k_blk, v_blk, k_ctx, v_ctx, ctx_len):
     """Denoiser attention of one layer (Architecture; Generation Process).

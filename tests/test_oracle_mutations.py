@@ -32,6 +32,7 @@ MUTATIONS = [
      "keys = np.concatenate([k_ctx[b, g, :L], 0 * k_blk[b, :, g]], axis=0)", 1),
     ("attn-values-are-keys", "vals = np.concatenate([v_ctx[b, g, :L], v_blk[b, :, g]], axis=0)",
      "vals = np.concatenate([k_ctx[b, g, :L], k_blk[b, :, g]], axis=0)", 1),
+    ("loops-no-scale", "scores.append(acc / math.sqrt(dh))", "scores.append(acc)", 1),
     ("attn-gqa-interleaved", "q_blk[b, :, g * G:(g + 1) * G, :]", "q_blk[b, :, g::Hkv, :]", 1),
     ("attn-softmax-wrong-axis", "p /= p.sum(axis=-1, keepdims=True)",
      "p /= p.sum(axis=0, keepdims=True)", 1),
@@ -89,6 +90,7 @@ MUTATIONS = [
      "k_ctx[b, :, L + s] = kv[b, s, Hkv * dh:]", 1),
     ("decode-context-not-grown", "blk = dict(inp, k_ctx=_to_bits(k_ctx), v_ctx=_to_bits(v_ctx),",
      "blk = dict(inp, k_ctx=inp[\"k_ctx\"], v_ctx=inp[\"v_ctx\"],", 1),
+    ("to-bits-shift", "return (u >> 16).astype(np.uint16)", "return (u >> 17).astype(np.uint16)", 1),
 ]
 
 
