@@ -107,6 +107,44 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return x > -126.0f ? r : 0.f;
 }
 
+// TMEM load of 16 columns (32x32b shape: a thread's lane, consecutive columns).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// TMEM store of 8 columns, same shape.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+               "r"(r[7])
+               : "memory");
+}
+// P for 16 score columns as 8 bf16 pairs; the last pair on the FMA pipe.
+__device__ __forceinline__ void exp_slice16(const uint32_t (&sv)[16], float c, float m, float& s0,
+                                            float& s1, uint32_t (&pk)[8]) {
+#pragma unroll
+  for (int j = 0; j < 16; j += 2) {
+    const float x0 = fmaf(__uint_as_float(sv[j]), c, -m);
+    const float x1 = fmaf(__uint_as_float(sv[j + 1]), c, -m);
+    float p0, p1;
+    if (j == 14) {
+      p0 = exp2_poly(x0);
+      p1 = exp2_poly(x1);
+    } else {
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    s0 += p0;
+    s1 += p1;
+    pk[j >> 1] = pack_bf16x2(p0, p1);
+  }
+}
+
 __global__ void __launch_bounds__(kAttnThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                 const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKb,
@@ -436,8 +474,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mc[(j >> 1) & 3] = fmax3(mc[(j >> 1) & 3], __uint_as_float(sa[j]), __uint_as_float(sa[j + 1]));
         }
         const float part = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
-        // The first exponential slice is read while the maxima are swapped.
-        tmem_ld32(tS, sa);
+        // The first exponential sub-slice is read while the maxima are swapped.
+        uint32_t s_even[16], s_odd[16];  // sub-slices 0, 2 and 1, 3
+        tmem_ld16(tS, s_even);
         // One buffer suffices: a warp writes tile t+1's value only after
         // S(t+1), which needs its partner's P(t), written after the read.
         xch[ch * 32 + lane] = bf16_bits(part);
@@ -463,30 +502,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // already); one pair in eight on the FMA pipe.
         float s0 = 0.f, s1 = 0.f;
         tmem_wait_ld();
+        // Four 16-column sub-slices; the next one's load is in flight while
+        // this one's exponentials run.  P of sub-slice k goes to columns
+        // [8k, 8k+8), which sub-slices already read cover.
 #pragma unroll 1
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          if (c0 > 0) {
-            tmem_ld32(tS + c0, sa);
-            tmem_wait_ld();
-          }
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float x0 = fmaf(__uint_as_float(sa[j]), c, -m);
-            const float x1 = fmaf(__uint_as_float(sa[j + 1]), c, -m);
-            float p0, p1;
-            if ((j & 15) == 14) {
-              p0 = exp2_poly(x0);
-              p1 = exp2_poly(x1);
-            } else {
-              p0 = ex2(x0);
-              p1 = ex2(x1);
-            }
-            s0 += p0;
-            s1 += p1;
-            pk[j >> 1] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tS + c0 / 2, pk);
+        for (int k = 0; k < 4; k += 2) {
+          uint32_t pk[8];
+          tmem_ld16(tS + 16 * (k + 1), s_odd);
+          exp_slice16(s_even, c, m, s0, s1, pk);
+          tmem_st8(tS + 8 * k, pk);
+          tmem_wait_ld();
+          if (k == 0) tmem_ld16(tS + 32, s_even);
+          exp_slice16(s_odd, c, m, s0, s1, pk);
+          tmem_st8(tS + 8 * (k + 1), pk);
+          if (k == 0) tmem_wait_ld();
         }
         l += s0 + s1;
         // O_h to the new max before P_h(t).V adds to it (s_full also
