@@ -304,6 +304,34 @@ def algorithmic(kind, d, inp, m_per_launch, launches, peaks):
     return "hbm", sum(by) / len(by), "GB/s", t_roof
 
 
+# ex2.approx retires 16 results per clock per SM on B200 in its f32, f16x2 and
+# bf16x2 forms alike (micro-benchmarked: one 1024-thread CTA per SM, eight
+# independent chains per thread).
+MUFU_EX2_PER_CLK_SM = 16
+NOMINAL_MAX_SM_MHZ = 1965.0
+
+
+def attn_exp_per_launch(d, inp):
+    """Exponentials one attention launch must evaluate: one per (query row,
+    key), i.e. sum over b of Hq * S * (L_b + S)."""
+    L = np.asarray(inp["ctx_len"], dtype=np.float64)
+    return float(d.Hq * d.S * (L + d.S).sum())
+
+
+def exp_roof(exps, avg_s, n_sm, clk):
+    """The attention kernel's third roof: exponentials per second against the
+    MUFU rate at the SM clock sampled under load (the nominal maximum clock
+    when no sample was taken)."""
+    mhz = float(clk["sm_mhz"]) if clk and clk.get("sm_mhz") else NOMINAL_MAX_SM_MHZ
+    peak = MUFU_EX2_PER_CLK_SM * n_sm * mhz * 1e6
+    ach = exps / avg_s
+    return {"per_launch": exps, "achieved_T_per_s": round(ach / 1e12, 3),
+            "peak_T_per_s": round(peak / 1e12, 3), "frac": round(ach / peak, 4),
+            "peak_source": f"{MUFU_EX2_PER_CLK_SM} ex2/clk/SM x {n_sm} SMs x {mhz:.0f} MHz "
+                           + ("(median under load)" if clk and clk.get("sm_mhz") else
+                              "(nominal max clock)")}
+
+
 def run_ours(args, rank, world, local):
     import torch
     import block_wise_diffusion_b200 as tt
@@ -433,6 +461,7 @@ def run_ours(args, rank, world, local):
     # rows of the vocabulary GEMM at step k: positions still masked at its start
     m_per_step = [int((m0 & (cs >= k)).sum()) for k in range(int(cs.max()) + 1)]
     peaks, peak_src = load_peaks()
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
     kernels = {}
     for kind, (kms, n) in sorted(table.items(), key=lambda kv: -kv[1][0]):
         e = {"launches": n, "total_ms": round(kms, 4), "avg_us": round(1e3 * kms / n, 2)}
@@ -442,6 +471,8 @@ def run_ours(args, rank, world, local):
             pk = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops_sustained"]
             e.update(bound=bound, achieved=round(ach, 2), unit=unit, frac=round(ach / pk, 4),
                      roofline_time_frac=round(t_roof / (kms / 1e3), 4))
+        if kind == "attn":
+            e["exp"] = exp_roof(attn_exp_per_launch(d, inp), kms / n / 1e3, n_sm, clk)
         kernels[kind] = e
     dom = max(table, key=lambda k: table[k][0])
     bound, per, unit, t_roof = algorithmic(dom, d, inp, m_per_step, table[dom][1], peaks)

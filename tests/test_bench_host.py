@@ -1,4 +1,5 @@
-"""Host-side logic of bench.py: the roofline classification per kernel kind."""
+"""Host-side logic of bench.py: the roofline classification per kernel kind
+and the attention kernel's exponential (MUFU) roof."""
 import numpy as np
 
 import bench
@@ -40,3 +41,23 @@ def test_attention_counts_context_and_block_bytes_and_flops():
     # tensor peak the FLOPs dominate
     assert b == "tensor" and per == flops
     assert bench.algorithmic("commit", d, inp, [], 1, PEAKS)[0] is None
+
+
+def test_attention_exponential_roof():
+    d = tt_inputs.workload("long")
+    inp = {"ctx_len": np.full(d.B, d.L_cap, np.int32)}
+    e = bench.attn_exp_per_launch(d, inp)
+    # one exponential per (query row, key): B * Hq * S * (L + S); 0.134e9 here
+    assert e == d.B * d.Hq * d.S * (d.L_cap + d.S)
+    assert abs(e - 0.134e9) < 0.001e9
+    ragged = {"ctx_len": np.array([0, 100, 5], np.int32)}
+    assert bench.attn_exp_per_launch(d, ragged) == d.Hq * d.S * (0 + 100 + 5 + 3 * d.S)
+    r = bench.exp_roof(e, 100e-6, 148, {"sm_mhz": 1500.0})
+    peak = 16 * 148 * 1500e6
+    assert abs(r["frac"] - round(e / 100e-6 / peak, 4)) < 1e-12
+    assert abs(r["peak_T_per_s"] - round(peak / 1e12, 3)) < 1e-12
+    assert "median under load" in r["peak_source"]
+    for clk in (None, {}, {"sm_mhz": None}):
+        r = bench.exp_roof(e, 100e-6, 148, clk)
+        assert r["peak_T_per_s"] == round(16 * 148 * 1965e6 / 1e12, 3)
+        assert "nominal" in r["peak_source"]
