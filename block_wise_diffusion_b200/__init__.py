@@ -130,6 +130,31 @@ def _ptr(x) -> int | None:
     return x.data_ptr()
 
 
+def _nbytes(x) -> int:
+    return x.numel() * x.element_size() if hasattr(x, "numel") else 0
+
+
+def _sized(x, name: str, nbytes: int) -> int | None:
+    """_ptr(x) after checking that a tensor holds at least ``nbytes``: the
+    shape include/twotower.h documents for the argument times its element
+    size.  The kernels address these buffers from the dims alone, so a short
+    tensor would be read or written past its end.  Raw integer addresses
+    carry no size and pass unchecked."""
+    if x is not None and not isinstance(x, int) and _nbytes(x) < nbytes:
+        raise ValueError(f"{name} holds {_nbytes(x)} bytes; these dims need {nbytes}")
+    return _ptr(x)
+
+
+def _ctx_bytes(d: Dims) -> int:
+    """bf16 [B, Hkv, L_cap, dh]: one context cache (K or V) of one layer."""
+    return d.B * d.Hkv * d.L_cap * d.dh * 2
+
+
+def _u_t_bytes(d: Dims) -> int:
+    """bf16 [H + 2*Hkv*dh, H]: one layer's linear update."""
+    return (d.H + 2 * d.Hkv * d.dh) * d.H * 2
+
+
 def _stream(stream) -> int | None:
     if stream is None:
         import torch
@@ -205,24 +230,41 @@ def tt_device_status(ws, stream=None) -> int:
 
 def tt_block_denoise_attn(d: Dims, q_blk, k_blk, v_blk, k_ctx, v_ctx, ctx_len, out, ws,
                           stream=None) -> None:
+    rows = d.B * d.S
     _check(lib().tt_block_denoise_attn(
-        ctypes.byref(d), _ptr(q_blk), _ptr(k_blk), _ptr(v_blk), _ptr(k_ctx), _ptr(v_ctx),
-        _ptr(ctx_len), _ptr(out), _ptr(ws), ws.numel() if hasattr(ws, "numel") else 0,
+        ctypes.byref(d), _sized(q_blk, "q_blk", rows * d.Hq * d.dh * 2),
+        _sized(k_blk, "k_blk", rows * d.Hkv * d.dh * 2),
+        _sized(v_blk, "v_blk", rows * d.Hkv * d.dh * 2), _sized(k_ctx, "k_ctx", _ctx_bytes(d)),
+        _sized(v_ctx, "v_ctx", _ctx_bytes(d)), _sized(ctx_len, "ctx_len", d.B * 4),
+        _sized(out, "out", rows * d.Hq * d.dh * 2), _ptr(ws), _nbytes(ws),
         _stream(stream)), "tt_block_denoise_attn")
 
 
 def tt_adaln_modulate(d: Dims, x, shift_scale, t, y, ws, stream=None) -> None:
+    rows = d.B * d.S
     _check(lib().tt_adaln_modulate(
-        ctypes.byref(d), _ptr(x), _ptr(shift_scale), _ptr(t), _ptr(y), _ptr(ws), ws.numel(),
-        _stream(stream)), "tt_adaln_modulate")
+        ctypes.byref(d), _sized(x, "x", rows * d.H * 2),
+        _sized(shift_scale, "shift_scale", 2 * d.H * 2), _sized(t, "t", d.B * 4),
+        _sized(y, "y", rows * d.H * 2), _ptr(ws), _nbytes(ws), _stream(stream)),
+        "tt_adaln_modulate")
 
 
 def tt_vocab_confidence_commit(d: Dims, y, w, gamma: float, logit_scale: float, tokens, masked,
                                conf_out, argmax_out, n_committed, ws, stream=None) -> None:
     _check(lib().tt_vocab_confidence_commit(
-        ctypes.byref(d), _ptr(y), _ptr(w), float(gamma), float(logit_scale), _ptr(tokens),
-        _ptr(masked), _ptr(conf_out), _ptr(argmax_out), _ptr(n_committed), _ptr(ws), ws.numel(),
-        _stream(stream)), "tt_vocab_confidence_commit")
+        ctypes.byref(d), *_vocab_args(d, y, w, gamma, logit_scale, tokens, masked, conf_out,
+                                      argmax_out, n_committed),
+        _ptr(ws), _nbytes(ws), _stream(stream)), "tt_vocab_confidence_commit")
+
+
+def _vocab_args(d: Dims, y, w, gamma, logit_scale, tokens, masked, conf_out, argmax_out,
+                n_committed) -> tuple:
+    rows = d.B * d.S
+    return (_sized(y, "y", rows * d.H * 2), _sized(w, "w", d.V * d.H * 2), float(gamma),
+            float(logit_scale), _sized(tokens, "tokens", rows * 4),
+            _sized(masked, "masked", rows), _sized(conf_out, "conf_out", rows * 4),
+            _sized(argmax_out, "argmax_out", rows * 4),
+            _sized(n_committed, "n_committed", d.B * 4))
 
 
 def tt_vocab_confidence_commit_noalloc(d: Dims, y, w, gamma: float, logit_scale: float,
@@ -232,8 +274,8 @@ def tt_vocab_confidence_commit_noalloc(d: Dims, y, w, gamma: float, logit_scale:
     allocate device memory; its scratch is a 16 MiB array built into the
     library (calls that overlap on the GPU must be serialised)."""
     _check(lib().tt_vocab_confidence_commit_noalloc(
-        ctypes.byref(d), _ptr(y), _ptr(w), float(gamma), float(logit_scale), _ptr(tokens),
-        _ptr(masked), _ptr(conf_out), _ptr(argmax_out), _ptr(n_committed), _stream(stream)),
+        ctypes.byref(d), *_vocab_args(d, y, w, gamma, logit_scale, tokens, masked, conf_out,
+                                      argmax_out, n_committed), _stream(stream)),
         "tt_vocab_confidence_commit_noalloc")
 
 
@@ -243,12 +285,32 @@ def tt_denoise_block_loop(d: Dims, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shif
     """Runs the loop; returns the number of steps that did work."""
     steps_run = ctypes.c_int32(0)
     _check(lib().tt_denoise_block_loop(
-        ctypes.byref(d), _ptr(k_ctx), _ptr(v_ctx), _ptr(ctx_len), _ptr(emb), _ptr(e_mask),
-        _ptr(u_t), _ptr(shift_scale), _ptr(w), float(gamma), float(logit_scale), int(max_steps),
-        _ptr(tokens), _ptr(masked), _ptr(steps_taken), _ptr(commit_step),
-        ctypes.addressof(steps_run), _ptr(ws), ws.numel(), _stream(stream)),
+        ctypes.byref(d), *_loop_args(d, 1, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale,
+                                     w),
+        float(gamma), float(logit_scale), int(max_steps),
+        *_state_args(d, tokens, masked, steps_taken, commit_step),
+        ctypes.addressof(steps_run), _ptr(ws), _nbytes(ws), _stream(stream)),
         "tt_denoise_block_loop")
     return int(steps_run.value)
+
+
+def _loop_args(d: Dims, n_layers: int, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale,
+               w) -> tuple:
+    """Checked pointers of the loop's inputs; per-layer tensors hold n_layers
+    stacked copies (layer outermost)."""
+    nl = max(int(n_layers), 0)
+    return (_sized(k_ctx, "k_ctx", nl * _ctx_bytes(d)), _sized(v_ctx, "v_ctx", nl * _ctx_bytes(d)),
+            _sized(ctx_len, "ctx_len", d.B * 4), _sized(emb, "emb", d.V * d.H * 2),
+            _sized(e_mask, "e_mask", d.H * 2), _sized(u_t, "u_t", nl * _u_t_bytes(d)),
+            _sized(shift_scale, "shift_scale", nl * 2 * d.H * 2),
+            _sized(w, "w", d.V * d.H * 2))
+
+
+def _state_args(d: Dims, tokens, masked, steps_taken, commit_step) -> tuple:
+    rows = d.B * d.S
+    return (_sized(tokens, "tokens", rows * 4), _sized(masked, "masked", rows),
+            _sized(steps_taken, "steps_taken", d.B * 4),
+            _sized(commit_step, "commit_step", rows * 4))
 
 
 def tt_decode_blocks(d: Dims, n_blocks: int, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t,
@@ -258,11 +320,15 @@ def tt_decode_blocks(d: Dims, n_blocks: int, k_ctx, v_ctx, ctx_len, emb, e_mask,
     committed (k_ctx, v_ctx and ctx_len are updated in place); returns the
     total number of steps that did work."""
     steps_run = ctypes.c_int32(0)
+    nb = max(int(n_blocks), 0)
+    rows = d.B * d.S
     _check(lib().tt_decode_blocks(
-        ctypes.byref(d), int(n_blocks), _ptr(k_ctx), _ptr(v_ctx), _ptr(ctx_len), _ptr(emb),
-        _ptr(e_mask), _ptr(u_t), _ptr(shift_scale), _ptr(w), _ptr(u_ctx), float(gamma),
-        float(logit_scale), _ptr(tokens), _ptr(steps_taken), _ptr(commit_step),
-        ctypes.addressof(steps_run), _ptr(ws), ws.numel(), _stream(stream)),
+        ctypes.byref(d), int(n_blocks),
+        *_loop_args(d, 1, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale, w),
+        _sized(u_ctx, "u_ctx", 2 * d.Hkv * d.dh * d.H * 2), float(gamma), float(logit_scale),
+        _sized(tokens, "tokens", nb * rows * 4), _sized(steps_taken, "steps_taken", nb * d.B * 4),
+        _sized(commit_step, "commit_step", nb * rows * 4),
+        ctypes.addressof(steps_run), _ptr(ws), _nbytes(ws), _stream(stream)),
         "tt_decode_blocks")
     return int(steps_run.value)
 
@@ -275,9 +341,10 @@ def tt_denoise_block_loop_layers(d: Dims, n_layers: int, k_ctx, v_ctx, ctx_len, 
     the layer outermost); returns the number of steps that did work."""
     steps_run = ctypes.c_int32(0)
     _check(lib().tt_denoise_block_loop_layers(
-        ctypes.byref(d), int(n_layers), _ptr(k_ctx), _ptr(v_ctx), _ptr(ctx_len), _ptr(emb),
-        _ptr(e_mask), _ptr(u_t), _ptr(shift_scale), _ptr(w), float(gamma), float(logit_scale),
-        int(max_steps), _ptr(tokens), _ptr(masked), _ptr(steps_taken), _ptr(commit_step),
-        ctypes.addressof(steps_run), _ptr(ws), ws.numel(), _stream(stream)),
+        ctypes.byref(d), int(n_layers),
+        *_loop_args(d, n_layers, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale, w),
+        float(gamma), float(logit_scale), int(max_steps),
+        *_state_args(d, tokens, masked, steps_taken, commit_step),
+        ctypes.addressof(steps_run), _ptr(ws), _nbytes(ws), _stream(stream)),
         "tt_denoise_block_loop_layers")
     return int(steps_run.value)

@@ -139,3 +139,57 @@ def test_binding_refuses_cpu_tensors(L):
     x = torch.zeros(4)
     with pytest.raises(ValueError):
         tt.tt_adaln_modulate(d, x, x, x, x, x)
+
+
+# ------------------------------------------- binding: buffer sizes vs the header
+def _documented_bytes(B, S, Hq, Hkv, dh, V, L_cap, n_layers, n_blocks):
+    """Bytes of every buffer argument, from the shapes include/twotower.h
+    documents for each entry point."""
+    H = Hq * dh
+    R = B * S
+    ctx = B * Hkv * L_cap * dh * 2
+    u_t = (H + 2 * Hkv * dh) * H * 2
+    vocab = dict(y=R * H * 2, w=V * H * 2, tokens=R * 4, masked=R, conf_out=R * 4,
+                 argmax_out=R * 4, n_committed=B * 4)
+    loop_in = dict(k_ctx=ctx, v_ctx=ctx, ctx_len=B * 4, emb=V * H * 2, e_mask=H * 2, u_t=u_t,
+                   shift_scale=2 * H * 2, w=V * H * 2)
+    state = dict(tokens=R * 4, masked=R, steps_taken=B * 4, commit_step=R * 4)
+    layers = dict(loop_in, **state)
+    for k in ("k_ctx", "v_ctx", "u_t", "shift_scale"):
+        layers[k] *= n_layers
+    return {
+        "tt_block_denoise_attn": dict(q_blk=R * Hq * dh * 2, k_blk=R * Hkv * dh * 2,
+                                      v_blk=R * Hkv * dh * 2, k_ctx=ctx, v_ctx=ctx,
+                                      ctx_len=B * 4, out=R * Hq * dh * 2),
+        "tt_adaln_modulate": dict(x=R * H * 2, shift_scale=2 * H * 2, t=B * 4, y=R * H * 2),
+        "tt_vocab_confidence_commit": vocab,
+        "tt_vocab_confidence_commit_noalloc": vocab,
+        "tt_denoise_block_loop": dict(loop_in, **state),
+        "tt_denoise_block_loop_layers": layers,
+        "tt_decode_blocks": dict(loop_in, u_ctx=2 * Hkv * dh * H * 2, tokens=n_blocks * R * 4,
+                                 steps_taken=n_blocks * B * 4, commit_step=n_blocks * R * 4),
+    }
+
+
+SCALARS = dict(gamma=0.8, logit_scale=1.0, max_steps=4, n_layers=3, n_blocks=2, stream=0)
+
+
+@pytest.mark.parametrize("fn", sorted(_documented_bytes(1, 1, 1, 1, 1, 1, 1, 1, 1)))
+def test_binding_checks_every_buffer_size(L, fn):
+    import inspect
+    import torch
+    shape = dict(B=2, S=16, Hq=4, Hkv=1, dh=64, V=1024, L_cap=40)
+    d = tt.Dims(shape["B"], shape["S"], shape["Hq"], shape["Hkv"], shape["dh"],
+                shape["Hq"] * shape["dh"], shape["V"], shape["L_cap"])
+    need = _documented_bytes(**shape, n_layers=SCALARS["n_layers"],
+                             n_blocks=SCALARS["n_blocks"])[fn]
+    wrapper = getattr(tt, fn)
+    params = [p for p in inspect.signature(wrapper).parameters if p != "d"]
+    buffers = [p for p in params if p not in SCALARS and p != "ws"]
+    assert sorted(buffers) == sorted(need), fn
+    for name in buffers:
+        for nbytes, message in ((need[name], "CUDA tensors only"), (need[name] - 1, "holds")):
+            kw = {p: SCALARS.get(p, FAKE) for p in params}
+            kw[name] = torch.zeros(nbytes, dtype=torch.uint8)      # a CPU buffer of that size
+            with pytest.raises(ValueError, match=message):
+                wrapper(d, **kw)
