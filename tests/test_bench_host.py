@@ -61,3 +61,40 @@ def test_attention_exponential_roof():
         r = bench.exp_roof(e, 100e-6, 148, clk)
         assert r["peak_T_per_s"] == round(16 * 148 * 1965e6 / 1e12, 3)
         assert "nominal" in r["peak_source"]
+
+
+def _reference_line(capsys, monkeypatch, *extra):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    assert bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "2",
+                       "--warmup", "3", *extra]) == 0
+    out = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(out) == 1
+    import json
+    return json.loads(out[0])
+
+
+def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
+    """The reference arm times the oracle on the host: one JSON line with the
+    same metric, unit and config as the GPU arm, its own cpu_baseline and an
+    e2e block with no host<->device bytes."""
+    j = _reference_line(capsys, monkeypatch)
+    assert j["impl"] == "reference" and j["metric"] == "committed tokens/s"
+    assert j["unit"] == "tokens/s" and j["higher_is_better"] is True
+    assert j["value"] > 0 and j["steps"] == 2 and j["warmup"] == 3 and j["n_gpus"] == 1
+    assert j["config"]["workload"].startswith("tiny-block-loop")
+    # 16 committed positions per sample; two timed samples
+    assert abs(j["ms_per_step"] * 1e-3 * j["value"] - 16) < 1e-6 * 16
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == j["value"] and cb["cores"] >= 1
+    assert "1 of 1 sequences" in cb["sample"]
+    assert j["e2e"] == {"value": j["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    assert bench.main(["--impl", "reference", "--gpus", "2", "--workload", "tiny"]) == 0
+    assert capsys.readouterr().out == ""
