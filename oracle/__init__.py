@@ -1,6 +1,6 @@
 """CPU oracle of the block-wise diffusion denoise step (test infrastructure).
 
 Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
-arm may import this package; the CUDA library never does.
+and reference arms may import this package; the CUDA library never does.
 """
 from . import twotower_oracle  # noqa: F401

@@ -1,7 +1,7 @@
 """Plain float64 CPU oracle of the block-wise diffusion denoise step.
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, the package's ``smoke()`` check and
-the benchmark's CPU-baseline arm may import this module.  The CUDA library
+the benchmark's CPU-baseline and reference arms may import this module.  The CUDA library
 never calls it, and it shares no code with the CUDA library: the only module
 both sides use is ``tt_inputs`` (seeded random draws, no method arithmetic).
 
@@ -48,7 +48,9 @@ function that uses it:
 
 Every function here is pinned by tests/test_oracle_pins.py against closed
 forms, brute force, invariants, a library softmax and the hand-worked commit
-example in tests/golden/.
+example in tests/golden/.  tests/test_oracle_mutations.py checks the pins
+themselves: it plants plausible mistakes in a copy of this file, one at a
+time, and each one must make a pin fail.
 """
 from __future__ import annotations
 
