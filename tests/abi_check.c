@@ -71,6 +71,19 @@ int main(void) {
                                      i32, i32, &steps_run, ws, ws_loop, NULL) ==
         TT_ERR_INVALID_ARG);
 
+  /* n_blocks outside 1..4096 */
+  CHECK(tt_decode_blocks(&d, 0, bf, bf, i32, bf, bf, bf, bf, bf, bf, 0.8f, 1.0f, i32, i32, i32,
+                         &steps_run, ws, ws_loop, NULL) == TT_ERR_INVALID_ARG);
+  CHECK(tt_decode_blocks(&d, 4097, bf, bf, i32, bf, bf, bf, bf, bf, bf, 0.8f, 1.0f, i32, i32, i32,
+                         &steps_run, ws, ws_loop, NULL) == TT_ERR_INVALID_ARG);
+
+  /* the allocation-free commit refuses a problem beyond its built-in scratch */
+  {
+    const tt_dims big = {128, 32, 32, 2, 128, 4096, 131072, 32768};
+    CHECK(tt_vocab_confidence_commit_noalloc(&big, bf, bf, 0.8f, 1.0f, i32, u8, f32, i32, i32,
+                                             NULL) == TT_ERR_WORKSPACE);
+  }
+
   /* the attention split knob is process-wide and bounded */
   CHECK(tt_set_attn_splits(65) == TT_ERR_INVALID_ARG);
   CHECK(tt_set_attn_splits(0) == TT_OK);

@@ -119,6 +119,11 @@ def test_commit_and_loop_argument_checks(L):
         *([FAKE] * 4), None, FAKE, wsl, None)
     assert layers(0) == 1 and "n_layers" in tt.tt_last_error()
     assert layers(65) == 1
+    blocks = lambda n: L.tt_decode_blocks(
+        ctypes.byref(d), n, *([FAKE] * 9), ctypes.c_float(0.8), ctypes.c_float(1.0),
+        *([FAKE] * 3), None, FAKE, wsl, None)
+    assert blocks(0) == 1 and "n_blocks" in tt.tt_last_error()
+    assert blocks(4097) == 1
 
 
 def test_split_knob(L):
