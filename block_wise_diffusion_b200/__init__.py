@@ -5,7 +5,9 @@ in ``libtwotower.so`` (built in-tree by ``block_wise_diffusion_b200.build``)
 with raw device pointers taken from torch tensors.  Nothing here computes:
 torch provides device memory and streams; all arithmetic runs in the
 library's sm_100a kernels.  There is no CPU path: if the library or a CUDA
-device is missing, the calls raise.
+device is missing, the calls raise.  Before a call, every tensor argument is
+checked to hold at least the bytes of the shape include/twotower.h documents
+for it, since the kernels address each buffer from the dims alone.
 """
 from __future__ import annotations
 
