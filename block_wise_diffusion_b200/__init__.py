@@ -18,7 +18,7 @@ __all__ = [
     "TTError", "Dims", "lib", "lib_path", "dims", "workspace", "tt_workspace_bytes",
     "tt_block_denoise_attn", "tt_adaln_modulate", "tt_vocab_confidence_commit",
     "tt_denoise_block_loop", "tt_denoise_block_loop_layers", "tt_decode_blocks",
-    "tt_vocab_confidence_commit_noalloc",
+    "tt_vocab_confidence_commit_noalloc", "tt_loop_last_step",
     "tt_device_status", "tt_launch_count", "tt_set_attn_splits",
     "tt_status_string", "tt_last_error", "EXPORTS", "tt_profile_enable", "tt_profile_read",
     "tt_selftest_timeout",
@@ -39,7 +39,7 @@ EXPORTS = (
     "tt_launch_count", "tt_set_attn_splits", "tt_block_denoise_attn", "tt_adaln_modulate",
     "tt_vocab_confidence_commit", "tt_denoise_block_loop", "tt_profile_enable", "tt_profile_read",
     "tt_vocab_confidence_commit_noalloc", "tt_selftest_timeout", "tt_denoise_block_loop_layers",
-    "tt_decode_blocks",
+    "tt_decode_blocks", "tt_loop_last_step",
 )
 KERNEL_KINDS = ("plan", "embed", "gemm_qkv", "attn", "merge", "adaln", "gemm_vocab", "commit",
                 "gather", "init", "splitk_reduce", "append")
@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.tt_decode_blocks.argtypes = (
             [ctypes.POINTER(Dims), ctypes.c_int32] + [_P] * 9
             + [ctypes.c_float, ctypes.c_float] + [_P] * 4 + [_P, ctypes.c_size_t, _P])
+        L.tt_loop_last_step.restype = ctypes.c_int
+        L.tt_loop_last_step.argtypes = [ctypes.POINTER(Dims), _P, ctypes.c_size_t] + [_P] * 5 + [_P]
         L.tt_denoise_block_loop_layers.restype = ctypes.c_int
         L.tt_denoise_block_loop_layers.argtypes = (
             [ctypes.POINTER(Dims), ctypes.c_int32] + [_P] * 8
@@ -350,3 +352,20 @@ def tt_denoise_block_loop_layers(d: Dims, n_layers: int, k_ctx, v_ctx, ctx_len, 
         ctypes.addressof(steps_run), _ptr(ws), _nbytes(ws), _stream(stream)),
         "tt_denoise_block_loop_layers")
     return int(steps_run.value)
+
+
+def tt_loop_last_step(d: Dims, ws, y_rows, row_ids, conf, argmax, stream=None) -> int:
+    """Copy out what the loop's last working step fed the vocabulary and the
+    commit rule (data copies only): the compacted adaLN rows into y_rows
+    [B*S, H] bf16, their row indices b*S+s into row_ids [B*S] int32, and the
+    confidence / argmax of each position masked at the start of the step into
+    conf [B*S] float32 and argmax [B*S] int32 (-1 elsewhere).  Returns the
+    number of compacted rows."""
+    rows = d.B * d.S
+    n = ctypes.c_int32(0)
+    _check(lib().tt_loop_last_step(
+        ctypes.byref(d), _ptr(ws), _nbytes(ws), _sized(y_rows, "y_rows", rows * d.H * 2),
+        _sized(row_ids, "row_ids", rows * 4), _sized(conf, "conf", rows * 4),
+        _sized(argmax, "argmax", rows * 4), ctypes.addressof(n), _stream(stream)),
+        "tt_loop_last_step")
+    return int(n.value)

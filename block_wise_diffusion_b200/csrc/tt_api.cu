@@ -22,6 +22,24 @@ static std::atomic<int> g_forced_splits{0};
 
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
 
+int num_sms() {
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    cudaGetLastError();  // no device here: clear the error and use the default
+    return kDefaultSMs;
+  }
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return kDefaultSMs;
+  }
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 // ----------------------------------------------------------------- profiler
 struct ProfRec {
   int kind;
@@ -198,18 +216,19 @@ static AttnGeom attn_geom(const tt_dims& d) {
   const long long units = (long long)d.B * d.Hkv * g.n_qtiles;
   const int ctx_tiles = (d.L_cap + kAttnBN - 1) / kAttnBN;
   const int forced = g_forced_splits.load();
+  const int sms = num_sms();
   // one CTA per (unit, split): fill the SMs once
-  int n = forced > 0 ? forced : (int)std::max<long long>(1, kNumSMs / units);
+  int n = forced > 0 ? forced : (int)std::max<long long>(1, sms / units);
   n = std::min(std::min(n, ctx_tiles + 1), 64);
   // Split 0 also runs the block's own key tile, so it gets one context tile
   // fewer: every split then runs at most c tiles, c = ceil((tiles + 1) / n).
   int c = (ctx_tiles + 1 + n - 1) / n;
-  if (forced <= 0 && units > kNumSMs) {
+  if (forced <= 0 && units > sms) {
     // More units than SMs: several waves whatever the split.  Context lengths
     // differ per sequence (and live on the device), so cap a split at about
     // an eighth of an SM's share of the largest possible work; the splits of
     // short sequences that fall past their context exit at once.
-    const long long per_sm = units * (long long)(ctx_tiles + 1) / kNumSMs;
+    const long long per_sm = units * (long long)(ctx_tiles + 1) / sms;
     c = (int)std::min<long long>(c, std::max<long long>(8, (per_sm + 7) / 8));
   }
   g.chunk = c * kAttnBN;
@@ -228,8 +247,9 @@ static int ksplit_for(const tt_dims& d, int n_out) {
   const int rows = d.B * d.S;
   const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_out + kQkvBN - 1) / kQkvBN);
   const int kb = d.H / kGemmBK;
+  const int sms = num_sms();
   int k = 1;
-  while (2 * k <= kb && kb % (2 * k) == 0 && tiles * 2 * k <= kNumSMs) k *= 2;
+  while (2 * k <= kb && kb % (2 * k) == 0 && tiles * 2 * k <= sms) k *= 2;
   return k;
 }
 static int qkv_ksplit(const tt_dims& d) { return ksplit_for(d, d.H + 2 * d.Hkv * d.dh); }
@@ -410,7 +430,7 @@ static tt_status run_vocab_gemm(const tt_dims& d, const Ws& w, const tt_bf16* W,
   a.err = w.ctrl;
   a.b_keep_tiles = keep_tiles;
   const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((d.V + kVocabBN - 1) / kVocabBN);
-  TT_LAUNCH(TT_K_GEMM_VOCAB, st, launch_gemm_vocab(tmA, tmB, a, std::min(tiles, kNumSMs), st));
+  TT_LAUNCH(TT_K_GEMM_VOCAB, st, launch_gemm_vocab(tmA, tmB, a, std::min(tiles, num_sms()), st));
   return TT_OK;
 }
 
@@ -436,6 +456,44 @@ static CommitArgs commit_args(const tt_dims& d, const Ws& w, float gamma, float 
 static tt_status read_ctrl(const Ws& w, cudaStream_t st, int* host) {
   TT_CUDA(cudaMemcpyAsync(host, w.ctrl, 8 * sizeof(int), cudaMemcpyDeviceToHost, st));
   TT_CUDA(cudaStreamSynchronize(st));
+  return TT_OK;
+}
+
+tt_status check_vocab_args(const tt_dims* d, const tt_bf16* y, const tt_bf16* w, float gamma,
+                           float logit_scale, const int32_t* tokens, const uint8_t* masked) {
+  TT_CHECK(check_dims(d));
+  TT_CHECK(check_ptr(y, "y", true));
+  TT_CHECK(check_ptr(w, "w", true));
+  TT_CHECK(check_ptr(tokens, "tokens", false));
+  TT_CHECK(check_ptr(masked, "masked", false));
+  if (!(gamma > 0.f && gamma <= 1.f))
+    return fail(TT_ERR_INVALID_ARG, "gamma=%g not in (0, 1]", (double)gamma);
+  if (!(logit_scale > 0.f) || !std::isfinite(logit_scale))
+    return fail(TT_ERR_INVALID_ARG, "logit_scale=%g must be finite and > 0", (double)logit_scale);
+  return TT_OK;
+}
+
+size_t vocab_scratch_bytes(const tt_dims& d) { return carve(d, TT_WS_VOCAB, nullptr).total; }
+
+// Plan -> row gather -> vocabulary GEMM with the confidence epilogue ->
+// commit, with the scratch carved from `scratch` (256-byte aligned, at least
+// vocab_scratch_bytes(d) bytes; the arguments already checked).
+tt_status run_vocab_commit(const tt_dims& d, void* scratch, const tt_bf16* y, const tt_bf16* W,
+                           float gamma, float logit_scale, int32_t* tokens, uint8_t* masked,
+                           float* conf_out, int32_t* argmax_out, int32_t* n_committed,
+                           cudaStream_t st) {
+  const Ws w = carve(d, TT_WS_VOCAB, scratch);
+  TT_CUDA(cudaMemsetAsync(w.ctrl, 0, w.ctrl_clear, st));
+  PlanArgs p{d.B, d.S, masked, w.rowlist, w.tvec, w.ctrl, 0};
+  TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
+  TT_LAUNCH(TT_K_GATHER, st, launch_gather_rows(y, d.H, w.y_c, d.H, w.rowlist, w.ctrl + CTRL_M,
+                                                d.B * d.S, nullptr, st));
+  TT_CHECK(run_vocab_gemm(d, w, W, logit_scale, w.ctrl + CTRL_M, nullptr, 0, st));
+  CommitArgs c = commit_args(d, w, gamma, logit_scale, tokens, masked);
+  c.conf_out = conf_out;
+  c.argmax_out = argmax_out;
+  c.n_committed = n_committed;
+  TT_LAUNCH(TT_K_COMMIT, st, launch_commit(c, st));
   return TT_OK;
 }
 
@@ -573,30 +631,11 @@ tt_status tt_vocab_confidence_commit(const tt_dims* d, const tt_bf16* y, const t
                                      uint8_t* masked, float* conf_out, int32_t* argmax_out,
                                      int32_t* n_committed, void* ws, size_t ws_bytes,
                                      void* stream) {
-  TT_CHECK(check_dims(d));
-  TT_CHECK(check_ptr(y, "y", true));
-  TT_CHECK(check_ptr(w, "w", true));
-  TT_CHECK(check_ptr(tokens, "tokens", false));
-  TT_CHECK(check_ptr(masked, "masked", false));
-  if (!(gamma > 0.f && gamma <= 1.f))
-    return fail(TT_ERR_INVALID_ARG, "gamma=%g not in (0, 1]", (double)gamma);
-  if (!(logit_scale > 0.f) || !std::isfinite(logit_scale))
-    return fail(TT_ERR_INVALID_ARG, "logit_scale=%g must be finite and > 0", (double)logit_scale);
+  TT_CHECK(check_vocab_args(d, y, w, gamma, logit_scale, tokens, masked));
   Ws ws_;
   TT_CHECK(check_ws(*d, TT_WS_VOCAB, ws, ws_bytes, &ws_));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  TT_CUDA(cudaMemsetAsync(ws_.ctrl, 0, ws_.ctrl_clear, st));
-  PlanArgs p{d->B, d->S, masked, ws_.rowlist, ws_.tvec, ws_.ctrl, 0};
-  TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
-  TT_LAUNCH(TT_K_GATHER, st, launch_gather_rows(y, d->H, ws_.y_c, d->H, ws_.rowlist, ws_.ctrl + CTRL_M,
-                             d->B * d->S, nullptr, st));
-  TT_CHECK(run_vocab_gemm(*d, ws_, w, logit_scale, ws_.ctrl + CTRL_M, nullptr, 0, st));
-  CommitArgs c = commit_args(*d, ws_, gamma, logit_scale, tokens, masked);
-  c.conf_out = conf_out;
-  c.argmax_out = argmax_out;
-  c.n_committed = n_committed;
-  TT_LAUNCH(TT_K_COMMIT, st, launch_commit(c, st));
-  return TT_OK;
+  return run_vocab_commit(*d, ws, y, w, gamma, logit_scale, tokens, masked, conf_out, argmax_out,
+                          n_committed, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // The block loop over n_layers denoiser layers (n_layers = 1: the
@@ -686,7 +725,7 @@ static tt_status denoise_block_loop_impl(
       const bool last = l == n_layers - 1;
       const tt_bf16* ss = shift_scale + (size_t)l * 2 * d->H;
       TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(l == 0 ? tmE : tmX, tmU[l], ga,
-                                                    std::min(qkv_tiles, kNumSMs), st));
+                                                    std::min(qkv_tiles, num_sms()), st));
       if (ga.ksplit > 1)
         TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
                                                           w.qkv, n_qkv, active, st));
@@ -752,6 +791,40 @@ tt_status tt_denoise_block_loop_layers(const tt_dims* d, int32_t n_layers, const
                                  steps_taken, commit_step, steps_run, ws, ws_bytes, stream);
 }
 
+tt_status tt_loop_last_step(const tt_dims* d, void* ws, size_t ws_bytes, tt_bf16* y_rows,
+                            int32_t* row_ids, float* conf, int32_t* argmax, int32_t* n_rows,
+                            void* stream) {
+  TT_CHECK(check_dims(d));
+  TT_CHECK(check_ptr(y_rows, "y_rows", true));
+  TT_CHECK(check_ptr(row_ids, "row_ids", false));
+  TT_CHECK(check_ptr(conf, "conf", false));
+  TT_CHECK(check_ptr(argmax, "argmax", false));
+  TT_CHECK(check_ptr(n_rows, "n_rows", false));
+  Ws w;
+  TT_CHECK(check_ws(*d, TT_WS_LOOP, ws, ws_bytes, &w));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int rows = d->B * d->S;
+  int h[8];
+  TT_CHECK(read_ctrl(w, st, h));
+  const int M = h[CTRL_M];
+  if (M < 0 || M > rows)
+    return fail(TT_ERR_INTERNAL, "workspace holds a row count of %d (B*S = %d): not a loop "
+                "workspace after a step", M, rows);
+  if (M > 0) {
+    TT_CUDA(cudaMemcpyAsync(y_rows, w.y_c, (size_t)M * d->H * 2, cudaMemcpyDeviceToDevice, st));
+    TT_CUDA(cudaMemcpyAsync(row_ids, w.rowlist, (size_t)M * sizeof(int), cudaMemcpyDeviceToDevice,
+                            st));
+  }
+  // per-row (confidence, token bits) pairs -> the two output arrays
+  TT_CUDA(cudaMemcpy2DAsync(conf, sizeof(float), w.rowres, sizeof(float2), sizeof(float), rows,
+                            cudaMemcpyDeviceToDevice, st));
+  TT_CUDA(cudaMemcpy2DAsync(argmax, sizeof(int32_t), reinterpret_cast<const char*>(w.rowres) + 4,
+                            sizeof(float2), sizeof(int32_t), rows, cudaMemcpyDeviceToDevice, st));
+  TT_CUDA(cudaStreamSynchronize(st));
+  *n_rows = M;
+  return TT_OK;
+}
+
 tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx, tt_bf16* v_ctx,
                            int32_t* ctx_len, const tt_bf16* emb, const tt_bf16* e_mask,
                            const tt_bf16* u_t, const tt_bf16* shift_scale, const tt_bf16* W,
@@ -799,7 +872,7 @@ tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx, t
     // The committed block joins the context: its rows of the workspace's
     // embeddings are Emb[token] (the commit re-embeds what it commits), so
     // [k | v] = Emb[token] . U_ctx^T, appended at each sequence's end.
-    TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(tmE, tmC, ga, std::min(tiles, kNumSMs), st));
+    TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(tmE, tmC, ga, std::min(tiles, num_sms()), st));
     if (ga.ksplit > 1)
       TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_kv,
                                                         w.qkv, n_kv, nullptr, st));

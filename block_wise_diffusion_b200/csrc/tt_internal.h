@@ -9,7 +9,12 @@
 namespace tt {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
-constexpr int kNumSMs = 148;
+
+// Streaming multiprocessors of the current device (cudaDevAttrMultiProcessorCount,
+// queried once per device); kDefaultSMs (a B200's count) when no device answers,
+// e.g. when workspace sizes are computed on a host without a GPU.
+constexpr int kDefaultSMs = 148;
+int num_sms();
 
 // Control block: the first 256 bytes of every workspace.
 enum CtrlWord {
@@ -199,6 +204,17 @@ void count_launch(int n = 1);
 tt_status set_error(tt_status s, const char* msg);
 // The shape checks of the public entry points.
 tt_status check_dims_public(const tt_dims* d);
+
+// The vocabulary confidence / commit step, shared by the workspace entry
+// point and the allocation-free one: argument checks, scratch bytes, and the
+// kernel sequence on a caller-chosen 256-byte-aligned scratch area.
+tt_status check_vocab_args(const tt_dims* d, const tt_bf16* y, const tt_bf16* w, float gamma,
+                           float logit_scale, const int32_t* tokens, const uint8_t* masked);
+size_t vocab_scratch_bytes(const tt_dims& d);
+tt_status run_vocab_commit(const tt_dims& d, void* scratch, const tt_bf16* y, const tt_bf16* W,
+                           float gamma, float logit_scale, int32_t* tokens, uint8_t* masked,
+                           float* conf_out, int32_t* argmax_out, int32_t* n_committed,
+                           cudaStream_t st);
 
 // Launch with programmatic dependent launch allowed: the kernel may be
 // scheduled while its predecessor in the stream is still finishing; every

@@ -76,7 +76,9 @@ TT_API const char* tt_status_string(tt_status s);
 /* Description of the last error raised on the calling thread ("" if none). */
 TT_API const char* tt_last_error(void);
 
-/* Bytes of workspace the call `which` needs for dims `d`; 0 if `d` is invalid
+/* Bytes of workspace the call `which` needs for dims `d` on the current
+ * device (the attention's split plan follows the device's SM count; a host
+ * without a GPU sizes for a B200's 148 SMs); 0 if `d` is invalid
  * (tt_last_error says why). */
 TT_API size_t tt_workspace_bytes(const tt_dims* d, int which);
 
@@ -253,8 +255,13 @@ TT_API tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, c
  *   other arguments, workspace (TT_WS_LOOP) and errors as
  *   tt_denoise_block_loop; one host synchronisation per block.
  * n_blocks outside 1..4096 is TT_ERR_INVALID_ARG.  A sequence whose cache has
- * no room for a block (ctx_len[b] + S > L_cap) is left unchanged and the call
- * returns TT_ERR_INVALID_ARG (recorded on the device).
+ * no room for a block (ctx_len[b] + S > L_cap) is found only when that block
+ * is appended, after its loop has run: the call then returns
+ * TT_ERR_INVALID_ARG (recorded on the device) with block j's tokens,
+ * steps_taken and commit_step written but nothing of block j appended for
+ * that sequence (its cache rows and ctx_len unchanged); blocks before j are
+ * complete and no later block runs.  Callers that know ctx_len on the host
+ * avoid this by checking ctx_len[b] + n_blocks*S <= L_cap first.
  */
 TT_API tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx,
                                   tt_bf16* v_ctx, int32_t* ctx_len, const tt_bf16* emb,
@@ -296,6 +303,36 @@ TT_API tt_status tt_denoise_block_loop_layers(const tt_dims* d, int32_t n_layers
                                               void* stream);
 
 /*
+ * Inspection of the block loop's last step: data copies only, no arithmetic.
+ * After tt_denoise_block_loop or tt_denoise_block_loop_layers has returned,
+ * its workspace still holds what the last step that did work fed the
+ * vocabulary projection - the adaLN rows of the positions masked at the
+ * start of that step, compacted in row order - and the confidence and
+ * argmax token the commit rule used for each of them.  This call copies them
+ * out, so a caller can check the projection and the commit rule on the
+ * kernels' own rows (run the loop with max_steps = 1 to see every step; a
+ * resumed loop continues exactly where the previous call stopped).  Source
+ * of the quantities: gist.science summary, "Training and Conditioning",
+ * Sampling (all masked positions are predicted in parallel; confident ones
+ * commit).
+ *
+ *   ws, ws_bytes  the TT_WS_LOOP workspace the loop ran with (read only)
+ *   y_rows   bf16 [B*S, H]  rows 0 .. n_rows-1 receive the compacted rows,
+ *            the rest are left untouched
+ *   row_ids  int32 [B*S]    row_ids[j] = b*S + s of compacted row j (j < n_rows)
+ *   conf     float [B*S]    confidence of each position masked at the start
+ *            of the step, -1 elsewhere
+ *   argmax   int32 [B*S]    its argmax token, -1 elsewhere
+ *   n_rows   host int32     number of compacted rows
+ * Blocking: synchronises `stream` (the loop's stream) before reading.  A
+ * workspace whose row count is out of range (never used by a loop) gives
+ * TT_ERR_INTERNAL.
+ */
+TT_API tt_status tt_loop_last_step(const tt_dims* d, void* ws, size_t ws_bytes, tt_bf16* y_rows,
+                                   int32_t* row_ids, float* conf, int32_t* argmax,
+                                   int32_t* n_rows, void* stream);
+
+/*
  * Allocation-free variant of tt_vocab_confidence_commit.
  * The paper has no counterpart: this entry point exists for callers that
  * cannot provide a workspace - code running inside another runtime's
@@ -315,7 +352,11 @@ TT_API tt_status tt_denoise_block_loop_layers(const tt_dims* d, int32_t n_layers
  * no cudaMalloc/cudaFree and no allocating library routine.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is cached per device together
+ *    with the identity of the context it belongs to, and looked up again
+ *    when the current context differs (after a device reset, whose new
+ *    context loads the array anew); a call that does this look-up must not
+ *    be captured either.
  *  - All calls share the one array and it keeps the last call's contents;
  *    the call clears what must start at zero.  Calls whose work overlaps on
  *    the GPU (different streams, or several host threads) race on it:

@@ -77,6 +77,16 @@ int main(void) {
   CHECK(tt_decode_blocks(&d, 4097, bf, bf, i32, bf, bf, bf, bf, bf, bf, 0.8f, 1.0f, i32, i32, i32,
                          &steps_run, ws, ws_loop, NULL) == TT_ERR_INVALID_ARG);
 
+  /* the last-step inspection needs a whole loop workspace and an n_rows slot */
+  {
+    int32_t n_rows = -3;
+    CHECK(tt_loop_last_step(&d, ws, ws_loop, bf, i32, f32, i32, NULL, NULL) ==
+          TT_ERR_INVALID_ARG);
+    CHECK(tt_loop_last_step(&d, ws, ws_vocab, bf, i32, f32, i32, &n_rows, NULL) ==
+          TT_ERR_WORKSPACE);
+    CHECK(n_rows == -3);
+  }
+
   /* the allocation-free commit refuses a problem beyond its built-in scratch */
   {
     const tt_dims big = {128, 32, 32, 2, 128, 4096, 131072, 32768};

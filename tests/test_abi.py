@@ -124,6 +124,13 @@ def test_commit_and_loop_argument_checks(L):
         *([FAKE] * 3), None, FAKE, wsl, None)
     assert blocks(0) == 1 and "n_blocks" in tt.tt_last_error()
     assert blocks(4097) == 1
+    n_rows = ctypes.c_int32(-3)
+    last = lambda ws_bytes, out: L.tt_loop_last_step(
+        ctypes.byref(d), FAKE, ws_bytes, FAKE, FAKE, FAKE, FAKE, out, None)
+    assert last(wsl, None) == 1 and "n_rows" in tt.tt_last_error()
+    assert last(wsl - 1, ctypes.addressof(n_rows)) == 3
+    assert last(tt.tt_workspace_bytes(d, tt.TT_WS_VOCAB), ctypes.addressof(n_rows)) == 3
+    assert n_rows.value == -3                               # nothing written on refusal
 
 
 def test_split_knob(L):
@@ -173,6 +180,7 @@ def _documented_bytes(B, S, Hq, Hkv, dh, V, L_cap, n_layers, n_blocks):
         "tt_denoise_block_loop_layers": layers,
         "tt_decode_blocks": dict(loop_in, u_ctx=2 * Hkv * dh * H * 2, tokens=n_blocks * R * 4,
                                  steps_taken=n_blocks * B * 4, commit_step=n_blocks * R * 4),
+        "tt_loop_last_step": dict(y_rows=R * H * 2, row_ids=R * 4, conf=R * 4, argmax=R * 4),
     }
 
 

@@ -45,11 +45,16 @@ def _with_workspace(D, d, y, w, gamma, scale, tokens, masked):
 
 
 def _no_alloc(D, d, y, w, gamma, scale, tokens, masked):
+    """One call, with every buffer allocated beforehand; returns its outputs
+    and the device's free memory just before and just after the call."""
     tk, mk = torch.from_numpy(tokens).cuda(), torch.from_numpy(masked).cuda()
     conf, amax, ncom = _outputs(d)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
     tt.tt_vocab_confidence_commit_noalloc(D, y, w, gamma, scale, tk, mk, conf, amax, ncom)
     torch.cuda.synchronize()
-    return [t.cpu().numpy() for t in (tk, mk, conf, amax, ncom)]
+    free1 = torch.cuda.mem_get_info()[0]
+    return [t.cpu().numpy() for t in (tk, mk, conf, amax, ncom)], (free0, free1)
 
 
 @pytest.mark.gpu
@@ -62,7 +67,11 @@ def test_no_alloc_matches_workspace_entry_point_twice(wl, B, scale, frac):
     for seed in (1, 2):                       # two calls in a row, different inputs
         y, w, tokens, masked = _case(d, seed, frac)
         ref = _with_workspace(D, d, y, w, gamma, scale, tokens, masked)
-        got = _no_alloc(D, d, y, w, gamma, scale, tokens, masked)
+        got, (free0, free1) = _no_alloc(D, d, y, w, gamma, scale, tokens, masked)
+        if seed == 2:
+            # the array and the kernels are loaded by now: a call takes no
+            # device memory at all
+            assert free1 == free0, (free0, free1)
         for name, a, b in zip(("tokens", "masked", "conf", "argmax", "n_committed"), got, ref):
             if name == "conf":
                 np.testing.assert_allclose(a, b, rtol=2e-4, err_msg=f"seed {seed}: {name}")
