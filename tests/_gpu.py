@@ -34,43 +34,26 @@ def rel_l2(a, b) -> float:
 
 
 def assert_close_bf16(got, ref, what=""):
+    """The attention bar: max-abs <= 2e-2 and rel-L2 <= 1e-2.  With the literal
+    input scale the outputs are of order 1e-3, where the absolute bound says
+    little, so max-abs is also held to 2e-2 of the output's own largest
+    magnitude; the margins are printed for every case."""
     err = np.abs(got - ref).max()
     rl = rel_l2(got, ref)
+    scale = float(np.abs(ref).max())
+    print(f"{what}: max-abs {err:.3e} (bound {MAX_ABS:g}; {err / max(scale, 1e-30):.3e} of "
+          f"max|ref| {scale:.3e}), rel-L2 {rl:.3e} (bound {REL_L2:g})")
     assert np.isfinite(got).all(), f"{what}: non-finite output"
     assert err <= MAX_ABS and rl <= REL_L2, f"{what}: max-abs {err:.3e} rel-L2 {rl:.3e}"
+    assert err <= MAX_ABS * scale, f"{what}: max-abs {err:.3e} against max|ref| {scale:.3e}"
     return err, rl
 
 
-# Near-tie exclusions.  The literal rule (confidence within 1e-3 of gamma, or
-# top-2 probability gap below 1e-3) is counted and reported; the tests apply
-# the narrower rule below, derived from fp32 accumulation error (logit errors
-# of order 1e-5 here), so that far more positions are compared bit-exactly.
-TIE_LOGIT = 2e-3      # top-2 logit gap (after logit_scale) below this: argmax excluded
-TIE_CONF_REL = 1e-3   # |conf - gamma| / gamma below this: threshold decision excluded
-TIE_FALLBACK_REL = 1e-4  # fallback between confidences this close (relative): excluded
-
-
-# End-to-end loop comparison (teacher-forced on tokens and mask only): the
-# oracle recomputes attention and y in float64, so its logits differ from the
-# kernel's by the attention difference the parity bar allows, carried through
-# LayerNorm (unit-variance rows) and a W row of unit norm.  Measured attention
-# differences are a few 1e-3 relative, i.e. logit differences of order
-# 1e-3..1e-2 per unit of logit_scale.  A committed token may therefore be the
-# oracle's runner-up when the oracle's top-2 gap is below this (times
-# logit_scale); it must still be one of the oracle's two best tokens.
-LOOP_TIE_LOGIT = 2e-2
-
-
-def spec_excluded(conf, gap_p, gamma):
-    return (np.abs(conf - gamma) < 1e-3) | (gap_p < 1e-3)
-
-
-def derived_excluded_argmax(gap_l):
-    return gap_l < TIE_LOGIT
-
-
-def derived_excluded_threshold(conf, gamma):
-    return np.abs(conf - gamma) < TIE_CONF_REL * gamma
+# Near-tie exclusion rules and the end-to-end loop comparison live with the
+# oracle (oracle/parity.py), so the benchmark's sampled check counts the same way.
+from oracle.parity import (LOOP_TIE_LOGIT, TIE_CONF_REL, TIE_FALLBACK_REL,  # noqa: E402,F401
+                           TIE_LOGIT, derived_excluded_argmax, derived_excluded_threshold,
+                           fallback_near_tie, spec_excluded)
 
 
 def workspace(d, which):

@@ -83,11 +83,14 @@ def test_reference_arm_prints_the_contract_line(capsys, monkeypatch):
     assert j["unit"] == "tokens/s" and j["higher_is_better"] is True
     assert j["value"] > 0 and j["steps"] == 2 and j["warmup"] == 3 and j["n_gpus"] == 1
     assert j["config"]["workload"].startswith("tiny-block-loop")
-    # 16 committed positions per sample; two timed samples
-    assert abs(j["ms_per_step"] * 1e-3 * j["value"] - 16) < 1e-6 * 16
+    # a sample is the first REF_SAMPLE_STEPS denoise steps of one sequence's
+    # block; at unit logit scale each commits one position
+    n = bench.REF_SAMPLE_STEPS
+    assert abs(j["ms_per_step"] * 1e-3 * j["value"] - n) < 1e-6 * n
+    assert j["denoise_steps_per_s"] == j["value"]
     cb = j["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == j["value"] and cb["cores"] >= 1
-    assert "1 of 1 sequences" in cb["sample"]
+    assert "1 of 1 sequences" in cb["sample"] and f"first {n} denoise steps" in cb["sample"]
     assert j["e2e"] == {"value": j["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
 
@@ -98,3 +101,17 @@ def test_reference_arm_other_ranks_exit_quietly(capsys, monkeypatch):
     monkeypatch.setenv("LOCAL_RANK", "1")
     assert bench.main(["--impl", "reference", "--gpus", "2", "--workload", "tiny"]) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_both_roofs_reports_each_view():
+    d = tt_inputs.workload("loop64")
+    inp = {"ctx_len": np.full(d.B, d.L_cap, np.int32)}
+    r = bench.both_roofs("attn", d, inp, [], 16, 100e-6, PEAKS)
+    by, fl = bench.per_launch("attn", d, inp, [], 16)
+    assert r["hbm"]["bytes_per_launch"] == by[0] and r["tensor"]["flops_per_launch"] == fl[0]
+    assert abs(r["hbm"]["achieved_GB_per_s"] - round(by[0] / 100e-6 / 1e9, 1)) < 1e-9
+    assert r["hbm"]["frac_of_8TBps"] == round(by[0] / 100e-6 / 1e9 / 8000.0, 4)
+    assert r["tensor"]["frac_of_sustained"] == round(fl[0] / 100e-6 / 1e12 / 1361.8, 4)
+    ms = [1024 - 64 * k for k in range(16)]
+    v = bench.both_roofs("gemm_vocab", d, inp, ms, 16, 450e-6, PEAKS)
+    assert v["tensor"]["flops_per_launch"] == sum(2.0 * m * d.V * d.H for m in ms) / 16

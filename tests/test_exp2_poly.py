@@ -1,4 +1,4 @@
-"""The attention kernel evaluates a quarter of its exponentials with a cubic
+"""The attention kernel evaluates an eighth of its exponentials with a cubic
 on the FMA pipe (exp2_poly in csrc/tt_attn.cu).  This re-evaluates that
 routine in float32 with the coefficients read from the kernel source and
 checks it against the exact 2^x: relative error below 1e-4 (P is then

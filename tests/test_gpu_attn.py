@@ -66,6 +66,14 @@ CASES = [
      np.array([500, 77]), True),
     ("block-S64-g4", tt_inputs.Dims(B=2, S=64, Hq=8, Hkv=2, dh=64, V=512, L_cap=300,
                                     ctx=("fixed", 300)), np.array([300, 0]), True),
+    # the top of the accepted envelope: G = 32, 64 and 128 query heads per KV
+    # head (a 128-row half holds 4, 2 or 1 block positions), H = 8192
+    ("gqa32", tt_inputs.Dims(B=2, S=16, Hq=32, Hkv=1, dh=64, V=512, L_cap=300,
+                             ctx=("fixed", 300)), np.array([300, 45]), True),
+    ("gqa64-H8192", tt_inputs.Dims(B=1, S=16, Hq=64, Hkv=1, dh=128, V=512, L_cap=150,
+                                   ctx=("fixed", 150)), np.array([150]), True),
+    ("gqa128-H8192", tt_inputs.Dims(B=2, S=32, Hq=128, Hkv=1, dh=64, V=512, L_cap=200,
+                                    ctx=("fixed", 200)), np.array([200, 3]), True),
 ]
 
 

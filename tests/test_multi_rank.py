@@ -54,3 +54,34 @@ def test_single_rank_is_identity():
     assert bench.reduce_max(3.5, 1) == 3.5
     assert bench.reduce_sum(2.0, 1) == 2.0
     assert bench.rank_seed(7, 0) == 7
+
+
+def test_gpus_n_without_a_launcher_starts_n_ranks(capfd, monkeypatch):
+    """bench.py --gpus 2 with no launcher starts the two ranks itself (here the
+    oracle arm, which needs no GPU: rank 0 prints the record, rank 1 exits)."""
+    import json
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT"):
+        monkeypatch.delenv(k, raising=False)
+    rc = bench.main(["--impl", "reference", "--workload", "tiny", "--gpus", "2", "--steps", "1",
+                     "--warmup", "3"])
+    out, err = capfd.readouterr()
+    assert rc == 0, err[-2000:]
+    assert "torch.distributed.run" in err and "--nproc-per-node=2" in err
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["n_gpus"] == 2
+
+
+def test_gpus_n_refuses_rather_than_running_one_replica(capfd, monkeypatch):
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    import torch
+    if torch.cuda.device_count() < 2:
+        assert bench.main(["--gpus", "2"]) == 2          # too few GPUs: an error, no record
+        assert "visible GPU" in capfd.readouterr().err
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "0")
+    assert bench.main(["--gpus", "4"]) == 2               # launcher and request disagree
+    out, err = capfd.readouterr()
+    assert out == "" and "WORLD_SIZE=2" in err
