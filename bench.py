@@ -4,17 +4,21 @@
 One step = one tt_denoise_block_loop call: a block of S masked positions per
 sequence is refined (re-embed + linear update -> block-denoise attention ->
 adaLN -> vocab GEMM with fused confidence -> commit) until every position is
-committed.  Default workload: 8 sequences, 32 query / 2 KV heads (GQA 16),
-d_head 128, hidden 4096, context 4096, S = 16, V = 131072, gamma 0.8, unit
-logit scale; synthetic seeded inputs resident in HBM.
+committed.  Default workload: the full block loop of 64 sequences, 32 query /
+2 KV heads (GQA 16), d_head 128, hidden 4096, context 8192, S = 16,
+V = 131072, gamma 0.8, unit logit scale; synthetic seeded inputs resident in
+HBM (``--workload`` picks the other shapes).
 
 Metric: committed tokens/s (whole job), with denoise steps/s alongside.
 Timing: CUDA events on the library's stream around each call, an L2 flush
 (256 MiB write) between calls outside the events, max over ranks.
 `--impl reference` times the float64 CPU oracle on a bounded sample instead.
+`--stage attn|vocab|blocks` times one other entry point on its own (for
+profilers; prints a plain line, not the benchmark record).
 
-Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
-torch.distributed.run (one rank per GPU, independent replicas, weak scaling).
+Launch: python bench.py [--gpus N --steps K --warmup W].  N > 1 runs one
+independent replica per GPU (weak scaling); under torch.distributed.run each
+process is one rank, and without a launcher bench.py starts N ranks itself.
 """
 from __future__ import annotations
 
@@ -55,7 +59,15 @@ def parse_args(argv=None):
     p.add_argument("--steps", type=int, default=10)
     p.add_argument("--warmup", type=int, default=3)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default="mid", choices=sorted(tt_inputs.WORKLOADS))
+    p.add_argument("--workload", default="loop64", choices=sorted(tt_inputs.WORKLOADS))
+    p.add_argument("--stage", default="loop", choices=["loop", "attn", "vocab", "blocks"],
+                   help="loop: the benchmark; attn / vocab / blocks: time one entry point "
+                        "alone (tt_block_denoise_attn, tt_vocab_confidence_commit with every "
+                        "position masked, tt_decode_blocks) for profilers")
+    p.add_argument("--B", type=int, default=None, help="--stage runs: override the batch")
+    p.add_argument("--V", type=int, default=None, help="--stage runs: override the vocabulary")
+    p.add_argument("--calls", type=int, default=2, help="--stage runs: timed calls")
+    p.add_argument("--n-blocks", type=int, default=4, help="--stage blocks: blocks per call")
     p.add_argument("--gamma", type=float, default=0.8)
     p.add_argument("--logit-scale", type=float, default=1.0)
     p.add_argument("--seed", type=int, default=0)
@@ -202,23 +214,48 @@ def gpu_uuid(torch, idx):
 
 
 # -------------------------------------------------------- CPU oracle arm
-def oracle_sample(d, inp, gamma, logit_scale, n_seq=3):
-    """Run the oracle's block loop on the first n_seq sequences of the workload
-    (a bounded sample: about 5 s of float64 work per sequence at the mid shapes)."""
-    from oracle import twotower_oracle as O
-    n_seq = min(n_seq, d.B)
+def sample_inputs(inp, bsel):
+    """The loop inputs restricted to the sequences ``bsel``."""
     one = dict(inp)
     for k in ("k_ctx", "v_ctx", "ctx_len", "tokens", "masked"):
-        one[k] = inp[k][:n_seq]
+        one[k] = inp[k][bsel]
     for k in ("k_ctx_l", "v_ctx_l"):
         if k in inp:
-            one[k] = inp[k][:, :n_seq]
+            one[k] = inp[k][:, bsel]
+    return one
+
+
+def oracle_sample(d, inp, gamma, logit_scale, n_seq=1, max_steps=None):
+    """Run the oracle's block loop on the first n_seq sequences of the workload
+    (all its steps, or the first max_steps): a bounded sample.  Returns
+    (seconds, committed positions, steps, n_seq)."""
+    from oracle import twotower_oracle as O
+    n_seq = min(n_seq, d.B)
+    one = sample_inputs(inp, slice(0, n_seq))
     t0 = time.perf_counter()
-    r = O.denoise_block_loop(one, gamma, logit_scale)
+    r = O.denoise_block_loop(one, gamma, logit_scale, max_steps=max_steps)
     dt = time.perf_counter() - t0
-    committed = int(inp["masked"][:n_seq].sum())
-    steps = len(r["trace"])
-    return dt, committed, steps, n_seq
+    committed = int((one["masked"].astype(bool) & ~r["masked"]).sum())
+    return dt, committed, len(r["trace"]), n_seq
+
+
+def oracle_check(d, inp, gamma, logit_scale, g_tokens, g_commit_step, bsel):
+    """The CPU-baseline leg: the oracle's block loop on the sequences ``bsel``,
+    teacher-forced on the GPU's trajectory of the timed call, timed on the
+    host cores; its comparison with the GPU's committed tokens gives the
+    parity counts (oracle.parity.compare_loop: compared and excluded
+    sequence-steps, literal-rule exclusions, near-tie top-2 flips,
+    disagreements outside the exclusions).  Returns (seconds, committed
+    positions, counts)."""
+    from oracle import parity as P
+    one = sample_inputs(inp, bsel)
+    t0 = time.perf_counter()
+    cnt, problems = P.compare_loop(one, g_tokens[bsel], g_commit_step[bsel], gamma, logit_scale)
+    dt = time.perf_counter() - t0
+    cnt["mismatches"] = len(problems)
+    if problems:
+        log("parity: " + "; ".join(problems[:5]))
+    return dt, int(one["masked"].sum()), cnt
 
 
 def blas_threads() -> int:
@@ -232,6 +269,12 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
+# denoise steps of one sequence's block that one reference-arm step runs
+# (the whole block when it has at most this many), so that the driver's
+# --steps 20 --warmup 5 run stays within a few minutes at the large shapes
+REF_SAMPLE_STEPS = 4
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -239,15 +282,17 @@ def run_reference(args, rank, world):
     inp = tt_inputs.generate(d, seed=rank_seed(args.seed, 0), n_layers=args.n_layers)
     times, tokens, steps = [], 0, 0
     for i in range(args.warmup + args.steps):
-        dt, c, s, _ = oracle_sample(d, inp, args.gamma, args.logit_scale, n_seq=1)
+        dt, c, s, _ = oracle_sample(d, inp, args.gamma, args.logit_scale, n_seq=1,
+                                    max_steps=REF_SAMPLE_STEPS)
         if i >= args.warmup:
             times.append(dt)
             tokens += c
             steps += s
     total = sum(times)
     value = tokens / total
-    sample = (f"1 of {d.B} sequences of the workload per step, full block loop "
-              f"({steps // max(1, args.steps)} denoise steps), float64 NumPy oracle")
+    sample = (f"1 of {d.B} sequences of the workload per step, the first "
+              f"{steps // max(1, args.steps)} denoise steps of its block "
+              f"({tokens // max(1, args.steps)} committed positions), float64 NumPy oracle")
     cores = blas_threads()
     line = {
         "impl": "reference", "metric": "committed tokens/s", "value": value,
@@ -266,19 +311,11 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------ GPU arm
-def algorithmic(kind, d, inp, m_per_launch, launches, peaks):
-    """(bound, algorithmic bytes or FLOPs per launch, unit, roofline time s) of a
-    kernel kind over its launches.
-
-    Each launch has algorithmic bytes and FLOPs; its floor is the larger of
-    bytes / HBM peak and FLOPs / sustained bf16 peak.  The bound reported is
-    the one whose floors dominate the sum over launches (the vocabulary GEMM
-    is HBM-bound at a few hundred rows and tensor-bound above; attention sits
-    at the ridge).  ``m_per_launch`` lists the vocabulary GEMM's rows per
-    launch (the still-masked positions of each step).
-    """
-    hbm = peaks["hbm_gbs"] * 1e9
-    tc = peaks["bf16_tflops_sustained"] * 1e12
+def per_launch(kind, d, inp, m_per_launch, launches):
+    """Algorithmic bytes and FLOPs of each launch of a kernel kind (lists), or
+    (None, None) for a kind without a roofline model.  ``m_per_launch`` lists
+    the vocabulary GEMM's rows per launch (the still-masked positions of each
+    step)."""
     if kind == "gemm_vocab":
         n_vt = -(-d.V // 224)
         ms = list(m_per_launch)[:launches] or [0]
@@ -295,7 +332,25 @@ def algorithmic(kind, d, inp, m_per_launch, launches, peaks):
         by = [n_qkv * d.H * 2 + d.B * d.S * (d.H + n_qkv) * 2] * launches
         fl = [2.0 * d.B * d.S * d.H * n_qkv] * launches
     else:
+        return None, None
+    return by, fl
+
+
+def algorithmic(kind, d, inp, m_per_launch, launches, peaks):
+    """(bound, algorithmic bytes or FLOPs per launch, unit, roofline time s) of a
+    kernel kind over its launches.
+
+    Each launch has algorithmic bytes and FLOPs; its floor is the larger of
+    bytes / HBM peak and FLOPs / sustained bf16 peak.  The bound reported is
+    the one whose floors dominate the sum over launches (the vocabulary GEMM
+    is HBM-bound at a few hundred rows and tensor-bound above; attention sits
+    at the ridge).
+    """
+    by, fl = per_launch(kind, d, inp, m_per_launch, launches)
+    if by is None:
         return None, None, None, None
+    hbm = peaks["hbm_gbs"] * 1e9
+    tc = peaks["bf16_tflops_sustained"] * 1e12
     t_h = sum(b / hbm for b in by)
     t_t = sum(f / tc for f in fl)
     t_roof = sum(max(b / hbm, f / tc) for b, f in zip(by, fl))
@@ -309,6 +364,27 @@ def algorithmic(kind, d, inp, m_per_launch, launches, peaks):
 # independent chains per thread).
 MUFU_EX2_PER_CLK_SM = 16
 NOMINAL_MAX_SM_MHZ = 1965.0
+
+
+SPEC_HBM_GBS = 8000.0  # the B200 spec sheet's ~8 TB/s, for context beside the measured copy
+
+
+def both_roofs(kind, d, inp, m_per_launch, launches, avg_s, peaks):
+    """A kernel's standing against both roofs, whichever bounds it: achieved
+    HBM GB/s (algorithmic bytes per launch / time) against the measured copy
+    bandwidth and against the spec sheet's 8 TB/s, and achieved TFLOP/s
+    against the sustained and burst dense-bf16 peaks (the tensor-pipe share
+    the algorithmic FLOPs need)."""
+    bl, fll = per_launch(kind, d, inp, m_per_launch, launches)
+    by, fl = sum(bl) / len(bl), sum(fll) / len(fll)
+    gbs = by / avg_s / 1e9
+    tfs = fl / avg_s / 1e12
+    return {"hbm": {"achieved_GB_per_s": round(gbs, 1), "bytes_per_launch": by,
+                    "frac_of_measured": round(gbs / peaks["hbm_gbs"], 4),
+                    "frac_of_8TBps": round(gbs / SPEC_HBM_GBS, 4)},
+            "tensor": {"achieved_TFLOP_per_s": round(tfs, 1), "flops_per_launch": fl,
+                       "frac_of_sustained": round(tfs / peaks["bf16_tflops_sustained"], 4),
+                       "frac_of_burst": round(tfs / peaks["bf16_tflops"], 4)}}
 
 
 def attn_exp_per_launch(d, inp):
@@ -474,6 +550,10 @@ def run_ours(args, rank, world, local):
         if kind == "attn":
             e["exp"] = exp_roof(attn_exp_per_launch(d, inp), kms / n / 1e3, n_sm, clk)
         kernels[kind] = e
+    for kind in ("attn", "gemm_vocab"):
+        if kind in kernels:
+            kms, n = table[kind]
+            kernels[kind].update(both_roofs(kind, d, inp, m_per_step, n, kms / n / 1e3, peaks))
     dom = max(table, key=lambda k: table[k][0])
     bound, per, unit, t_roof = algorithmic(dom, d, inp, m_per_step, table[dom][1], peaks)
     roofline = None
@@ -488,12 +568,17 @@ def run_ours(args, rank, world, local):
                     "algorithmic_per_launch": per,
                     "roofline_time_frac": round(t_roof / (table[dom][0] / 1e3), 4)}
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, c, s, n = oracle_sample(d, inp, args.gamma, args.logit_scale)
+        # the first and the last sequence of the timed batch (its last call)
+        bsel = np.array(sorted({0, d.B - 1}))
+        dt, c, cnt = oracle_check(d, inp, args.gamma, args.logit_scale,
+                                  tokens.cpu().numpy(), commit_step.cpu().numpy(), bsel)
         cpu = {"value": c / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": f"{n} of {d.B} sequences of the workload, full block loop ({s} denoise "
-                         f"steps, {dt:.1f} s), float64 NumPy oracle"}
+               "sample": f"sequences {bsel.tolist()} of {d.B}, full block loop ({dt:.1f} s), "
+                         "float64 NumPy oracle, teacher-forced on the timed call's trajectory"}
+        parity = dict(cnt, sample=f"sequences {bsel.tolist()} of the last timed call, end to end "
+                                  "against the float64 oracle; exclusions as oracle/parity.py")
 
     if world > 1:
         import torch.distributed as dist
@@ -514,17 +599,157 @@ def run_ours(args, rank, world, local):
         "roofline": roofline,
         "kernels": kernels,
         "cpu_baseline": cpu,
+        "parity": parity,
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
+# --------------------------------------------------- single-stage runs
+def _dev_bf16(bits):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def stage_attn(d):
+    """(call, check) for tt_block_denoise_attn on seeded inputs."""
+    import torch
+    import block_wise_diffusion_b200 as tt
+    inp = tt_inputs.generate(d, seed=0, names=["q_blk", "k_blk", "v_blk", "k_ctx", "v_ctx"])
+    q, kb, vb, kc, vc = (_dev_bf16(inp[k]) for k in ("q_blk", "k_blk", "v_blk", "k_ctx", "v_ctx"))
+    cl = torch.from_numpy(inp["ctx_len"]).cuda()
+    D = tt.dims(d)
+    out = torch.empty((d.B, d.S, d.Hq, d.dh), dtype=torch.bfloat16, device="cuda")
+    ws = tt.workspace(D, tt.TT_WS_ATTN)
+
+    def call():
+        tt.tt_block_denoise_attn(D, q, kb, vb, kc, vc, cl, out, ws)
+
+    return call, lambda: tt.tt_device_status(ws)
+
+
+def stage_vocab(d):
+    """(call, check) for tt_vocab_confidence_commit with every position masked
+    (all B*S rows go through the GEMM)."""
+    import torch
+    import block_wise_diffusion_b200 as tt
+    inp = tt_inputs.generate(d, seed=0, names=["w"])
+    rng = np.random.default_rng(0)
+    y = _dev_bf16(tt_inputs.bf16_bits(rng.standard_normal((d.B * d.S, d.H)).astype(np.float32)))
+    w = _dev_bf16(inp["w"])
+    D = tt.dims(d)
+    ws = tt.workspace(D, tt.TT_WS_VOCAB)
+    tok = torch.full((d.B, d.S), -1, dtype=torch.int32, device="cuda")
+    msk0 = torch.ones((d.B, d.S), dtype=torch.uint8, device="cuda")
+    msk = msk0.clone()
+    conf = torch.empty((d.B, d.S), dtype=torch.float32, device="cuda")
+    am = torch.empty((d.B, d.S), dtype=torch.int32, device="cuda")
+    nc = torch.empty((d.B,), dtype=torch.int32, device="cuda")
+
+    def call():
+        msk.copy_(msk0)  # the call commits positions: start every call fully masked
+        tt.tt_vocab_confidence_commit(D, y, w, 0.8, 1.0, tok, msk, conf, am, nc, ws)
+
+    return call, lambda: tt.tt_device_status(ws)
+
+
+def stage_blocks(d, n_blocks, logit_scale):
+    """(call, check) for tt_decode_blocks over n_blocks blocks (the context is
+    reset before each call)."""
+    import torch
+    import block_wise_diffusion_b200 as tt
+    inp = tt_inputs.generate(d, seed=0)
+    kc0, vc0 = _dev_bf16(inp["k_ctx"]), _dev_bf16(inp["v_ctx"])
+    kc, vc = kc0.clone(), vc0.clone()
+    cl0 = torch.from_numpy(inp["ctx_len"]).cuda()
+    cl = cl0.clone()
+    X = {k: _dev_bf16(inp[k]) for k in ("emb", "e_mask", "u_t", "shift_scale", "w", "u_ctx")}
+    D = tt.dims(d)
+    tok = torch.empty((n_blocks, d.B, d.S), dtype=torch.int32, device="cuda")
+    steps = torch.empty((n_blocks, d.B), dtype=torch.int32, device="cuda")
+    cs = torch.empty((n_blocks, d.B, d.S), dtype=torch.int32, device="cuda")
+    ws = tt.workspace(D, tt.TT_WS_LOOP)
+
+    def call():
+        kc.copy_(kc0)
+        vc.copy_(vc0)
+        cl.copy_(cl0)
+        tt.tt_decode_blocks(D, n_blocks, kc, vc, cl, X["emb"], X["e_mask"], X["u_t"],
+                            X["shift_scale"], X["w"], X["u_ctx"], 0.8, logit_scale, tok, steps,
+                            cs, ws)
+
+    return call, lambda: tt.tt_device_status(ws)
+
+
+def run_stage(args) -> int:
+    """One entry point on its own: a warm-up call, then --calls calls timed
+    together with CUDA events (no L2 flush), then the device status word."""
+    import dataclasses
+    import torch
+    import block_wise_diffusion_b200 as tt
+    tt.lib()
+    over = {k: v for k, v in (("B", args.B), ("V", args.V)) if v is not None}
+    d = tt_inputs.workload(args.workload, **over)
+    if args.stage == "blocks":
+        d = dataclasses.replace(d, L_cap=d.L_cap + args.n_blocks * d.S)  # room for the blocks
+        call, check = stage_blocks(d, args.n_blocks, args.logit_scale)
+    else:
+        call, check = (stage_attn if args.stage == "attn" else stage_vocab)(d)
+    call()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(args.calls):
+        call()
+    ev[1].record()
+    torch.cuda.synchronize()
+    if check() != 0:
+        raise RuntimeError("device reported an error")
+    us = ev[0].elapsed_time(ev[1]) * 1e3 / args.calls
+    msg = f"ok {args.stage} {d}: {us:.1f} us per call (mean of {args.calls}, no L2 flush)"
+    if args.stage == "blocks":
+        msg += f", {args.n_blocks * d.B * d.S / (us * 1e-6):.0f} committed tokens/s"
+    print(msg, flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- launch
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(n: int, argv) -> int:
+    """Run this script as n local ranks under torch.distributed.run (one per
+    GPU, rendezvous on 127.0.0.1) and return its exit status; rank 0 prints
+    the record."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={free_port()}",
+           os.path.abspath(__file__), *argv]
+    log("launching: " + " ".join(cmd))
+    return subprocess.call(cmd)
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     args = parse_args(argv)
     rank, world, local = dist_env()
-    if args.gpus != world and world != 1:
-        log(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.stage != "loop":
+        return run_stage(args)
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # no launcher: start the ranks here rather than run one replica
+        if args.impl == "ours":
+            import torch
+            n = torch.cuda.device_count()
+            if n < args.gpus:
+                log(f"error: --gpus {args.gpus} but this host has {n} visible GPU(s)")
+                return 2
+        return spawn_ranks(args.gpus, argv)
+    if world > 1 and args.gpus != world:
+        log(f"error: --gpus {args.gpus} but WORLD_SIZE={world}")
+        return 2
     if args.impl == "reference":
         return run_reference(args, rank, world)
     return run_ours(args, rank, world, local)
