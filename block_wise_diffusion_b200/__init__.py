@@ -42,7 +42,7 @@ EXPORTS = (
     "tt_decode_blocks", "tt_loop_last_step",
 )
 KERNEL_KINDS = ("plan", "embed", "gemm_qkv", "attn", "merge", "adaln", "gemm_vocab", "commit",
-                "gather", "init", "splitk_reduce", "append")
+                "gather", "init", "splitk_reduce", "append", "attn_plan")
 
 
 class TTError(RuntimeError):

@@ -202,10 +202,12 @@ static tt_status check_ptr(const void* p, const char* name, bool need16) {
 
 // ------------------------------------------------------------ geometry
 struct AttnGeom {
-  int G, s_per_half, rows_per_half, halves, n_qtiles, n_splits, chunk, first;
+  int G, s_per_half, rows_per_half, halves, n_qtiles, units, n_ctas, slots;
   size_t part_o_bytes, part_ml_bytes;
 };
 
+// Query packing (S positions x G heads in 128-row halves) and the persistent
+// grid: one CTA per SM unless tt_set_attn_splits fixed the count.
 static AttnGeom attn_geom(const tt_dims& d) {
   AttnGeom g;
   g.G = d.Hq / d.Hkv;
@@ -213,31 +215,12 @@ static AttnGeom attn_geom(const tt_dims& d) {
   g.rows_per_half = g.s_per_half * g.G;
   g.halves = std::min(2, d.S / g.s_per_half);
   g.n_qtiles = d.S / (g.halves * g.s_per_half);
-  const long long units = (long long)d.B * d.Hkv * g.n_qtiles;
-  const int ctx_tiles = (d.L_cap + kAttnBN - 1) / kAttnBN;
+  g.units = d.B * d.Hkv * g.n_qtiles;
   const int forced = g_forced_splits.load();
-  const int sms = num_sms();
-  // one CTA per (unit, split): fill the SMs once
-  int n = forced > 0 ? forced : (int)std::max<long long>(1, sms / units);
-  n = std::min(std::min(n, ctx_tiles + 1), 64);
-  // Split 0 also runs the block's own key tile, so it gets one context tile
-  // fewer: every split then runs at most c tiles, c = ceil((tiles + 1) / n).
-  int c = (ctx_tiles + 1 + n - 1) / n;
-  if (forced <= 0 && units > sms) {
-    // More units than SMs: several waves whatever the split.  Context lengths
-    // differ per sequence (and live on the device), so cap a split at about
-    // an eighth of an SM's share of the largest possible work; the splits of
-    // short sequences that fall past their context exit at once.
-    const long long per_sm = units * (long long)(ctx_tiles + 1) / sms;
-    c = (int)std::min<long long>(c, std::max<long long>(8, (per_sm + 7) / 8));
-  }
-  g.chunk = c * kAttnBN;
-  g.first = (c - 1) * kAttnBN;
-  n = 1 + (std::max(0, d.L_cap - g.first) + g.chunk - 1) / g.chunk;
-  g.n_splits = n;
-  const size_t rows = (size_t)units * n * 256;
-  g.part_o_bytes = n > 1 ? rows * d.dh * sizeof(float) : 0;
-  g.part_ml_bytes = n > 1 ? rows * 2 * sizeof(float) : 0;
+  g.n_ctas = forced > 0 ? forced : num_sms();
+  g.slots = g.units + g.n_ctas - 1;
+  g.part_o_bytes = (size_t)g.slots * 256 * d.dh * sizeof(float);
+  g.part_ml_bytes = (size_t)g.slots * 256 * 2 * sizeof(float);
   return g;
 }
 
@@ -279,10 +262,11 @@ struct Ws {
   float* tvec = nullptr;
   uint16_t* egath = nullptr;
   uint16_t* qkv = nullptr;
-  uint16_t* attn_out = nullptr;
   uint16_t* y_c = nullptr;
   float* part_o = nullptr;
   float* part_ml = nullptr;
+  int* tile_start = nullptr;   // attention plan: tiles per unit, prefix sums
+  int* first_unit = nullptr;   // attention plan: first unit of each CTA
   float4* stats = nullptr;
   float* qkv_partial = nullptr;
   uint16_t* xrows = nullptr;  // loop: one layer's modulated rows for the next layer
@@ -305,10 +289,10 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
   }
   if (which == TT_WS_ATTN || which == TT_WS_LOOP) {
     const AttnGeom g = attn_geom(d);
-    if (g.n_splits > 1) {
-      w.part_o = c.take<float>(g.part_o_bytes);
-      w.part_ml = c.take<float>(g.part_ml_bytes);
-    }
+    w.tile_start = c.take<int>((size_t)(g.units + 1) * sizeof(int));
+    w.first_unit = c.take<int>((size_t)g.n_ctas * sizeof(int));
+    w.part_o = c.take<float>(g.part_o_bytes);
+    w.part_ml = c.take<float>(g.part_ml_bytes);
   }
   if (which == TT_WS_VOCAB || which == TT_WS_LOOP) {
     w.rowlist = c.take<int>(2 * rows * sizeof(int));
@@ -322,7 +306,6 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     w.egath = c.take<uint16_t>(rows * d.H * 2);
     w.xrows = c.take<uint16_t>(rows * d.H * 2);
     w.qkv = c.take<uint16_t>(rows * n_qkv * 2);
-    w.attn_out = c.take<uint16_t>(rows * d.H * 2);
     // tile-major partials: ks planes of whole 128 x kQkvBN tiles, for the
     // linear update or the context projection, whichever needs more
     const size_t pb = std::max(splitk_bytes(d, (int)n_qkv, qkv_ksplit(d)),
@@ -384,9 +367,10 @@ static AttnArgs attn_args(const tt_dims& d, const AttnGeom& g, const int32_t* ct
   a.rows_per_half = g.rows_per_half;
   a.halves = g.halves;
   a.n_qtiles = g.n_qtiles;
-  a.n_splits = g.n_splits;
-  a.chunk = g.chunk;
-  a.first = g.first;
+  a.units = g.units;
+  a.n_ctas = g.n_ctas;
+  a.tile_start = w.tile_start;
+  a.first_unit = w.first_unit;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.dh));
   a.out = out;
   a.ldo = d.H;
@@ -400,14 +384,24 @@ static AttnArgs attn_args(const tt_dims& d, const AttnGeom& g, const int32_t* ct
   return a;
 }
 
-// The attention launch; with `merge` the split partials are combined into
+// The attention's tile plan (prefix sums of tiles per unit from the device
+// context lengths, first unit of each CTA): once per call, since ctx_len does
+// not change within one.
+static tt_status run_attn_plan(const tt_dims& d, const AttnGeom& g, const int32_t* ctx_len,
+                               const Ws& w, cudaStream_t st) {
+  const AttnArgs a = attn_args(d, g, ctx_len, nullptr, w, nullptr);
+  TT_LAUNCH(TT_K_ATTN_PLAN, st, launch_attn_plan(a, st));
+  return TT_OK;
+}
+
+// The attention launch; with `merge` the segment partials are combined into
 // `out` by the merge kernel (the loop fuses that merge into adaLN instead).
 static tt_status run_attn(const tt_dims& d, const AttnGeom& g, const AttnMaps& m,
                           const int32_t* ctx_len, tt_bf16* out, const Ws& w, const int* active,
                           bool merge, cudaStream_t st) {
   const AttnArgs a = attn_args(d, g, ctx_len, out, w, active);
   TT_LAUNCH(TT_K_ATTN, st, launch_attn(m.q, m.kc, m.vc, m.kb, m.vb, a, st));
-  if (merge && g.n_splits > 1) TT_LAUNCH(TT_K_MERGE, st, launch_attn_merge(a, st));
+  if (merge) TT_LAUNCH(TT_K_MERGE, st, launch_attn_merge(a, st));
   return TT_OK;
 }
 
@@ -605,6 +599,7 @@ tt_status tt_block_denoise_attn(const tt_dims* d, const tt_bf16* q_blk, const tt
                            v_ctx, &m));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   TT_CUDA(cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st));
+  TT_CHECK(run_attn_plan(*d, g, ctx_len, w, st));
   return run_attn(*d, g, m, ctx_len, out, w, nullptr, true, st);
 }
 
@@ -621,8 +616,7 @@ tt_status tt_adaln_modulate(const tt_dims* d, const tt_bf16* x, const tt_bf16* s
   TT_CHECK(check_ws(*d, TT_WS_ADALN, ws, ws_bytes, &w));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   TT_CUDA(cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st));
-  TT_LAUNCH(TT_K_ADALN, st, launch_adaln(x, shift_scale, t, y, d->B * d->S, d->S, d->H, nullptr,
-                                         nullptr, nullptr, nullptr, st));
+  TT_LAUNCH(TT_K_ADALN, st, launch_adaln(x, shift_scale, t, y, d->B * d->S, d->S, d->H, st));
   return TT_OK;
 }
 
@@ -696,6 +690,7 @@ static tt_status denoise_block_loop_impl(
 
   TT_CUDA(cudaMemsetAsync(w.ctrl, 0, w.ctrl_clear, st));
   TT_LAUNCH(TT_K_INIT, st, launch_loop_init(d->B, d->S, steps_taken, commit_step, w.ctrl, st));
+  TT_CHECK(run_attn_plan(*d, g, ctx_len, w, st));
   // a step runs while masked positions remain (commit decrements the count)
   const int* active = w.ctrl + CTRL_REMAINING;
   GemmArgs ga{};
@@ -729,19 +724,14 @@ static tt_status denoise_block_loop_impl(
       if (ga.ksplit > 1)
         TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
                                                           w.qkv, n_qkv, active, st));
-      TT_CHECK(run_attn(*d, g, maps[l], ctx_len, w.attn_out, w, active, false, st));
+      TT_CHECK(run_attn(*d, g, maps[l], ctx_len, nullptr, w, active, false, st));
       // The last layer keeps the masked rows, compacted, for the vocabulary;
       // earlier layers modulate every row (all positions are keys of the
       // next layer).  A null row list selects the latter.
       uint16_t* y = last ? w.y_c : w.xrows;
       int* rl = last ? w.rowlist : nullptr;
-      if (g.n_splits > 1) {
-        const AttnArgs aa = attn_args(*d, g, ctx_len, w.attn_out, w, active);
-        TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, ss, y, masked, rl, w.ctrl, st));
-      } else {
-        TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, ss, nullptr, y, rows, d->S, d->H,
-                                               masked, rl, w.ctrl, active, st));
-      }
+      const AttnArgs aa = attn_args(*d, g, ctx_len, nullptr, w, active);
+      TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, ss, y, masked, rl, w.ctrl, st));
     }
     TT_CHECK(run_vocab_gemm(*d, w, W, logit_scale, w.ctrl + CTRL_M, active, w_keep_tiles, st));
     CommitArgs c = commit_args(*d, w, gamma, logit_scale, tokens, masked);

@@ -1,37 +1,42 @@
-// Block-denoise attention (one denoiser layer), split over context keys.
+// Block-denoise attention (one denoiser layer).
 //
 // "Architecture" / "Generation Process" of the gist.science summary: every
 // block query attends to the frozen context tower's K/V of the same layer and
-// to the block's own S keys, with no mask inside the block.  This kernel runs
-// one softmax over [context keys ; block keys] per query row.
+// to the block's own S keys, with no mask inside the block.  One softmax
+// runs over [block keys ; context keys] per query row (the order of keys does
+// not change a softmax).
 //
-// Work unit (one CTA): a KV head g of sequence b, a query tile of up to 256
-// rows (block positions x the G query heads sharing g, packed so one K/V
-// tile feeds every row) and a contiguous split of the context keys; split 0
-// also owns the block's own S keys.  The rows form two 128-row halves, each
-// an M=128 tcgen05 tile with its own TMEM columns.  Per 128-key tile i and
-// half h:
+// Work units and schedule.  A unit is a KV head g of sequence b and a query
+// tile of up to 256 rows (block positions x the G query heads sharing g,
+// packed so one K/V tile feeds every row).  Its keys form tiles of 128: tile
+// 0 holds the block's own S keys, tiles 1.. the context keys.  All units'
+// tiles are laid end to end (attn_plan_kernel writes the prefix sums from the
+// device-side context lengths) and cut into one contiguous range per CTA of a
+// persistent grid (one CTA per SM), so every SM streams the same number of
+// K/V tiles whatever the batch and the lengths.  A CTA walks its range as
+// segments, one per unit it touches, and writes per segment the unnormalised
+// O and the row maxima and sums; a merge combines a unit's segments.
+//
+// Inside a CTA the unit's rows form two 128-row halves, each an M=128
+// tcgen05 tile with its own TMEM columns.  Per 128-key tile i and half h:
 //   S_h  = Q_h . K(i)^T       (TMEM, 128 fp32 columns; Q and K from smem)
-//   P_h  = exp2(S_h*c - m)    (bf16 pairs, written back into S_h's columns)
+//   P_h  = exp2(S_h*c - m)    (bf16 pairs, written back over S_h's columns)
 //   O_h += P_h . V(i)         (TMEM accumulator; A = P_h read from TMEM)
-// so P never goes through shared memory.  Roles (20 warps):
+// so P never goes through shared memory.  Roles (12 warps):
 //   warp 0     TMA for Q and K (3-slot ring);
-//   warps 1, 2 MMA issue for half 0 / half 1: P_h(i).V(i) as soon as
-//              softmax h has written P_h(i), then S_h(i+1) into the same
-//              columns (tcgen05 MMAs of one thread execute in issue order);
-//   warp 3     TMEM owner; TMA for V (2-slot ring) and zeroing of the V rows
+//   warp 1     TMEM owner; TMA for V (2-slot ring) and zeroing of the V rows
 //              past the last valid key that a 16-key MMA step still reads;
-//   warps 4-11 / 12-19  softmax of half 0 / half 1.  Warp w serves the 32
-//              rows of its TMEM lane quarter (w % 4) and one 64-key column
-//              half of every tile; the two warps of a row swap partial row
-//              maxima through shared memory.  Thread = row: no shuffles.
+//   warps 2, 3 MMA issue for half 0 / half 1: P_h(i).V(i) once softmax h has
+//              written P_h(i), then S_h(i+1) into the same columns (tcgen05
+//              MMAs of one thread execute in issue order);
+//   warps 4-7 / 8-11  softmax of half 0 / half 1: thread = query row (TMEM
+//              lane), the whole 128-key row of S in registers, so the row
+//              maximum needs no exchange and S is read from TMEM once.
 // The two softmax groups take turns tile by tile, so the tensor core runs
-// one half's MMAs during the other half's softmax.  An eighth of the
+// one half's MMAs during the other half's softmax.  Part of the
 // exponentials run on the FMA pipe (exp2_poly) to offload the MUFU unit.
 // The running max only moves (and O is rescaled in TMEM) when it grows by
-// more than 2^8; the final O / l is exact for any stale max.  With one split
-// the CTA writes the bf16 output; otherwise (unnormalised O, max, sum)
-// partials for a merge kernel.
+// more than 2^8; the final O / l is exact for any stale max.
 #include <math.h>
 
 #include "tt_ptx.cuh"
@@ -49,9 +54,16 @@ constexpr int kKSlots = 3, kVSlots = 2;       // K and V ring depths
 constexpr uint32_t kKVSub = kAttnBN * 128;    // 128 keys x 64 dh bf16 (128-byte rows) = 16 KB
 constexpr uint32_t kQSub = 16384;             // 128 rows x 64 dh bf16
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
+// Of every 16 exponential pairs of a 32-key chunk, this many run on the FMA
+// pipe (exp2_poly), the rest on MUFU.
+#ifndef TT_ATTN_POLY_PAIRS
+#define TT_ATTN_POLY_PAIRS 3
+#endif
+constexpr int kPolyPairs = TT_ATTN_POLY_PAIRS;
+constexpr int kPolyStride = kPolyPairs > 0 ? 16 / kPolyPairs : 17;  // pairs j = stride-1, 2*stride-1, ...
 
 struct AttnSmem {
-  uint32_t q, k, v, bars, xchg, total;
+  uint32_t q, k, v, bars, total;
 };
 
 __host__ __device__ inline AttnSmem attn_layout(int dh, int halves) {
@@ -61,8 +73,7 @@ __host__ __device__ inline AttnSmem attn_layout(int dh, int halves) {
   L.k = L.q + (uint32_t)halves * nsub * kQSub;
   L.v = L.k + kKSlots * nsub * kKVSub;
   L.bars = L.v + kVSlots * nsub * kKVSub;
-  L.xchg = L.bars + 256;      // row-max exchange: [half][quarter][column half][lane] bf16
-  L.total = L.xchg + 1024;
+  L.total = L.bars + 256;
   return L;
 }
 
@@ -70,22 +81,60 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// A unit's context length, clamped to [0, L_cap] (an out-of-range length is
+// reported by the plan kernel).
+__device__ __forceinline__ int unit_len(const AttnArgs& a, int b) {
+  return min(max(a.ctx_len[b], 0), a.L_cap);
+}
+
+struct UnitInfo {
+  int b, g, qt, L;
+};
+__device__ __forceinline__ UnitInfo unit_info(const AttnArgs& a, int u) {
+  UnitInfo ui;
+  const int pair = u / a.n_qtiles;
+  ui.qt = u - pair * a.n_qtiles;
+  ui.b = pair / a.Hkv;
+  ui.g = pair - ui.b * a.Hkv;
+  ui.L = unit_len(a, ui.b);
+  return ui;
+}
+
 struct TileInfo {
   int is_blk, key0, nvalid;
 };
-__device__ __forceinline__ TileInfo tile_info(int t, int has_blk, int k0, int k1, int S) {
+// Local tile tl of a unit: 0 is the block's own S keys, tl >= 1 the context
+// keys (tl-1)*128 .. min(tl*128, L) - 1.
+__device__ __forceinline__ TileInfo tile_info(int tl, int L, int S) {
   TileInfo ti;
-  if (has_blk && t == 0) {
+  if (tl == 0) {
     ti.is_blk = 1;
     ti.key0 = 0;
     ti.nvalid = S;
   } else {
     ti.is_blk = 0;
-    ti.key0 = k0 + (t - has_blk) * kAttnBN;
-    ti.nvalid = min(kAttnBN, k1 - ti.key0);
+    ti.key0 = (tl - 1) * kAttnBN;
+    ti.nvalid = min(kAttnBN, L - ti.key0);
   }
   return ti;
 }
+
+// The CTA's range [lo, hi) of the tile sequence and its segments, walked the
+// same way by every role: segment = (unit u, local tiles [a, b)).
+struct SegWalk {
+  const int* start;
+  int t, hi, u;
+  __device__ __forceinline__ bool next(int& unit, int& a, int& b) {
+    if (t >= hi) return false;
+    const int s0 = start[u], s1 = start[u + 1];
+    unit = u;
+    a = t - s0;
+    b = min(hi, s1) - s0;
+    t = min(hi, s1);
+    ++u;
+    return true;
+  }
+};
 
 // 2^x on the FMA pipe, to take part of the exponentials off the MUFU unit
 // (Cody-Waite style range reduction): n = round(x) by the float trick of
@@ -107,32 +156,17 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return x > -126.0f ? r : 0.f;
 }
 
-// TMEM load of 16 columns (32x32b shape: a thread's lane, consecutive columns).
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-// TMEM store of 8 columns, same shape.
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
-               "r"(r[7])
-               : "memory");
-}
-// P for 16 score columns as 8 bf16 pairs; the last pair on the FMA pipe.
-__device__ __forceinline__ void exp_slice16(const uint32_t (&sv)[16], float c, float m, float& s0,
-                                            float& s1, uint32_t (&pk)[8]) {
+// P for a 32-key chunk of S (registers) as 16 bf16 pairs, written in place:
+// pair j goes to sv[2j] (the registers of S it came from are dead by then);
+// kPolyPairs of the pairs on the FMA pipe.
+__device__ __forceinline__ void exp_chunk32(uint32_t (&sv)[32], float c, float m, float& s0,
+                                            float& s1) {
 #pragma unroll
-  for (int j = 0; j < 16; j += 2) {
-    const float x0 = fmaf(__uint_as_float(sv[j]), c, -m);
-    const float x1 = fmaf(__uint_as_float(sv[j + 1]), c, -m);
+  for (int j = 0; j < 16; ++j) {
+    const float x0 = fmaf(__uint_as_float(sv[2 * j]), c, -m);
+    const float x1 = fmaf(__uint_as_float(sv[2 * j + 1]), c, -m);
     float p0, p1;
-    if (j == 14) {
+    if (j % kPolyStride == kPolyStride - 1) {
       p0 = exp2_poly(x0);
       p1 = exp2_poly(x1);
     } else {
@@ -141,7 +175,99 @@ __device__ __forceinline__ void exp_slice16(const uint32_t (&sv)[16], float c, f
     }
     s0 += p0;
     s1 += p1;
-    pk[j >> 1] = pack_bf16x2(p0, p1);
+    sv[2 * j] = pack_bf16x2(p0, p1);
+  }
+}
+
+// TMEM store of 16 columns from the even registers of a 32-register chunk
+// (32x32b shape: a thread's lane, consecutive columns).
+__device__ __forceinline__ void tmem_st16_even(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[2]), "r"(r[4]), "r"(r[6]), "r"(r[8]), "r"(r[10]), "r"(r[12]), "r"(r[14]),
+      "r"(r[16]), "r"(r[18]), "r"(r[20]), "r"(r[22]), "r"(r[24]), "r"(r[26]), "r"(r[28]),
+      "r"(r[30])
+      : "memory");
+}
+
+// TMEM load of 16 columns (32x32b shape: a thread's lane, consecutive columns).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ float max32(const uint32_t (&v)[32], float m) {
+  float a = m, b = -INFINITY, cc = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 30; j += 6) {
+    a = fmax3(a, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
+    b = fmax3(b, __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+    cc = fmax3(cc, __uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+  }
+  a = fmax3(a, __uint_as_float(v[30]), __uint_as_float(v[31]));
+  return fmax3(a, b, cc);
+}
+
+__device__ __forceinline__ void mask32(uint32_t (&v)[32], int base, int nv) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = base + j < nv ? v[j] : __float_as_uint(-INFINITY);
+}
+
+// Tiles per unit and their exclusive prefix sums (one CTA), then the first
+// unit of every CTA of the attention's persistent grid.
+__global__ void __launch_bounds__(1024) attn_plan_kernel(const AttnArgs a) {
+  griddep_launch();
+  griddep_wait();
+  __shared__ int warp_tot[32];
+  __shared__ int running;
+  int* start = a.tile_start;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  if (tid == 0) running = 0;
+  __syncthreads();
+  for (int base = 0; base < a.units; base += blockDim.x) {
+    const int u = base + tid;
+    int n = 0;
+    if (u < a.units) {
+      const int b = u / (a.Hkv * a.n_qtiles);
+      const int L = a.ctx_len[b];
+      if ((L < 0 || L > a.L_cap) && (u % (a.Hkv * a.n_qtiles)) == 0)
+        atomicCAS(a.err, 0, (int)TT_ERR_INVALID_ARG);
+      n = 1 + (min(max(L, 0), a.L_cap) + kAttnBN - 1) / kAttnBN;
+    }
+    int incl = n;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < nw; ++w) {
+      before += w < warp ? warp_tot[w] : 0;
+      total += warp_tot[w];
+    }
+    if (u < a.units) start[u] = running + before + incl - n;
+    __syncthreads();
+    if (tid == 0) running += total;
+    __syncthreads();
+  }
+  if (tid == 0) start[a.units] = running;
+  __syncthreads();
+  // CTA c's range starts at lo(c) = c*T/P; the unit holding lo(c) is its
+  // first.  Unit u holds [s0, s1), i.e. the CTAs ceil(s0*P/T) ..
+  // ceil(s1*P/T) - 1.
+  const long long T = running, P = a.n_ctas;
+  for (int u = tid; u < a.units; u += blockDim.x) {
+    const long long s0 = start[u], s1 = start[u + 1];
+    const long long c0 = (s0 * P + T - 1) / T, c1 = (s1 * P + T - 1) / T;
+    for (long long c = c0; c < c1 && c < P; ++c) a.first_unit[c] = u;
   }
 }
 
@@ -153,29 +279,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   griddep_wait();
   extern __shared__ uint8_t smem_raw[];
   if (a.active != nullptr && *a.active == 0) return;
-  const int split = blockIdx.x, qt = blockIdx.y, pair = blockIdx.z;
-  const int b = pair / a.Hkv, g = pair % a.Hkv;
-  int L = a.ctx_len[b];
-  if (L < 0 || L > a.L_cap) {
-    if (threadIdx.x == 0) atomicCAS(a.err, 0, (int)TT_ERR_INVALID_ARG);
-    L = min(max(L, 0), a.L_cap);
-  }
-  const int k0 = split == 0 ? 0 : a.first + (split - 1) * a.chunk;
-  const int k1 = min(split == 0 ? a.first : k0 + a.chunk, L);
-  const int n_ctx_tiles = k1 > k0 ? (k1 - k0 + kAttnBN - 1) / kAttnBN : 0;
-  const int has_blk = split == 0 ? 1 : 0;
-  const int n_tiles = has_blk + n_ctx_tiles;
-  const int unit = (pair * a.n_qtiles + qt) * a.n_splits + split;
+  const int cta = blockIdx.x;
+  const long long T = a.tile_start[a.units];
+  const int lo = (int)((long long)cta * T / a.n_ctas);
+  const int hi = (int)((long long)(cta + 1) * T / a.n_ctas);
+  if (lo >= hi) return;
+  const int u0 = a.first_unit[cta];
   const int dh = a.dh, nsub = dh / 64;
   const int halves = a.halves;
-
-  if (n_tiles == 0) {  // an empty split (only split > 0): contributes nothing
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
-      a.part_ml[((size_t)unit * 256 + i) * 2 + 0] = -INFINITY;
-      a.part_ml[((size_t)unit * 256 + i) * 2 + 1] = 0.f;
-    }
-    return;
-  }
 
   const AttnSmem SL = attn_layout(dh, halves);
   uint8_t* base = align1024(smem_raw);
@@ -184,16 +295,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint8_t* sV = base + SL.v;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + SL.bars);
   uint64_t* q_full = bars;
-  uint64_t* k_full = q_full + 1;         // [kKSlots]
+  uint64_t* q_empty = q_full + 1;        // one arrival per half: its last S of the segment done
+  uint64_t* k_full = q_empty + 1;        // [kKSlots]
   uint64_t* k_empty = k_full + kKSlots;  // [kKSlots], one arrival per half
   uint64_t* v_full = k_empty + kKSlots;  // [kVSlots]
   uint64_t* v_empty = v_full + kVSlots;  // [kVSlots], one arrival per half
   uint64_t* v_ready = v_empty + kVSlots; // [kVSlots]: V landed and its padding rows cleared
   uint64_t* s_full = v_ready + kVSlots;  // [half]: S_h(i) ready (and P_h(i-1).V done)
   uint64_t* p_full = s_full + 2;         // [half]: P_h(i) written, O_h corrected
-  uint64_t* o_full = p_full + 2;         // [half]
-  uint64_t* xbar = o_full + 2;           // [half][quarter]: both column halves' row maxima written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 8);
+  uint64_t* o_full = p_full + 2;         // [half]: the segment's last P.V done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -203,7 +314,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const uint32_t tO0 = halves * kAttnBN;
 
   // Rows of a half that the Q box does not cover must be finite (they only
-  // produce output rows that are discarded): clear Q when the box is short.
+  // produce output rows that are discarded): clear Q once when the box is
+  // short; the boxes of later segments rewrite only the covered rows.
   if (a.rows_per_half < 128) {
     uint4* q4 = reinterpret_cast<uint4*>(sQ);
     const int n4 = halves * nsub * (int)kQSub / 16;
@@ -212,6 +324,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, halves);
     for (int s = 0; s < kKSlots; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], halves);
@@ -223,14 +336,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&s_full[h], 1);
-      mbar_init(&p_full[h], 256);
+      mbar_init(&p_full[h], 128);
       mbar_init(&o_full[h], 1);
     }
-    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 3) {
+  if (warp == 1) {
     tmem_alloc(tmem_slot, tmem_cols);
     tmem_relinquish();
   }
@@ -238,384 +350,353 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int pos0 = qt * halves * a.s_per_half;  // first block position of this query tile
+  SegWalk walk{a.tile_start, lo, hi, u0};
+  int su, sa, sb;  // current segment: unit, local tiles [sa, sb)
 
-  if (warp < 4) {
-    if (warp == 0) {
-      // ------------------------------------------------ TMA producer: Q, K
-      if (lane == 0) {
-        prefetch_tmap(&tmQ);
-        prefetch_tmap(&tmKc);
-        const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer: Q, K
+    if (lane == 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmKc);
+      prefetch_tmap(&tmKb);
+      const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
+      int kt = 0, qi = 0;
+      bool ok = true;
+      while (ok && walk.next(su, sa, sb)) {
+        const UnitInfo ui = unit_info(a, su);
+        // Q of this segment's unit, once both halves' last S of the
+        // previous segment has read the buffer
+        if (qi > 0 && !mbar_wait(q_empty, (uint32_t)(qi - 1) & 1u, a.err, abort_flag,
+                                 WHERE_ATTN_PRODUCER))
+          break;
+        const int pos0 = ui.qt * halves * a.s_per_half;
         mbar_arrive_expect_tx(q_full, (uint32_t)(halves * nsub * a.rows_per_half * 128));
         for (int h = 0; h < halves; ++h)
           for (int xh = 0; xh < nsub; ++xh)
-            tma_load_3d(sQ + (h * nsub + xh) * kQSub, &tmQ, q_full, xh * 64, g * a.G,
-                        b * a.S + pos0 + h * a.s_per_half);
-        const int row_base = (b * a.Hkv + g) * a.L_cap;
-        for (int t = 0; t < n_tiles; ++t) {
-          const TileInfo ti = tile_info(t, has_blk, k0, k1, a.S);
+            tma_load_3d(sQ + (h * nsub + xh) * kQSub, &tmQ, q_full, xh * 64, ui.g * a.G,
+                        ui.b * a.S + pos0 + h * a.s_per_half);
+        ++qi;
+        const int row_base = (ui.b * a.Hkv + ui.g) * a.L_cap;
+        for (int tl = sa; tl < sb; ++tl, ++kt) {
+          const TileInfo ti = tile_info(tl, ui.L, a.S);
           const uint32_t bytes = ti.is_blk ? (uint32_t)(nsub * a.S * 128) : (uint32_t)(nsub * kKVSub);
-          const int ks = t % kKSlots;
-          if (!mbar_wait(&k_empty[ks], ((uint32_t)(t / kKSlots) & 1u) ^ 1u, a.err, abort_flag,
-                         WHERE_ATTN_PRODUCER))
+          const int ks = kt % kKSlots;
+          if (!mbar_wait(&k_empty[ks], ((uint32_t)(kt / kKSlots) & 1u) ^ 1u, a.err, abort_flag,
+                         WHERE_ATTN_PRODUCER)) {
+            ok = false;
             break;
-          TT_TRACE_POINT(true, 0, t);
+          }
           uint8_t* dk = sK + ks * nsub * kKVSub;
           mbar_arrive_expect_tx(&k_full[ks], bytes);
           for (int xh = 0; xh < nsub; ++xh) {
             if (ti.is_blk)
-              tma_load_3d(dk + xh * kKVSub, &tmKb, &k_full[ks], xh * 64, g, b * a.S);
+              tma_load_3d(dk + xh * kKVSub, &tmKb, &k_full[ks], xh * 64, ui.g, ui.b * a.S);
             else
-              tma_load_2d_hint(dk + xh * kKVSub, &tmKc, &k_full[ks], xh * 64, row_base + ti.key0,
-                               pol_kv);
+              tma_load_2d_hint(dk + xh * kKVSub, &tmKc, &k_full[ks], xh * 64,
+                               row_base + ti.key0, pol_kv);
           }
         }
       }
-    } else if (warp == 1 || warp == 2) {
-      // ------------------------------------------- MMA issuer of half (warp-1)
-      const int h = warp - 1;
-      if (h < halves) {
-        const uint32_t idS = idesc_bf16(128, kAttnBN, false, false);
-        const uint32_t idO = idesc_bf16(128, dh, false, true);
-        const uint32_t tS = tmem + h * kAttnBN, tOh = tmem + tO0 + h * dh;
-        // Descriptor bases; each MMA adds a compile-time offset (the start
-        // address field is address >> 4 in the low bits, and no smem address
-        // carries out of it), so an issue costs a few instructions: the
-        // issuing warp shares its SMSP with busy softmax warps.
-        const uint64_t dQ = sdesc_sw128(smem_u32(sQ) + h * nsub * kQSub, 16, 1024);
-        const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
-        const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kKVSub, 1024);
-        // S_h(t) = Q_h . K(t)^T
-        auto scores = [&](int t) -> bool {
-          const int ks = t % kKSlots;
-          if (!mbar_wait(&k_full[ks], (uint32_t)(t / kKSlots) & 1u, a.err, abort_flag,
-                         WHERE_ATTN_MMA))
-            return false;
-          if (h == 0) TT_TRACE_POINT(lane == 0, 1, t);
-          tc_fence_after();
-          if (lane == 0) {
-            const uint64_t dK = dK0 + (uint64_t)((uint32_t)(ks * nsub) * (kKVSub >> 4));
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              if (kk < dh / 16)
-                umma_bf16_ss(tS, dQ + (uint64_t)(((kk >> 2) * kQSub + (kk & 3) * 32) >> 4),
-                             dK + (uint64_t)(((kk >> 2) * kKVSub + (kk & 3) * 32) >> 4), idS,
-                             kk > 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------- TMA producer: V; V padding
+    // Lane 0 streams V (own loop, so K never waits for a V slot).  The P.V
+    // MMA reads V rows up to the next multiple of 16 past the valid keys;
+    // those rows hold whatever the cache holds beyond the context (or an
+    // older tile's rows), and P is zero there but 0 * NaN is NaN, so the
+    // warp zeroes them before either half's MMA may read the slot.  V(t) is
+    // issued before V(t-1) is cleaned, keeping two loads in flight.
+    if (lane == 0) {
+      prefetch_tmap(&tmVc);
+      prefetch_tmap(&tmVb);
+    }
+    const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
+    int vt = 0, prev_nv = -1;
+    bool ok = true;
+    auto clean = [&](int t, int nvalid) -> bool {
+      const int vs = t % kVSlots;
+      const bool landed = mbar_wait(&v_full[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
+                                    WHERE_ATTN_MMA);
+      if (!__all_sync(0xffffffffu, landed)) return false;
+      const int pad = ((nvalid + 15) & ~15) - nvalid;
+      if (pad > 0) {
+        for (int xh = 0; xh < nsub; ++xh) {
+          uint4* dst = reinterpret_cast<uint4*>(sV + (vs * nsub + xh) * kKVSub + nvalid * 128);
+          for (int i = lane; i < pad * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&v_ready[vs]);
+      return true;
+    };
+    while (ok && walk.next(su, sa, sb)) {
+      const UnitInfo ui = unit_info(a, su);
+      const int row_base = (ui.b * a.Hkv + ui.g) * a.L_cap;
+      for (int tl = sa; tl < sb; ++tl, ++vt) {
+        const TileInfo ti = tile_info(tl, ui.L, a.S);
+        int good = 1;
+        if (lane == 0) {
+          const uint32_t bytes =
+              ti.is_blk ? (uint32_t)(nsub * a.S * 128) : (uint32_t)(nsub * kKVSub);
+          const int vs = vt % kVSlots;
+          good = mbar_wait(&v_empty[vs], ((uint32_t)(vt / kVSlots) & 1u) ^ 1u, a.err, abort_flag,
+                           WHERE_ATTN_PRODUCER);
+          if (good) {
+            uint8_t* dv = sV + vs * nsub * kKVSub;
+            mbar_arrive_expect_tx(&v_full[vs], bytes);
+            for (int xh = 0; xh < nsub; ++xh) {
+              if (ti.is_blk)
+                tma_load_3d(dv + xh * kKVSub, &tmVb, &v_full[vs], xh * 64, ui.g, ui.b * a.S);
+              else
+                tma_load_2d_hint(dv + xh * kKVSub, &tmVc, &v_full[vs], xh * 64,
+                                 row_base + ti.key0, pol_kv);
             }
-            umma_commit(&s_full[h]);
-            umma_commit(&k_empty[ks]);
           }
-          __syncwarp();
-          if (h == 0) TT_TRACE_POINT(lane == 0, 2, t);
-          return true;
-        };
-        // O_h += P_h(t) . V(t), once warp 3 has cleared V(t)'s padding rows
-        auto pv = [&](int t) -> bool {
-          if (!mbar_wait(&p_full[h], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_MMA))
-            return false;
-          TT_TRACE_POINT(lane == 0, 3 + h, t);
-          const int vs = t % kVSlots;
-          const int ksteps = (tile_info(t, has_blk, k0, k1, a.S).nvalid + 15) >> 4;
-          if (!mbar_wait(&v_ready[vs], (uint32_t)(t / kVSlots) & 1u, a.err, abort_flag,
-                         WHERE_ATTN_MMA))
-            return false;
+        }
+        if (__shfl_sync(0xffffffffu, good, 0) == 0 || (vt > 0 && !clean(vt - 1, prev_nv))) {
+          ok = false;
+          break;
+        }
+        prev_nv = ti.nvalid;
+      }
+    }
+    if (ok && vt > 0) clean(vt - 1, prev_nv);
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------- MMA issuer of half (warp-2)
+    const int h = warp - 2;
+    if (h < halves) {
+      const uint32_t idS = idesc_bf16(128, kAttnBN, false, false);
+      const uint32_t idO = idesc_bf16(128, dh, false, true);
+      const uint32_t tS = tmem + h * kAttnBN, tOh = tmem + tO0 + h * dh;
+      // Descriptor bases; each MMA adds a compile-time offset (the start
+      // address field is address >> 4 in the low bits, and no smem address
+      // carries out of it), so an issue costs a few instructions.
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ) + h * nsub * kQSub, 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kKVSub, 1024);
+      // S_h = Q_h . K(kt)^T
+      auto scores = [&](int kt) -> bool {
+        const int ks = kt % kKSlots;
+        if (!mbar_wait(&k_full[ks], (uint32_t)(kt / kKSlots) & 1u, a.err, abort_flag,
+                       WHERE_ATTN_MMA))
+          return false;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t dK = dK0 + (uint64_t)((uint32_t)(ks * nsub) * (kKVSub >> 4));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            if (kk < dh / 16)
+              umma_bf16_ss(tS, dQ + (uint64_t)(((kk >> 2) * kQSub + (kk & 3) * 32) >> 4),
+                           dK + (uint64_t)(((kk >> 2) * kKVSub + (kk & 3) * 32) >> 4), idS,
+                           kk > 0);
+          }
+          umma_commit(&s_full[h]);
+          umma_commit(&k_empty[ks]);
+        }
+        __syncwarp();
+        return true;
+      };
+      int kt = 0, pt = 0, qi = 0;
+      bool ok = true;
+      while (ok && walk.next(su, sa, sb)) {
+        const UnitInfo ui = unit_info(a, su);
+        const int n = sb - sa;
+        ok = mbar_wait(q_full, (uint32_t)qi & 1u, a.err, abort_flag, WHERE_ATTN_MMA);
+        if (ok) tc_fence_after();
+        if (ok) ok = scores(kt);
+        if (ok && n == 1 && lane == 0) umma_commit(q_empty);
+        for (int i = 0; ok && i < n; ++i, ++pt) {
+          // O_h += P_h(i) . V(i), once warp 1 has cleared V(i)'s padding rows
+          if (!mbar_wait(&p_full[h], (uint32_t)pt & 1u, a.err, abort_flag, WHERE_ATTN_MMA) ||
+              !mbar_wait(&v_ready[(kt + i) % kVSlots], (uint32_t)((kt + i) / kVSlots) & 1u, a.err,
+                         abort_flag, WHERE_ATTN_MMA)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
+          const int ksteps = (tile_info(sa + i, ui.L, a.S).nvalid + 15) >> 4;
           if (lane == 0) {
             // V as an MN-major operand: 64-wide dh blocks kKVSub apart, 8-key
-            // groups 1 KB apart, 16 keys (2 KB) per MMA.  P of keys 0..63
-            // sits in columns 0..31, of keys 64..127 in columns 64..95.
+            // groups 1 KB apart, 16 keys (2 KB) per MMA; P of keys
+            // 16kk..16kk+15 in columns 8kk..8kk+7.
+            const int vs = (kt + i) % kVSlots;
             const uint64_t dV = dV0 + (uint64_t)((uint32_t)(vs * nsub) * (kKVSub >> 4));
 #pragma unroll
             for (int kk = 0; kk < kAttnBN / 16; ++kk) {
               if (kk < ksteps)
-                umma_bf16_ts(tOh, tS + kk * 8 + (kk >= 4 ? 32 : 0), dV + (uint64_t)(kk * (2048 >> 4)),
-                             idO, (t > 0 || kk > 0) ? 1u : 0u);
+                umma_bf16_ts(tOh, tS + kk * 8, dV + (uint64_t)(kk * (2048 >> 4)), idO,
+                             (i > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&v_empty[vs]);
           }
           __syncwarp();
-          return true;
-        };
-        bool ok = mbar_wait(q_full, 0, a.err, abort_flag, WHERE_ATTN_MMA);
-        if (ok) tc_fence_after();
-        if (ok) ok = scores(0);
-        for (int t = 0; ok && t < n_tiles; ++t) {
-          ok = pv(t);
-          if (ok && t + 1 < n_tiles) ok = scores(t + 1);
+          if (i + 1 < n) {
+            ok = scores(kt + i + 1);
+            if (ok && i + 2 == n && lane == 0) umma_commit(q_empty);
+          }
         }
-        if (lane == 0) umma_commit(&o_full[h]);
+        if (ok && lane == 0) umma_commit(&o_full[h]);
         __syncwarp();
-      }
-    } else {
-      // ------------------------------------------- TMA producer: V; V padding
-      // Lane 0 streams V (own loop, so K never waits for a V slot).  The
-      // P.V MMA reads V rows up to the next multiple of 16 past the valid
-      // keys; those rows hold whatever the cache holds beyond the context (or
-      // an older tile's rows), and P is zero there but 0 * NaN is NaN, so the
-      // warp zeroes them before either half's MMA may read the slot.  V(t) is
-      // issued before V(t-1) is cleaned, keeping two loads in flight.
-      if (lane == 0) prefetch_tmap(&tmVc);
-      const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
-      const int row_base = (b * a.Hkv + g) * a.L_cap;
-      for (int t = 0; t <= n_tiles; ++t) {
-        if (t < n_tiles) {
-          int good = 1;
-          if (lane == 0) {
-            const TileInfo ti = tile_info(t, has_blk, k0, k1, a.S);
-            const uint32_t bytes =
-                ti.is_blk ? (uint32_t)(nsub * a.S * 128) : (uint32_t)(nsub * kKVSub);
-            const int vs = t % kVSlots;
-            good = mbar_wait(&v_empty[vs], ((uint32_t)(t / kVSlots) & 1u) ^ 1u, a.err,
-                             abort_flag, WHERE_ATTN_PRODUCER);
-            if (good) {
-              uint8_t* dv = sV + vs * nsub * kKVSub;
-              mbar_arrive_expect_tx(&v_full[vs], bytes);
-              for (int xh = 0; xh < nsub; ++xh) {
-                if (ti.is_blk)
-                  tma_load_3d(dv + xh * kKVSub, &tmVb, &v_full[vs], xh * 64, g, b * a.S);
-                else
-                  tma_load_2d_hint(dv + xh * kKVSub, &tmVc, &v_full[vs], xh * 64,
-                                   row_base + ti.key0, pol_kv);
-              }
-            }
-          }
-          if (__shfl_sync(0xffffffffu, good, 0) == 0) break;
-        }
-        if (t >= 1) {
-          const int tc = t - 1, vs = tc % kVSlots;
-          const bool landed = mbar_wait(&v_full[vs], (uint32_t)(tc / kVSlots) & 1u, a.err,
-                                        abort_flag, WHERE_ATTN_MMA);
-          if (!__all_sync(0xffffffffu, landed)) break;
-          const int nvalid = tile_info(tc, has_blk, k0, k1, a.S).nvalid;
-          const int pad = ((nvalid + 15) & ~15) - nvalid;
-          if (pad > 0) {
-            for (int xh = 0; xh < nsub; ++xh) {
-              uint4* dst = reinterpret_cast<uint4*>(sV + (vs * nsub + xh) * kKVSub + nvalid * 128);
-              for (int i = lane; i < pad * 8; i += 32) dst[i] = make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&v_ready[vs]);
-        }
+        kt += n;
+        ++qi;
       }
     }
   } else {
     // ---------------------------------------------------- softmax groups
-    // Half wg is served by warps 4+8*wg .. 11+8*wg.  Warp w owns the rows of
-    // its TMEM lane quarter q = w % 4 and one column half ch of every tile
-    // (S columns ch*64..+63, the O columns ch*dh/2..+dh/2-1), so two warps
-    // per SMSP share a row: they swap their partial row maxima through
-    // shared memory (as bf16, rounded the same way on both sides, so both
-    // use the identical stabiliser) and add their row sums at the end.
-    const int wg = (warp - 4) >> 3;
-    const int ch = ((warp - 4) >> 2) & 1;
+    // Half wg is served by warps 4+4*wg .. 7+4*wg; warp w owns the rows of
+    // its TMEM lane quarter q = w % 4, one row per thread, all 128 key
+    // columns of every tile.
+    const int wg = (warp - 4) >> 2;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     if (wg < halves) {
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-      const uint32_t tS = tmem + wg * kAttnBN + lane_off + ch * 64;
-      const int dh2 = dh / 2;
-      const uint32_t tO = tmem + tO0 + wg * dh + lane_off + ch * dh2;
-      uint16_t* xch = reinterpret_cast<uint16_t*>(base + SL.xchg) + (wg * 4 + q) * 64;
-      uint64_t* xb = &xbar[wg * 4 + q];
+      const uint32_t tS = tmem + wg * kAttnBN + lane_off;
+      const uint32_t tO = tmem + tO0 + wg * dh + lane_off;
       const float c = a.scale_log2;
-      float m = -INFINITY, l = 0.f;
+      int pt = 0, qi = 0;
       bool ok = true;
-      for (int t = 0; t < n_tiles; ++t) {
-        // The two halves take turns (0 on tile t, then 1 on tile t, then 0
-        // on t+1): the tensor core runs one half's P.V and next S while the
-        // other half's softmax runs, instead of both halves contending for
-        // MUFU and then both waiting for their MMAs.  p_full[other] marks
-        // the other half's tile done.
-        if (halves == 2 && (wg == 1 || t > 0) &&
-            !mbar_wait(&p_full[wg ^ 1], (uint32_t)(wg == 1 ? t : t - 1) & 1u, a.err, abort_flag,
-                       WHERE_ATTN_SOFTMAX)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(&s_full[wg], (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
-          ok = false;
-          break;
-        }
-        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 5 + 5 * wg, t);
-        tc_fence_after();
-        // Columns past the valid keys (the block's own tile, or the last
-        // tile of a split) are overwritten with -inf: nothing to the max,
-        // exp2 gives 0 on both exponential paths.
-        const int nv = tile_info(t, has_blk, k0, k1, a.S).nvalid - ch * 64;
-        if (nv < 64) {
-          for (int c0 = max(nv, 0) & ~31; c0 < 64; c0 += 32) {
-            uint32_t v[32];
-            if (c0 < nv) {
-              tmem_ld32(tS + c0, v);
+      while (ok && walk.next(su, sa, sb)) {
+        const UnitInfo ui = unit_info(a, su);
+        float m = -INFINITY, l = 0.f;
+        for (int i = sa; i < sb; ++i, ++pt) {
+          // The two halves take turns (0 on tile t, then 1 on tile t, then 0
+          // on t+1): the tensor core runs one half's P.V and next S while
+          // the other half's softmax runs.  p_full[other] marks the other
+          // half's turn done.
+          if (halves == 2 && (wg == 1 || pt > 0) &&
+              !mbar_wait(&p_full[wg ^ 1], (uint32_t)(wg == 1 ? pt : pt - 1) & 1u, a.err,
+                         abort_flag, WHERE_ATTN_SOFTMAX)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(&s_full[wg], (uint32_t)pt & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nv = tile_info(i, ui.L, a.S).nvalid;
+          // The row of S: up to four 32-key chunks (only those holding valid
+          // keys), one TMEM read.  Keys past nv become -inf.
+          uint32_t s0[32], s1[32], s2[32], s3[32];
+          tmem_ld32(tS, s0);
+          if (nv > 32) tmem_ld32(tS + 32, s1);
+          if (nv > 64) tmem_ld32(tS + 64, s2);
+          if (nv > 96) tmem_ld32(tS + 96, s3);
+          tmem_wait_ld();
+          float mt;
+          if (nv >= kAttnBN) {
+            mt = fmaxf(max32(s0, -INFINITY), max32(s1, -INFINITY));
+            mt = fmaxf(mt, fmaxf(max32(s2, -INFINITY), max32(s3, -INFINITY)));
+          } else {
+            mask32(s0, 0, nv);
+            mt = max32(s0, -INFINITY);
+            if (nv > 32) {
+              mask32(s1, 32, nv);
+              mt = max32(s1, mt);
+            }
+            if (nv > 64) {
+              mask32(s2, 64, nv);
+              mt = max32(s2, mt);
+            }
+            if (nv > 96) {
+              mask32(s3, 96, nv);
+              mt = max32(s3, mt);
+            }
+          }
+          const float mxs = mt * c;
+          const bool need = mxs > m + kRescaleThreshold;
+          float alpha = 1.f;
+          if (need) {
+            alpha = ex2(m - mxs);
+            m = mxs;
+          }
+          l *= alpha;
+          // P = exp2(S*c - m) as bf16 pairs over the chunk's own first 16
+          // columns' worth: chunk k's 16 pair columns go to columns 16k..,
+          // all of which were read above.
+          float sa0 = 0.f, sa1 = 0.f;
+          exp_chunk32(s0, c, m, sa0, sa1);
+          tmem_st16_even(tS, s0);
+          if (nv > 32) {
+            exp_chunk32(s1, c, m, sa0, sa1);
+            tmem_st16_even(tS + 16, s1);
+          }
+          if (nv > 64) {
+            exp_chunk32(s2, c, m, sa0, sa1);
+            tmem_st16_even(tS + 32, s2);
+          }
+          if (nv > 96) {
+            exp_chunk32(s3, c, m, sa0, sa1);
+            tmem_st16_even(tS + 48, s3);
+          }
+          l += sa0 + sa1;
+          // O_h to the new max before P_h(i).V adds to it (s_full also
+          // covered P_h(i-1).V, so O_h is settled).  A segment's first P.V
+          // overwrites O, so its first tile needs none.
+          if (i > sa && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < dh; c0 += 16) {
+              uint32_t o[16];
+              tmem_ld16(tO + c0, o);
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = c0 + j < nv ? v[j] : __float_as_uint(-INFINITY);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(-INFINITY);
+              for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+              tmem_st16(tO + c0, o);
             }
-            tmem_st32(tS + c0, v);
           }
           tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_full[wg]);
         }
-        float mc[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) mc[k] = -INFINITY;
-        uint32_t sa[32];
-#pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
-          tmem_ld32(tS + c0, sa);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; j += 2)
-            mc[(j >> 1) & 3] = fmax3(mc[(j >> 1) & 3], __uint_as_float(sa[j]), __uint_as_float(sa[j + 1]));
-        }
-        const float part = fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]);
-        // The first exponential sub-slice is read while the maxima are swapped.
-        uint32_t s_even[16], s_odd[16];  // sub-slices 0, 2 and 1, 3
-        tmem_ld16(tS, s_even);
-        // One buffer suffices: a warp writes tile t+1's value only after
-        // S(t+1), which needs its partner's P(t), written after the read.
-        xch[ch * 32 + lane] = bf16_bits(part);
-        mbar_arrive(xb);
-        if (!mbar_wait(xb, (uint32_t)t & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
-          tmem_wait_ld();
+        if (!ok) break;
+        // The segment's partial: unnormalised O (tile-major [slot][dh/4][256
+        // rows][4], so a warp's float4 store covers 32 consecutive rows, 512
+        // contiguous bytes), the running max (log2 units) and the row sum.
+        if (!mbar_wait(&o_full[wg], (uint32_t)qi & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
           ok = false;
           break;
         }
-        const float mx = fmaxf(bf16_value(xch[lane]), bf16_value(xch[32 + lane]));
-        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 6 + 5 * wg, t);
-        const float mxs = mx * c;
-        const bool need = mxs > m + kRescaleThreshold;
-        float alpha = 1.f;
-        if (need) {
-          alpha = ex2(m - mxs);
-          m = mxs;
-        }
-        l *= alpha;
-        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 7 + 5 * wg, t);
-        // P = exp2(S*c - m) as bf16 pairs, written into this warp's own S
-        // columns (slice i's 16 pair columns over slice i's first half, read
-        // already); one pair in eight on the FMA pipe.
-        float s0 = 0.f, s1 = 0.f;
-        tmem_wait_ld();
-        // Four 16-column sub-slices; the next one's load is in flight while
-        // this one's exponentials run.  P of sub-slice k goes to columns
-        // [8k, 8k+8), which sub-slices already read cover.
-#pragma unroll 1
-        for (int k = 0; k < 4; k += 2) {
-          uint32_t pk[8];
-          tmem_ld16(tS + 16 * (k + 1), s_odd);
-          exp_slice16(s_even, c, m, s0, s1, pk);
-          tmem_st8(tS + 8 * k, pk);
-          tmem_wait_ld();
-          if (k == 0) tmem_ld16(tS + 32, s_even);
-          exp_slice16(s_odd, c, m, s0, s1, pk);
-          tmem_st8(tS + 8 * (k + 1), pk);
-          if (k == 0) tmem_wait_ld();
-        }
-        l += s0 + s1;
-        // O_h to the new max before P_h(t).V adds to it (s_full also
-        // covered P_h(t-1).V, so O_h is settled).
-        if (t > 0 && __any_sync(0xffffffffu, need)) {
-          for (int c0 = 0; c0 < dh2; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c0, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(tO + c0, o);
-          }
-        }
-        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 8 + 5 * wg, t);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[wg]);
-        TT_TRACE_POINT(lane == 0 && q == 0 && ch == 0, 9 + 5 * wg, t);
-      }
-      // Column half 1 hands its row sum to column half 0, which writes the
-      // whole row.  o_full (the last P.V done) implies both warps have read
-      // the last tile's maxima, so the buffer is free.
-      if (ok) ok = mbar_wait(&o_full[wg], 0, a.err, abort_flag, WHERE_ATTN_SOFTMAX);
-      if (ok) {
-        if (ch == 1) {
-          const uint32_t lb = __float_as_uint(l);
-          xch[lane] = (uint16_t)(lb & 0xffffu);
-          xch[32 + lane] = (uint16_t)(lb >> 16);
-        }
-        mbar_arrive(xb);
-        ok = mbar_wait(xb, (uint32_t)n_tiles & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX);
-      }
-      if (ok && ch == 0) {
-        l += __uint_as_float((uint32_t)xch[lane] | ((uint32_t)xch[32 + lane] << 16));
         tc_fence_after();
-        const uint32_t tOr = tmem + tO0 + wg * dh + lane_off;  // the whole O row
+        const int slot = su + cta;
         const bool valid = r < a.rows_per_half;
-        const int s = pos0 + wg * a.s_per_half + r / a.G;
-        const int head = g * a.G + r % a.G;
-        if (a.n_splits == 1) {
-          const float inv = 1.f / l;
-          uint16_t* dst = a.out + (size_t)(b * a.S + s) * a.ldo + head * dh;
-          for (int c0 = 0; c0 < dh; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tOr + c0, o);
-            tmem_wait_ld();
-            if (valid) {
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-                w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-                w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-                w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
-                *reinterpret_cast<uint4*>(dst + c0 + 8 * v) = w;
-              }
-            }
-          }
-        } else {
-          // Partial O is tile-major, [unit][dh/4][256 rows][4]: a warp's
-          // float4 store covers 32 consecutive rows, 512 contiguous bytes.
-          const int r256 = wg * 128 + r;
-          const size_t prow_i = (size_t)unit * 256 + r256;
-          float* po = a.part_o + (size_t)unit * dh * 256 + (size_t)r256 * 4;
-          for (int c0 = 0; c0 < dh; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tOr + c0, o);
-            tmem_wait_ld();
-            if (valid) {
-#pragma unroll
-              for (int v = 0; v < 8; ++v)
-                *reinterpret_cast<float4*>(po + (size_t)(c0 / 4 + v) * 1024) =
-                    make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
-            }
-          }
+        const int r256 = wg * 128 + r;
+        float* po = a.part_o + (size_t)slot * dh * 256 + (size_t)r256 * 4;
+        for (int c0 = 0; c0 < dh; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_wait_ld();
           if (valid) {
-            a.part_ml[prow_i * 2 + 0] = m;
-            a.part_ml[prow_i * 2 + 1] = l;
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              *reinterpret_cast<float4*>(po + (size_t)(c0 / 4 + v) * 1024) =
+                  make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                              __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
           }
         }
+        if (valid)
+          *reinterpret_cast<float2*>(a.part_ml + ((size_t)slot * 256 + r256) * 2) =
+              make_float2(m, l);
+        ++qi;
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 3) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
   }
 }
 
-// Thread per (query row, 4-column group): combine the splits' partials,
+// Thread per (unit, query row, 4-column group): combine the unit's segment
+// partials,
 //   O = sum_i 2^(m_i - m*) O_i / sum_i 2^(m_i - m*) l_i,
-// in one pass over the splits (running max, rescaled sums), four splits'
-// loads in flight before any is used.  Consecutive threads take consecutive
-// rows, so the tile-major partial reads are coalesced.  An empty split
-// (l = 0, O never written) is skipped by selection.
+// in one pass (running max, rescaled sums), four segments' loads in flight
+// before any is used.  Consecutive threads take consecutive rows, so the
+// tile-major partial reads are coalesced.
 __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a) {
   griddep_launch();
   griddep_wait();
@@ -624,24 +705,25 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a) {
   const int ngrp = a.dh / 4;
   const int row256 = (int)(i & 255);
   const int grp = (int)((i >> 8) % ngrp);
-  const int pq = (int)((i >> 8) / ngrp);  // pair * n_qtiles + qt
-  if (pq >= a.B * a.Hkv * a.n_qtiles) return;
+  const int u = (int)((i >> 8) / ngrp);
+  if (u >= a.units) return;
   const int h = row256 >> 7, r = row256 & 127;
   if (h >= a.halves || r >= a.rows_per_half) return;
-  const int pair = pq / a.n_qtiles, qt = pq % a.n_qtiles;
+  const int qt = u % a.n_qtiles, pair = u / a.n_qtiles;
   const int b = pair / a.Hkv, g = pair % a.Hkv;
+  const SegRange sr = unit_segments(a, u);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f, mrun = -INFINITY;
-  for (int sp0 = 0; sp0 < a.n_splits; sp0 += 4) {
+  for (int c0 = sr.c_first; c0 <= sr.c_last; c0 += 4) {
     float2 ml[4];
     float4 o[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const size_t pt = (size_t)pq * a.n_splits + sp0 + k;
-      const bool in = sp0 + k < a.n_splits;
-      ml[k] = in ? *reinterpret_cast<const float2*>(a.part_ml + (pt * 256 + row256) * 2)
+      const bool in = seg_ran(a, sr, c0 + k);
+      const size_t slot = (size_t)u + c0 + k;
+      ml[k] = in ? *reinterpret_cast<const float2*>(a.part_ml + (slot * 256 + row256) * 2)
                  : make_float2(-INFINITY, 0.f);
-      o[k] = in ? *reinterpret_cast<const float4*>(a.part_o + ((pt * ngrp + grp) * 256 + row256) * 4)
+      o[k] = in ? *reinterpret_cast<const float4*>(a.part_o + ((slot * ngrp + grp) * 256 + row256) * 4)
                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
@@ -685,12 +767,16 @@ cudaError_t launch_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKc, const C
   cudaError_t e =
       cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.n_splits, a.n_qtiles, a.B * a.Hkv);
-  return launch_k(attn_kernel, grid, dim3(kAttnThreads), smem, st, tmQ, tmKc, tmVc, tmKb, tmVb, a);
+  return launch_k(attn_kernel, dim3(a.n_ctas), dim3(kAttnThreads), smem, st, tmQ, tmKc, tmVc, tmKb,
+                  tmVb, a);
+}
+
+cudaError_t launch_attn_plan(const AttnArgs& a, cudaStream_t st) {
+  return launch_k(attn_plan_kernel, dim3(1), dim3(1024), 0, st, a);
 }
 
 cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t st) {
-  const long long threads = (long long)a.B * a.Hkv * a.n_qtiles * 256 * (a.dh / 4);
+  const long long threads = (long long)a.units * 256 * (a.dh / 4);
   const int blocks = (int)((threads + 255) / 256);
   return launch_k(attn_merge_kernel, dim3(blocks), dim3(256), 0, st, a);
 }

@@ -42,15 +42,16 @@ enum WhereTag {
 };
 
 // ------------------------------------------------------------------ GEMM
-// C = A[M, K] . B[N, K]^T with both operands K-major bf16.  BM=128, BN=256,
-// BK=64.  Two epilogues: vocabulary statistics (per row and 256-wide column
-// tile: max logit, sum of exp relative to it, argmax) or a plain bf16 store.
-// Tile widths: the vocabulary GEMM uses N tiles of 224 columns (131072
-// columns -> 586 tiles, 3.96 per SM, so the last round is nearly full) with
-// a 5-deep ring; the linear update uses 256-column tiles with a 4-deep ring.
+// C = A[M, K] . B[N, K]^T with both operands K-major bf16, BM=128, BK=64.
+// Two epilogues: vocabulary statistics (per row and column tile: max logit,
+// sum of exp relative to it, argmax) or a plain bf16 store.  Tile widths: the
+// vocabulary GEMM uses N tiles of 224 columns (131072 columns -> 586 tiles,
+// 3.96 per SM, so the last round is nearly full) with a 5-deep ring; the
+// linear update uses 256-column tiles (4608 columns x 1024 rows -> 144
+// tiles, one wave) with a 4-deep ring.
 constexpr int kGemmBM = 128, kGemmBK = 64;
 constexpr int kVocabBN = 224, kVocabStages = 5;
-constexpr int kQkvBN = 128, kQkvStages = 6;
+constexpr int kQkvBN = 256, kQkvStages = 4;
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr size_t gemm_smem_bytes(int bn, int stages) {
   return (size_t)stages * (kGemmBM + bn) * kGemmBK * 2 + 1024 + 256;
@@ -89,34 +90,63 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int
 
 // ------------------------------------------------------------- attention
 constexpr int kAttnBN = 128;       // keys per tile
-// warp 0 TMA, warps 1-2 MMA (one per 128-row half), warp 3 TMEM owner and
-// V padding, warps 4-11 / 12-19 softmax of half 0 / half 1
-constexpr int kAttnThreads = 640;
+// warp 0 TMA Q/K, warp 1 TMEM owner and TMA V + V padding, warps 2-3 MMA
+// (one per 128-row half), warps 4-7 / 8-11 softmax of half 0 / half 1
+constexpr int kAttnThreads = 384;
 
+// A unit is (sequence b, KV head g, query tile qt), u = (b*Hkv + g)*n_qtiles
+// + qt.  Its keys form 1 + ceil(L_b / 128) tiles (tile 0: the block's own S
+// keys).  All units' tiles laid end to end form T tiles, cut into n_ctas
+// contiguous ranges [c*T/n_ctas, (c+1)*T/n_ctas), one per CTA of a
+// persistent grid.  The piece of unit u that CTA c runs (a segment) stores
+// its partial at slot u + c: along the tile sequence both u and c only grow
+// and one of them grows at each new segment, so slots are distinct and
+// fewer than units + n_ctas.
 struct AttnArgs {
   int B, S, Hq, Hkv, dh, G, L_cap;
   const int* ctx_len;
   const int* active;    // optional device flag
   int s_per_half;       // block positions per 128-row half
   int rows_per_half;    // s_per_half * G
-  int halves;           // 128-row halves per query tile and CTA (1 or 2)
-  int n_qtiles;         // CTAs along the query axis per (b, g)
-  int n_splits;         // key splits
-  int chunk;            // context keys per split > 0 (multiple of kAttnBN)
-  int first;            // context keys of split 0, which also runs the block's own tile
+  int halves;           // 128-row halves per query tile (1 or 2)
+  int n_qtiles;         // query tiles per (b, g)
+  int units;            // B * Hkv * n_qtiles
+  int n_ctas;           // CTAs of the persistent grid
+  int* tile_start;      // [units + 1] exclusive prefix sums of tiles per unit (device)
+  int* first_unit;      // [n_ctas] the unit holding each CTA's first tile (device)
   float scale_log2;     // log2(e) / sqrt(dh)
   uint16_t* out;        // bf16 [B*S, ldo]
   int ldo;
   int kv_keep;          // 1: load K/V with evict-last (small cache re-read every step)
-  float* part_o;        // [units][dh/4][256 rows][4] unnormalised partial outputs
-  float* part_ml;       // [units][256][2] (running max in log2 units, sum)
+  float* part_o;        // [units + n_ctas - 1][dh/4][256 rows][4] unnormalised partial outputs
+  float* part_ml;       // [units + n_ctas - 1][256][2] (running max in log2 units, sum)
   int* err;
 };
 size_t attn_smem_bytes(int dh, int halves);
+cudaError_t launch_attn_plan(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKc, const CUtensorMap& tmVc,
                         const CUtensorMap& tmKb, const CUtensorMap& tmVb, const AttnArgs& a,
                         cudaStream_t st);
 cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t st);
+
+#ifdef __CUDACC__
+// The CTAs that ran unit u lie in [c_first, c_last]: c(t) = ((t+1)*n_ctas - 1)
+// / T is the CTA whose range holds tile t (the largest c with c*T/n_ctas <=
+// t).  With fewer tiles than CTAs some CTAs in between have empty ranges and
+// wrote nothing (seg_ran tells).
+struct SegRange {
+  int c_first, c_last;
+  long long T;
+};
+__device__ __forceinline__ SegRange unit_segments(const AttnArgs& a, int u) {
+  const long long T = a.tile_start[a.units], P = a.n_ctas;
+  const long long t0 = a.tile_start[u], t1 = a.tile_start[u + 1] - 1;
+  return SegRange{(int)(((t0 + 1) * P - 1) / T), (int)(((t1 + 1) * P - 1) / T), T};
+}
+__device__ __forceinline__ bool seg_ran(const AttnArgs& a, const SegRange& r, int c) {
+  return c <= r.c_last && (long long)c * r.T / a.n_ctas < (long long)(c + 1) * r.T / a.n_ctas;
+}
+#endif
 
 // ------------------------------------------------------ small kernels
 struct PlanArgs {
@@ -130,15 +160,14 @@ struct PlanArgs {
 };
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st);
 
-// masked == nullptr: all rows, t[b] per sequence.  Otherwise (block loop)
-// only masked rows, with their compact index and t_b computed in the kernel;
-// writes rowlist[j] and ctrl[CTRL_M].
+// adaLN of every row, t[b] per sequence.
 cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
-                         uint16_t* y, int rows, int S, int H, const uint8_t* masked,
-                         int* rowlist, int* ctrl, const int* active, cudaStream_t st);
+                         uint16_t* y, int rows, int S, int H, cudaStream_t st);
 
-// Split merge + adaLN for the masked rows of the loop (attention split > 1);
-// compacts on the fly like launch_adaln's loop mode.
+// Block loop: the attention's segment merge + adaLN.  With a row list, only
+// the masked rows, written compacted (their compact index and t_b computed in
+// the kernel; writes rowlist[j] and ctrl[CTRL_M]); with rowlist == nullptr
+// every row at its own index (a denoiser layer before the last).
 cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, uint16_t* y,
                                const uint8_t* masked, int* rowlist, int* ctrl, cudaStream_t st);
 
@@ -150,10 +179,10 @@ cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_
                          const uint16_t* e_mask, uint16_t* dst, int rows, int H, int V,
                          const int* active, int* err, cudaStream_t st);
 
-// The commit runs as B*ceil(S/kCommitRows) CTAs (one warp per block row); the
+// The commit runs as B*S CTAs of kCommitThreads (one per block row); the
 // last CTA of a sequence to finish (a per-sequence counter) applies the
 // commit rule to the whole sequence.
-constexpr int kCommitRows = 4;
+constexpr int kCommitThreads = 256;
 struct CommitArgs {
   int B, S, n_vt;
   float2* rowres;       // [B*S] (confidence, token bits) of each row

@@ -250,24 +250,14 @@ __device__ bool loop_row(const uint8_t* __restrict__ masked, int rows, int S, in
 
 __global__ void __launch_bounds__(kAdaThreads)
     adaln_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ ss,
-                 const float* __restrict__ t, uint16_t* __restrict__ y, int rows, int S, int H,
-                 const uint8_t* __restrict__ masked, int* __restrict__ rowlist, int* ctrl,
-                 const int* active) {
+                 const float* __restrict__ t, uint16_t* __restrict__ y, int S, int H) {
   griddep_launch();
   griddep_wait();
   __shared__ float red[kAdaThreads / 32];
-  if (active != nullptr && *active == 0) return;
-  // masked == nullptr: every row, t per sequence from `t`; otherwise the block
-  // loop's masked rows only, written compacted.
-  int j = blockIdx.x, src = blockIdx.x;
-  float tb;
-  if (masked == nullptr) {
-    tb = t[src / S];
-  } else if (!loop_row(masked, rows, S, src, rowlist, ctrl, &j, &tb)) {
-    return;
-  }
+  const int row = blockIdx.x;
+  const float tb = t[row / S];
   const int nvec = H / 8;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)src * H);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
   float v[kAdaMaxVec][8];
   float s = 0.f;
 #pragma unroll
@@ -285,15 +275,16 @@ __global__ void __launch_bounds__(kAdaThreads)
       for (int e = 0; e < 8; ++e) s += v[k][e];
     }
   }
-  adaln_finish(v, s, H, tb, ss, y + (size_t)j * H, red);
+  adaln_finish(v, s, H, tb, ss, y + (size_t)row * H, red);
 }
 
-// Attention split merge fused with adaLN (block loop): one CTA per masked
-// row (b, s).  For each query head the split partials are combined,
+// Attention merge fused with adaLN (block loop): one CTA per block row (b, s),
+// returning at once for a committed row unless every row is wanted.  For
+// each query head the unit's segment partials are combined,
 //   o = sum_i 2^(m_i - m*) O_i / sum_i 2^(m_i - m*) l_i,
 // rounded to bf16 (the attention output's storage precision), and the whole
 // row then goes through adaln_finish.
-// KG four-column groups per thread (H <= KG * 4 * kAdaThreads); NB splits'
+// KG four-column groups per thread (H <= KG * 4 * kAdaThreads); NB segments'
 // loads in flight per round.
 template <int KG, int NB>
 __global__ void __launch_bounds__(kAdaThreads)
@@ -314,17 +305,17 @@ __global__ void __launch_bounds__(kAdaThreads)
   const int qt = s / sq, within = s % sq;
   const int hh = within / a.s_per_half, sl = within % a.s_per_half;
   // Each thread merges up to KG four-column groups of the row in one pass
-  // over the splits (running max, rescaled sums), loading NB splits' data
-  // for all its groups before using any.  Group gi covers head
+  // over the segments (running max, rescaled sums), loading NB segments'
+  // data for all its groups before using any.  Group gi covers head
   // gi % Hq, columns 4*(gi / Hq)..+3: consecutive threads take consecutive
-  // heads, i.e. consecutive rows of the tile-major partials (coalesced).  An
-  // empty split (l = 0, O never written) is skipped by selection.
+  // heads, i.e. consecutive rows of the tile-major partials (coalesced).
   constexpr int kG = KG;
   const int ngrp = a.dh / 4, ng = a.Hq * ngrp;
-  size_t pt0[kG];  // partial tile of split 0
-  int r256[kG], grp[kG], i0[kG];
+  int unit[kG], n_seg[kG], r256[kG], grp[kG], i0[kG];
+  SegRange sr[kG];
   bool gin[kG];
   float mrun[kG], den[kG], v[kG][4];
+  int max_seg = 0;
 #pragma unroll
   for (int k = 0; k < kG; ++k) {
     const int gi = (int)threadIdx.x + k * kAdaThreads;
@@ -334,25 +325,28 @@ __global__ void __launch_bounds__(kAdaThreads)
     grp[k] = gc / a.Hq;
     i0[k] = head * a.dh + grp[k] * 4;
     const int g = head / a.G, jh = head % a.G;
-    pt0[k] = (size_t)((b * a.Hkv + g) * a.n_qtiles + qt) * a.n_splits;
+    unit[k] = (b * a.Hkv + g) * a.n_qtiles + qt;
+    sr[k] = unit_segments(a, unit[k]);
+    n_seg[k] = gin[k] ? sr[k].c_last - sr[k].c_first + 1 : 0;
+    max_seg = max(max_seg, n_seg[k]);
     r256[k] = hh * 128 + sl * a.G + jh;
     mrun[k] = -INFINITY;
     den[k] = 0.f;
 #pragma unroll
     for (int e = 0; e < 4; ++e) v[k][e] = 0.f;
   }
-  for (int sp0 = 0; sp0 < a.n_splits; sp0 += NB) {
+  for (int sp0 = 0; sp0 < max_seg; sp0 += NB) {
     float2 ml[NB][kG];
     float4 x[NB][kG];
 #pragma unroll
     for (int i = 0; i < NB; ++i) {
 #pragma unroll
       for (int k = 0; k < kG; ++k) {
-        if (sp0 + i < a.n_splits && gin[k]) {
-          const size_t pt = pt0[k] + sp0 + i;
-          ml[i][k] = *reinterpret_cast<const float2*>(a.part_ml + (pt * 256 + r256[k]) * 2);
+        if (sp0 + i < n_seg[k] && seg_ran(a, sr[k], sr[k].c_first + sp0 + i)) {
+          const size_t slot = (size_t)unit[k] + sr[k].c_first + sp0 + i;
+          ml[i][k] = *reinterpret_cast<const float2*>(a.part_ml + (slot * 256 + r256[k]) * 2);
           x[i][k] = *reinterpret_cast<const float4*>(
-              a.part_o + ((pt * ngrp + grp[k]) * 256 + r256[k]) * 4);
+              a.part_o + ((slot * ngrp + grp[k]) * 256 + r256[k]) * 4);
         } else {
           ml[i][k] = make_float2(-INFINITY, 0.f);
         }
@@ -438,87 +432,96 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------- commit
-// One warp per block row, kCommitRows rows per CTA.  A masked position's
-// tile statistics are merged into its confidence
+// Merge of one tile-statistics entry into a running (best tile maximum v*,
+// its tile and token, Z = sum_t z_t 2^(c (v_t - v*))); a strictly greater
+// maximum wins, equal maxima keep the lower tile (hence the lowest id).
+struct RowBest {
+  float v, Z;
+  int t, tok;
+};
+__device__ __forceinline__ void rb_merge(RowBest& x, const RowBest& y, float c) {
+  if (y.Z == 0.f && y.v == -INFINITY) return;
+  const float nv = fmaxf(x.v, y.v);
+  x.Z = (x.v == nv ? x.Z : x.Z * ex2((x.v - nv) * c)) + (y.v == nv ? y.Z : y.Z * ex2((y.v - nv) * c));
+  if (y.v > x.v || (y.v == x.v && y.t < x.t)) {
+    x.v = y.v;
+    x.t = y.t;
+    x.tok = y.tok;
+  }
+}
+
+// One CTA per block row.  A masked position's ceil(V/224) tile statistics
+// are merged by all kCommitThreads threads (every load of the row in flight
+// at once) into its confidence
 //   conf = 1 / sum_t z_t 2^(c*(v_t - v*)),  token = argmax column of the
 // tile with the largest v_t (lowest tile on ties, hence lowest id).
 // The last CTA of a sequence to finish then applies the commit rule
 // across the sequence's S positions.
-__global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitArgs a) {
+__global__ void __launch_bounds__(kCommitThreads) commit_kernel(const CommitArgs a) {
   griddep_launch();
   griddep_wait();
+  constexpr int kWarps = kCommitThreads / 32;
   __shared__ int s_last;
-  __shared__ int s_tok[kCommitRows * 32];
-  __shared__ int s_com[kCommitRows * 32];
-  __shared__ float s_bc[kCommitRows];
-  __shared__ int s_bs[kCommitRows];
+  __shared__ int s_tok[kCommitThreads];
+  __shared__ int s_com[kCommitThreads];
+  __shared__ float s_bc[kWarps];
+  __shared__ int s_bs[kWarps];
+  __shared__ RowBest s_rb[kWarps];
   if (a.active != nullptr && *a.active == 0) return;
-  const int S = a.S, per_seq = (S + kCommitRows - 1) / kCommitRows;
-  const int b = blockIdx.x / per_seq;
+  const int S = a.S;
+  const int row = blockIdx.x, b = row / S;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int s_row = (blockIdx.x % per_seq) * kCommitRows + warp;
-  const bool row_ok = s_row < S;  // S < kCommitRows leaves warps without a row
-  const int row = b * S + min(s_row, S - 1);
   const int M = a.M_dev != nullptr ? *a.M_dev : a.B * S;
-  float conf = -1.f;
-  int tok = -1;
-  if (row_ok && a.masked[row] != 0) {
+  const float c = a.scale_log2;
+  if (a.masked[row] != 0) {
     const int j = a.rowlist[a.B * S + row];  // this row's compact index
+    RowBest rb{-INFINITY, 0.f, 0x7fffffff, -1};
     if (j >= 0 && j < M) {
-      // One pass over the row's tiles (lane t reads tiles t, t+32, ...):
-      // running best tile maximum v*, its token, and
-      //   Z = sum_t z_t 2^(c (v_t - v*)),
-      // rescaled whenever v* grows.  t increases per lane, so a strict >
-      // keeps the lowest tile on ties.
+      // thread i reads tiles i, i + kCommitThreads, ...: all loads first
       const float4* st = a.stats + (size_t)j * a.n_vt;
-      const float c = a.scale_log2;
-      float bv = -INFINITY, Z = 0.f;
-      int bt = 0x7fffffff, btok = -1;
-      for (int t0 = lane; t0 < a.n_vt; t0 += 32 * 8) {
-        float4 q[8];  // eight loads in flight before any is used
+      constexpr int kPer = 4;  // up to kPer * kCommitThreads tiles in one round
+      for (int t0 = threadIdx.x; t0 < a.n_vt; t0 += kPer * kCommitThreads) {
+        float4 q[kPer];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          q[i] = t0 + 32 * i < a.n_vt ? st[t0 + 32 * i] : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+        for (int i = 0; i < kPer; ++i) {
+          const int t = t0 + i * kCommitThreads;
+          q[i] = t < a.n_vt ? st[t] : make_float4(-INFINITY, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (q[i].x > bv) {
-            Z = (bv == -INFINITY ? 0.f : Z * ex2((bv - q[i].x) * c)) + q[i].y;
-            bv = q[i].x;
-            bt = t0 + 32 * i;
-            btok = __float_as_int(q[i].z);
-          } else if (q[i].x > -INFINITY) {
-            Z += q[i].y * ex2((q[i].x - bv) * c);
-          }
-        }
+        for (int i = 0; i < kPer; ++i)
+          if (q[i].x > -INFINITY)
+            rb_merge(rb, RowBest{q[i].x, q[i].y, t0 + i * kCommitThreads, __float_as_int(q[i].z)},
+                     c);
       }
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int ot = __shfl_xor_sync(0xffffffffu, bt, o);
-        const int otok = __shfl_xor_sync(0xffffffffu, btok, o);
-        const float oZ = __shfl_xor_sync(0xffffffffu, Z, o);
-        const float nv = fmaxf(bv, ov);
-        Z = (bv == nv ? Z : Z * ex2((bv - nv) * c)) + (ov == nv ? oZ : oZ * ex2((ov - nv) * c));
-        if (ov > bv || (ov == bv && ot < bt)) {
-          bv = ov;
-          bt = ot;
-          btok = otok;
-        }
-      }
-      conf = 1.f / Z;
-      tok = bt < a.n_vt ? btok : -1;
     }
+    for (int o = 16; o > 0; o >>= 1) {
+      RowBest y;
+      y.v = __shfl_xor_sync(0xffffffffu, rb.v, o);
+      y.Z = __shfl_xor_sync(0xffffffffu, rb.Z, o);
+      y.t = __shfl_xor_sync(0xffffffffu, rb.t, o);
+      y.tok = __shfl_xor_sync(0xffffffffu, rb.tok, o);
+      rb_merge(rb, y, c);
+    }
+    if (lane == 0) s_rb[warp] = rb;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      RowBest x = s_rb[0];
+      for (int w = 1; w < kWarps; ++w) rb_merge(x, s_rb[w], c);
+      const bool found = j >= 0 && j < M && x.t < a.n_vt;
+      a.rowres[row] = make_float2(found ? 1.f / x.Z : -1.f, __int_as_float(found ? x.tok : -1));
+    }
+  } else if (threadIdx.x == 0) {
+    a.rowres[row] = make_float2(-1.f, __int_as_float(-1));
   }
-  if (lane == 0 && row_ok) a.rowres[row] = make_float2(conf, __int_as_float(tok));
-  __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    s_last = atomicAdd(a.seqcnt + b, 1) == per_seq - 1;
+    s_last = atomicAdd(a.seqcnt + b, 1) == S - 1;
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
   {
-    // One thread per position of sequence b (S <= kCommitRows * 32).
+    // One thread per position of sequence b (S <= kCommitThreads).
     const int s = threadIdx.x;
     const bool in = s < S;
     const int r = b * S + min(s, S - 1);
@@ -553,7 +556,7 @@ __global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitAr
         s_bs[warp] = bs;
       }
       __syncthreads();
-      for (int w = 0; w < kCommitRows; ++w) {
+      for (int w = 0; w < kWarps; ++w) {
         if (s_bc[w] > bc || (s_bc[w] == bc && s_bs[w] < bs)) {
           bc = s_bc[w];
           bs = s_bs[w];
@@ -593,17 +596,17 @@ __global__ void __launch_bounds__(kCommitRows * 32) commit_kernel(const CommitAr
     int nc = 0;
     for (int s = 0; s < S; ++s) nc += s_com[s];
     const long long total = (long long)nc * nv;
-    for (long long v0 = threadIdx.x; v0 < total; v0 += 8 * kCommitRows * 32) {
+    for (long long v0 = threadIdx.x; v0 < total; v0 += 8 * kCommitThreads) {
       uint4 buf[8];
       uint4* dst[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const long long v = v0 + (long long)k * kCommitRows * 32;
+        const long long v = v0 + (long long)k * kCommitThreads;
         dst[k] = nullptr;
         if (v < total) {
-          int c = (int)(v / nv), s = 0;
-          for (;; ++s) {  // the c-th committed position
-            if (s_com[s] && c-- == 0) break;
+          int cc = (int)(v / nv), s = 0;
+          for (;; ++s) {  // the cc-th committed position
+            if (s_com[s] && cc-- == 0) break;
           }
           const int i = (int)(v % nv);
           buf[k] = __ldg(reinterpret_cast<const uint4*>(a.emb + (size_t)s_tok[s] * a.H) + i);
@@ -686,11 +689,9 @@ cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
-                         uint16_t* y, int rows, int S, int H, const uint8_t* masked,
-                         int* rowlist, int* ctrl, const int* active, cudaStream_t st) {
+                         uint16_t* y, int rows, int S, int H, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  return launch_k(adaln_kernel, dim3(rows), dim3(kAdaThreads), 0, st, x, shift_scale, t, y, rows,
-                  S, H, masked, rowlist, ctrl, active);
+  return launch_k(adaln_kernel, dim3(rows), dim3(kAdaThreads), 0, st, x, shift_scale, t, y, S, H);
 }
 
 cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, uint16_t* y,
@@ -720,8 +721,7 @@ cudaError_t launch_embed(const int* tokens, const uint8_t* masked, const uint16_
 }
 
 cudaError_t launch_commit(const CommitArgs& a, cudaStream_t st) {
-  const int per_seq = (a.S + kCommitRows - 1) / kCommitRows;
-  return launch_k(commit_kernel, dim3(a.B * per_seq), dim3(kCommitRows * 32), 0, st, a);
+  return launch_k(commit_kernel, dim3(a.B * a.S), dim3(kCommitThreads), 0, st, a);
 }
 
 cudaError_t launch_selftest_wait(int* ctrl, unsigned long long limit_ns, cudaStream_t st) {

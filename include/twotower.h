@@ -98,16 +98,17 @@ TT_API tt_status tt_selftest_timeout(void* ws, int32_t limit_us, void* stream);
 /* Number of kernels this library has launched in this process so far. */
 TT_API uint64_t tt_launch_count(void);
 
-/* Number of key splits the attention uses (0 = choose automatically, the
- * default; otherwise at most 64).  Process-wide; results are independent of
- * it up to float rounding. */
+/* Number of CTAs the attention's key tiles are divided over (0 = one per SM,
+ * the default; otherwise at most 64): all units' tiles, laid end to end, are
+ * cut into that many equal contiguous ranges.  Process-wide; results are
+ * independent of it up to float rounding. */
 TT_API tt_status tt_set_attn_splits(int32_t n_splits);
 
 /* Kernel kinds of the per-kernel profiler. */
 enum {
   TT_K_PLAN = 0, TT_K_EMBED = 1, TT_K_GEMM_QKV = 2, TT_K_ATTN = 3, TT_K_MERGE = 4,
   TT_K_ADALN = 5, TT_K_GEMM_VOCAB = 6, TT_K_COMMIT = 7, TT_K_GATHER = 8, TT_K_INIT = 9,
-  TT_K_REDUCE = 10, TT_K_APPEND = 11, TT_K_COUNT = 12
+  TT_K_REDUCE = 10, TT_K_APPEND = 11, TT_K_ATTN_PLAN = 12, TT_K_COUNT = 13
 };
 
 /* Per-kernel profiler: while enabled, every kernel this library launches is

@@ -64,7 +64,14 @@ def fallback_near_tie(conf_masked) -> bool:
     return bool(len(cb) > 1 and cb[0] != cb[1] and (cb[0] - cb[1]) / cb[0] < TIE_FALLBACK_REL)
 
 
-def compare_loop(inp, g_tokens, g_commit_step, gamma, logit_scale):
+# End-to-end comparison with the kernel's own vocabulary rows at hand: the
+# rows of every step must agree with the oracle's float64 rows within this
+# relative L2 (the attention bar of rel-L2 1e-2 carried through LayerNorm,
+# which is scale-free, plus the bf16 rounding of the rows, 2^-9 relative).
+Y_REL_L2 = 2e-2
+
+
+def compare_loop(inp, g_tokens, g_commit_step, gamma, logit_scale, g_rows=None):
     """End-to-end comparison of a kernel's block loop with the oracle's.
 
     The oracle runs teacher-forced: each of its steps starts from the state
@@ -72,6 +79,14 @@ def compare_loop(inp, g_tokens, g_commit_step, gamma, logit_scale):
     final tokens), so one near tie cannot cascade.  ``inp`` holds the loop's
     inputs (tt_inputs arrays, already restricted to the sequences to check);
     ``g_tokens`` / ``g_commit_step`` [B,S] are the kernel's results.
+
+    ``g_rows`` (optional): per step k, a dict {(b, s): the kernel's adaLN row
+    of masked position (b, s), float64}.  With it a sequence-step whose
+    decisions the oracle's own arithmetic takes differently on the kernel's
+    rows than on its float64 rows is excluded and counted as explained by
+    the row difference, and the rows' relative L2 difference is measured
+    (``y_rel_l2_max``; the caller holds it to Y_REL_L2).  Without it the
+    fixed near-tie bands above decide.
 
     Returns (counts, problems): counts of compared and excluded
     sequence-steps, compared committed tokens, near-tie top-2 flips and
@@ -88,10 +103,28 @@ def compare_loop(inp, g_tokens, g_commit_step, gamma, logit_scale):
     r = O.denoise_block_loop(inp, gamma, logit_scale, max_steps=int(cs.max()) + 1, teacher=state)
     w64 = None
     cnt = dict(seq_steps=0, seq_steps_excluded=0, tokens=0, top2_flips=0, spec_excluded=0)
+    if g_rows is not None:
+        cnt.update(y_explained=0, y_rel_l2_max=0.0)
     problems = []
     for k, st in enumerate(r["trace"]):
-        _, m_k = state(k)
+        tok_k, m_k = state(k)
         cnt["spec_excluded"] += int((m_k & spec_excluded(st["conf"], st["gap_p"], gamma)).sum())
+        alt = None
+        if g_rows is not None:
+            # the oracle's decisions on the kernel's rows of this step
+            if w64 is None:
+                w64 = O.from_bf16(inp["w"])
+            keys = [(b, s) for b in range(m_k.shape[0]) for s in range(m_k.shape[1]) if m_k[b, s]]
+            yg = np.stack([g_rows[k][key] for key in keys])
+            yo = np.stack([st["y"][b, s] for b, s in keys])
+            rel = np.linalg.norm(yg - yo, axis=1) / np.maximum(np.linalg.norm(yo, axis=1), 1e-30)
+            cnt["y_rel_l2_max"] = max(cnt["y_rel_l2_max"], float(rel.max()))
+            c_g, t_g, _, _ = O.vocab_confidence(yg, w64, logit_scale)
+            conf_g = np.full(m_k.shape, np.nan)
+            tok_g = np.full(m_k.shape, -1, np.int64)
+            for j, (b, s) in enumerate(keys):
+                conf_g[b, s], tok_g[b, s] = c_g[j], t_g[j]
+            alt = O.commit(conf_g, tok_g, tok_k, m_k, gamma)
         for b in range(m_k.shape[0]):
             if not m_k[b].any():
                 continue
@@ -102,6 +135,11 @@ def compare_loop(inp, g_tokens, g_commit_step, gamma, logit_scale):
             ex |= (ora_c & derived_excluded_argmax(st["gap_l"][b])).any()
             if st["fallback"][b]:
                 ex |= fallback_near_tie(conf[m_k[b]])
+            if not ex and alt is not None and (
+                    not np.array_equal(alt[2][b], ora_c)
+                    or not np.array_equal(alt[0][b][ora_c], st["tokens"][b][ora_c])):
+                cnt["y_explained"] += 1
+                ex = True
             if ex:
                 cnt["seq_steps_excluded"] += 1
                 continue

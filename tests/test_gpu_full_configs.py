@@ -33,8 +33,9 @@ def test_loop64_gamma_sweep_sampled_sequences(loop64, gamma, logit_scale):
     check_invariants(d, inp, g)
     if logit_scale == 1.0:
         assert g["steps_run"] == 16          # nothing reaches gamma: one commit per step
-    stepwise_equals_single_call(d, inp, gamma, logit_scale, g, bsel=[0, 63])
-    n_cmp, n_ex = compare_teacher_forced(inp, g, gamma, logit_scale, bsel=np.array([0, 63]))
+    steps = stepwise_equals_single_call(d, inp, gamma, logit_scale, g, bsel=[0, 63])
+    n_cmp, n_ex = compare_teacher_forced(inp, g, gamma, logit_scale, bsel=np.array([0, 63]),
+                                      steps=steps)
     print(f"loop64 gamma={gamma} scale={logit_scale}: steps {g['steps_run']}, "
           f"compared {n_cmp} sequence-steps, excluded {n_ex}")
     assert n_cmp > 0 and n_ex <= 3
@@ -52,8 +53,8 @@ def test_loop_ragged16_sampled_sequences(ragged16):
     check_invariants(d, inp, g)
     cl = inp["ctx_len"]
     sel = np.array(sorted({int(np.argmin(cl)), int(np.argmax(cl)), 7}))
-    stepwise_equals_single_call(d, inp, 0.8, 8.0, g, bsel=sel)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, 8.0, bsel=sel)
+    steps = stepwise_equals_single_call(d, inp, 0.8, 8.0, g, bsel=sel)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, 8.0, bsel=sel, steps=steps)
     print(f"ragged16 loop: sequences {sel.tolist()} (ctx {cl[sel].tolist()}), "
           f"compared {n_cmp} sequence-steps, excluded {n_ex}")
     assert n_cmp > 0 and n_ex <= 3
@@ -68,8 +69,8 @@ def test_loop_ragged32_sampled_sequences(logit_scale):
     check_invariants(d, inp, g)
     cl = inp["ctx_len"]
     sel = np.array(sorted({int(np.argmin(cl)), int(np.argmax(cl)), 11}))
-    stepwise_equals_single_call(d, inp, 0.8, logit_scale, g, bsel=sel)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, bsel=sel)
+    steps = stepwise_equals_single_call(d, inp, 0.8, logit_scale, g, bsel=sel)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, bsel=sel, steps=steps)
     print(f"ragged32 loop scale={logit_scale}: sequences {sel.tolist()} "
           f"(ctx {cl[sel].tolist()}), compared {n_cmp} sequence-steps, excluded {n_ex}")
     assert n_cmp > 0 and n_ex <= 3
@@ -85,8 +86,9 @@ def test_loop_long_context_full_batch(logit_scale):
     check_invariants(d, inp, g)
     if logit_scale == 1.0:
         assert g["steps_run"] == 16
-    stepwise_equals_single_call(d, inp, 0.8, logit_scale, g)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, bsel=np.array([0, 3]))
+    steps = stepwise_equals_single_call(d, inp, 0.8, logit_scale, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, bsel=np.array([0, 3]),
+                                      steps=steps)
     print(f"long loop scale={logit_scale}: compared {n_cmp} sequence-steps, excluded {n_ex}")
     assert n_cmp > 0 and n_ex <= 2
 

@@ -181,7 +181,7 @@ def stepwise_equals_single_call(d, inp, gamma, logit_scale, single, n_layers=1, 
     cnt = check_stagewise(d, steps, inp["w"], gamma, logit_scale, bsel=bsel)
     assert cnt["seq_steps"] > 0
     assert cnt["seq_steps_excluded"] <= max_seq_steps_excluded, cnt
-    return cnt
+    return steps
 
 
 def slice_batch(inp, bsel):
@@ -194,20 +194,48 @@ def slice_batch(inp, bsel):
     return out
 
 
-def compare_teacher_forced(inp, g, gamma, logit_scale, bsel=None):
+def rows_by_position(steps, S, bsel=None):
+    """The stepwise run's vocabulary rows as {(b, s): float64 row} per step,
+    b counted within ``bsel`` (all sequences by default)."""
+    out = []
+    for st in steps:
+        rows = {}
+        for j, rid in enumerate(st["row_ids"]):
+            b, s = divmod(int(rid), S)
+            if bsel is None:
+                rows[(b, s)] = st["y"][j]
+            elif b in bsel:
+                rows[(bsel.index(b), s)] = st["y"][j]
+        out.append({k: O.from_bf16(v) for k, v in rows.items()})
+    return out
+
+
+def compare_teacher_forced(inp, g, gamma, logit_scale, bsel=None, steps=None):
     """End-to-end comparison (oracle.parity.compare_loop) on the sequences
     ``bsel``; every disagreement outside the exclusions fails, near-tie top-2
-    flips are reported and bounded.  Returns (compared, excluded)
-    sequence-steps."""
+    flips are reported and bounded.  With ``steps`` (the step-at-a-time run of
+    the same trajectory) the kernel's rows are compared with the oracle's
+    (relative L2 within oracle.parity.Y_REL_L2) and decisions that the
+    oracle itself takes differently on the two sets of rows are excluded and
+    counted.  Returns (compared, excluded) sequence-steps."""
+    S = inp["masked"].shape[1]
+    g_rows = None
+    if steps is not None:
+        g_rows = rows_by_position(steps, S, None if bsel is None else [int(b) for b in bsel])
     if bsel is not None:
         inp = slice_batch(inp, bsel)
         g = {k: (v[bsel] if isinstance(v, np.ndarray) else v) for k, v in g.items()}
-    cnt, problems = P.compare_loop(inp, g["tokens"], g["commit_step"], gamma, logit_scale)
+    cnt, problems = P.compare_loop(inp, g["tokens"], g["commit_step"], gamma, logit_scale,
+                                   g_rows=g_rows)
     print(f"end-to-end: {cnt}")
     assert not problems, problems[:5]
     # a flip needs the oracle's top-2 logit gap below the attention-error
     # band; with these inputs that is a minority of the committed tokens
     assert cnt["top2_flips"] <= max(1, cnt["tokens"] // 4), cnt
+    if g_rows is not None:
+        assert cnt["y_rel_l2_max"] <= P.Y_REL_L2, cnt
+        n = cnt["seq_steps"] + cnt["seq_steps_excluded"]
+        assert cnt["y_explained"] <= max(1, n // 4), cnt
     return cnt["seq_steps"], cnt["seq_steps_excluded"]
 
 
@@ -235,8 +263,8 @@ def test_loop_tiny(gamma, logit_scale):
     inp = tt_inputs.generate(d, seed=31)
     g = run_loop_gpu(d, inp, gamma, logit_scale)
     check_invariants(d, inp, g)
-    stepwise_equals_single_call(d, inp, gamma, logit_scale, g)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, gamma, logit_scale)
+    steps = stepwise_equals_single_call(d, inp, gamma, logit_scale, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, gamma, logit_scale, steps=steps)
     assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
 
 
@@ -247,8 +275,8 @@ def test_loop_tiny_block_of_32(gamma, logit_scale):
     inp = tt_inputs.generate(d, seed=34)
     g = run_loop_gpu(d, inp, gamma, logit_scale)
     check_invariants(d, inp, g)
-    stepwise_equals_single_call(d, inp, gamma, logit_scale, g)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, gamma, logit_scale)
+    steps = stepwise_equals_single_call(d, inp, gamma, logit_scale, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, gamma, logit_scale, steps=steps)
     assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
 
 
@@ -260,8 +288,8 @@ def test_loop_autoregressive_step_s1(logit_scale):
     g = run_loop_gpu(d, inp, 0.8, logit_scale)
     check_invariants(d, inp, g)
     assert g["steps_run"] == 1 and np.all(g["steps_taken"] == 1)
-    stepwise_equals_single_call(d, inp, 0.8, logit_scale, g, max_seq_steps_excluded=1)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale)
+    steps = stepwise_equals_single_call(d, inp, 0.8, logit_scale, g, max_seq_steps_excluded=1)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, steps=steps)
     assert n_cmp + n_ex == d.B and n_ex <= 1, (n_cmp, n_ex)
 
 
@@ -271,8 +299,8 @@ def test_loop_larger_blocks(S, logit_scale):
     inp = tt_inputs.generate(d, seed=43)
     g = run_loop_gpu(d, inp, 0.8, logit_scale)
     check_invariants(d, inp, g)
-    stepwise_equals_single_call(d, inp, 0.8, logit_scale, g)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale)
+    steps = stepwise_equals_single_call(d, inp, 0.8, logit_scale, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, steps=steps)
     assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
 
 
@@ -285,8 +313,8 @@ def test_loop_widest_hidden_and_group(logit_scale):
     inp = tt_inputs.generate(d, seed=44)
     g = run_loop_gpu(d, inp, 0.8, logit_scale)
     check_invariants(d, inp, g)
-    stepwise_equals_single_call(d, inp, 0.8, logit_scale, g)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale)
+    steps = stepwise_equals_single_call(d, inp, 0.8, logit_scale, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, steps=steps)
     assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
 
 
@@ -322,8 +350,9 @@ def test_loop_full_mid_shape_sampled_sequences(logit_scale):
     check_invariants(d, inp, g)
     if logit_scale == 1.0:
         assert g["steps_run"] == 16
-    stepwise_equals_single_call(d, inp, 0.8, logit_scale, g)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, bsel=np.array([0, 5]))
+    steps = stepwise_equals_single_call(d, inp, 0.8, logit_scale, g)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, bsel=np.array([0, 5]),
+                                      steps=steps)
     print(f"mid loop scale={logit_scale}: compared {n_cmp} sequence-steps, excluded {n_ex}")
     assert n_cmp > 0 and n_ex <= 2
 
@@ -334,8 +363,8 @@ def test_loop_layers_tiny(n_layers, logit_scale):
     inp = tt_inputs.generate(d, seed=47, n_layers=n_layers)
     g = run_loop_layers_gpu(d, inp, n_layers, 0.8, logit_scale)
     check_invariants(d, inp, g)
-    stepwise_equals_single_call(d, inp, 0.8, logit_scale, g, n_layers=n_layers)
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale)
+    steps = stepwise_equals_single_call(d, inp, 0.8, logit_scale, g, n_layers=n_layers)
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, logit_scale, steps=steps)
     assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
 
 
@@ -353,8 +382,8 @@ def test_loop_layers_mid_shape_sampled_sequences():
     inp = tt_inputs.generate(d, seed=2, n_layers=2)
     g = run_loop_layers_gpu(d, inp, 2, 0.8, 8.0)
     check_invariants(d, inp, g)
-    stepwise_equals_single_call(d, inp, 0.8, 8.0, g, n_layers=2, bsel=[1, 6])
-    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, 8.0, bsel=np.array([1, 6]))
+    steps = stepwise_equals_single_call(d, inp, 0.8, 8.0, g, n_layers=2, bsel=[1, 6])
+    n_cmp, n_ex = compare_teacher_forced(inp, g, 0.8, 8.0, bsel=np.array([1, 6]), steps=steps)
     print(f"mid 2-layer loop: compared {n_cmp} sequence-steps, excluded {n_ex}")
     assert n_cmp > 0 and n_ex <= 2
 

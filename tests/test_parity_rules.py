@@ -61,3 +61,26 @@ def test_exclusion_rules_on_hand_values():
     assert not P.fallback_near_tie([0.3, 0.3, 0.1])        # exact tie: compared (lowest s wins)
     assert not P.fallback_near_tie([0.3, 0.2])
     assert not P.fallback_near_tie([0.3])
+
+
+def test_rows_supplied_compare_clean_and_measure_the_row_difference():
+    """With the kernel's rows at hand the comparison measures them against
+    the oracle's; the oracle's own rows give zero difference and nothing to
+    explain, slightly perturbed rows a small difference."""
+    d, inp, tok, cs = _tiny_run(12.0)
+    m0 = inp["masked"].astype(bool)
+
+    def state(step):
+        done = (cs >= 0) & (cs < step)
+        return np.where(done, tok, inp["tokens"]), m0 & ~done
+
+    r = O.denoise_block_loop(inp, 0.8, 12.0, max_steps=int(cs.max()) + 1, teacher=state)
+    rows = [{(b, s): st["y"][b, s] for b in range(d.B) for s in range(d.S) if state(k)[1][b, s]}
+            for k, st in enumerate(r["trace"])]
+    cnt, problems = P.compare_loop(inp, tok, cs, 0.8, 12.0, g_rows=rows)
+    assert problems == [] and cnt["y_rel_l2_max"] == 0.0 and cnt["y_explained"] == 0
+    rng = np.random.default_rng(1)
+    noisy = [{k: v * (1 + 1e-3 * rng.standard_normal(v.shape)) for k, v in st.items()}
+             for st in rows]
+    cnt, _ = P.compare_loop(inp, tok, cs, 0.8, 12.0, g_rows=noisy)
+    assert 5e-4 < cnt["y_rel_l2_max"] < 2e-3
