@@ -220,7 +220,7 @@ static AttnGeom attn_geom(const tt_dims& d) {
   g.n_ctas = forced > 0 ? forced : num_sms();
   g.slots = g.units + g.n_ctas - 1;
   g.part_o_bytes = (size_t)g.slots * 256 * d.dh * sizeof(float);
-  g.part_ml_bytes = (size_t)g.slots * 256 * 2 * sizeof(float);
+  g.part_ml_bytes = (size_t)g.slots * 256 * 4 * sizeof(float);
   return g;
 }
 
@@ -267,6 +267,8 @@ struct Ws {
   float* part_ml = nullptr;
   int* tile_start = nullptr;   // attention plan: tiles per unit, prefix sums
   int* first_unit = nullptr;   // attention plan: first unit of each CTA
+  int2* unit_ctas = nullptr;   // attention plan: first and last CTA of each unit
+  int* cta_ran = nullptr;      // attention plan: CTAs whose range holds a tile
   float4* stats = nullptr;
   float* qkv_partial = nullptr;
   uint16_t* xrows = nullptr;  // loop: one layer's modulated rows for the next layer
@@ -291,6 +293,8 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     const AttnGeom g = attn_geom(d);
     w.tile_start = c.take<int>((size_t)(g.units + 1) * sizeof(int));
     w.first_unit = c.take<int>((size_t)g.n_ctas * sizeof(int));
+    w.unit_ctas = c.take<int2>((size_t)g.units * sizeof(int2));
+    w.cta_ran = c.take<int>((size_t)g.n_ctas * sizeof(int));
     w.part_o = c.take<float>(g.part_o_bytes);
     w.part_ml = c.take<float>(g.part_ml_bytes);
   }
@@ -371,6 +375,8 @@ static AttnArgs attn_args(const tt_dims& d, const AttnGeom& g, const int32_t* ct
   a.n_ctas = g.n_ctas;
   a.tile_start = w.tile_start;
   a.first_unit = w.first_unit;
+  a.unit_ctas = w.unit_ctas;
+  a.cta_ran = w.cta_ran;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.dh));
   a.out = out;
   a.ldo = d.H;

@@ -22,18 +22,19 @@
 //   S_h  = Q_h . K(i)^T       (TMEM, 128 fp32 columns; Q and K from smem)
 //   P_h  = exp2(S_h*c - m)    (bf16 pairs, written back over S_h's columns)
 //   O_h += P_h . V(i)         (TMEM accumulator; A = P_h read from TMEM)
-// so P never goes through shared memory.  Roles (12 warps):
+// so P never goes through shared memory.  Roles (20 warps):
 //   warp 0     TMA for Q and K (3-slot ring);
 //   warp 1     TMEM owner; TMA for V (2-slot ring) and zeroing of the V rows
 //              past the last valid key that a 16-key MMA step still reads;
-//   warps 2, 3 MMA issue for half 0 / half 1: P_h(i).V(i) once softmax h has
-//              written P_h(i), then S_h(i+1) into the same columns (tcgen05
-//              MMAs of one thread execute in issue order);
-//   warps 4-7 / 8-11  softmax of half 0 / half 1: thread = query row (TMEM
-//              lane), the whole 128-key row of S in registers, so the row
-//              maximum needs no exchange and S is read from TMEM once.
+//   warps 2, 3 MMA issue for half 0 / half 1: P_h(i).V(i) as soon as
+//              softmax h has written P_h(i), then S_h(i+1) into the same
+//              columns (tcgen05 MMAs of one thread execute in issue order);
+//   warps 4-11 / 12-19  softmax of half 0 / half 1.  Warp w serves the 32
+//              rows of its TMEM lane quarter (w % 4) and one 64-key column
+//              half of every tile; the two warps of a row swap partial row
+//              maxima through shared memory.  Thread = row: no shuffles.
 // The two softmax groups take turns tile by tile, so the tensor core runs
-// one half's MMAs during the other half's softmax.  Part of the
+// one half's MMAs during the other half's softmax.  An eighth of the
 // exponentials run on the FMA pipe (exp2_poly) to offload the MUFU unit.
 // The running max only moves (and O is rescaled in TMEM) when it grows by
 // more than 2^8; the final O / l is exact for any stale max.
@@ -54,16 +55,9 @@ constexpr int kKSlots = 3, kVSlots = 2;       // K and V ring depths
 constexpr uint32_t kKVSub = kAttnBN * 128;    // 128 keys x 64 dh bf16 (128-byte rows) = 16 KB
 constexpr uint32_t kQSub = 16384;             // 128 rows x 64 dh bf16
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
-// Of every 16 exponential pairs of a 32-key chunk, this many run on the FMA
-// pipe (exp2_poly), the rest on MUFU.
-#ifndef TT_ATTN_POLY_PAIRS
-#define TT_ATTN_POLY_PAIRS 3
-#endif
-constexpr int kPolyPairs = TT_ATTN_POLY_PAIRS;
-constexpr int kPolyStride = kPolyPairs > 0 ? 16 / kPolyPairs : 17;  // pairs j = stride-1, 2*stride-1, ...
 
 struct AttnSmem {
-  uint32_t q, k, v, bars, total;
+  uint32_t q, k, v, bars, xchg, total;
 };
 
 __host__ __device__ inline AttnSmem attn_layout(int dh, int halves) {
@@ -72,8 +66,9 @@ __host__ __device__ inline AttnSmem attn_layout(int dh, int halves) {
   L.q = 0;
   L.k = L.q + (uint32_t)halves * nsub * kQSub;
   L.v = L.k + kKSlots * nsub * kKVSub;
-  L.bars = L.v + kVSlots * nsub * kKVSub;
-  L.total = L.bars + 256;
+  L.bars = L.v + kVSlots * nsub * kKVSub;  // 28 mbarriers, then control words
+  L.xchg = L.bars + 256;      // row-max exchange: [half][quarter][column half][lane] bf16
+  L.total = L.xchg + 1024;
   return L;
 }
 
@@ -156,41 +151,6 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return x > -126.0f ? r : 0.f;
 }
 
-// P for a 32-key chunk of S (registers) as 16 bf16 pairs, written in place:
-// pair j goes to sv[2j] (the registers of S it came from are dead by then);
-// kPolyPairs of the pairs on the FMA pipe.
-__device__ __forceinline__ void exp_chunk32(uint32_t (&sv)[32], float c, float m, float& s0,
-                                            float& s1) {
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float x0 = fmaf(__uint_as_float(sv[2 * j]), c, -m);
-    const float x1 = fmaf(__uint_as_float(sv[2 * j + 1]), c, -m);
-    float p0, p1;
-    if (j % kPolyStride == kPolyStride - 1) {
-      p0 = exp2_poly(x0);
-      p1 = exp2_poly(x1);
-    } else {
-      p0 = ex2(x0);
-      p1 = ex2(x1);
-    }
-    s0 += p0;
-    s1 += p1;
-    sv[2 * j] = pack_bf16x2(p0, p1);
-  }
-}
-
-// TMEM store of 16 columns from the even registers of a 32-register chunk
-// (32x32b shape: a thread's lane, consecutive columns).
-__device__ __forceinline__ void tmem_st16_even(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[2]), "r"(r[4]), "r"(r[6]), "r"(r[8]), "r"(r[10]), "r"(r[12]), "r"(r[14]),
-      "r"(r[16]), "r"(r[18]), "r"(r[20]), "r"(r[22]), "r"(r[24]), "r"(r[26]), "r"(r[28]),
-      "r"(r[30])
-      : "memory");
-}
-
 // TMEM load of 16 columns (32x32b shape: a thread's lane, consecutive columns).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -199,25 +159,36 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
+      : "r"(taddr));
 }
-
-__device__ __forceinline__ float max32(const uint32_t (&v)[32], float m) {
-  float a = m, b = -INFINITY, cc = -INFINITY;
+// P for 16 score columns as 8 bf16 pairs, written in place: pair j/2 goes to
+// sv[j] (the registers of S it came from are dead by then); the last pair
+// on the FMA pipe.
+__device__ __forceinline__ void exp_slice16(uint32_t (&sv)[16], float c, float m, float& s0,
+                                            float& s1) {
 #pragma unroll
-  for (int j = 0; j < 30; j += 6) {
-    a = fmax3(a, __uint_as_float(v[j]), __uint_as_float(v[j + 1]));
-    b = fmax3(b, __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-    cc = fmax3(cc, __uint_as_float(v[j + 4]), __uint_as_float(v[j + 5]));
+  for (int j = 0; j < 16; j += 2) {
+    const float x0 = fmaf(__uint_as_float(sv[j]), c, -m);
+    const float x1 = fmaf(__uint_as_float(sv[j + 1]), c, -m);
+    float p0, p1;
+    if (j == 14) {
+      p0 = exp2_poly(x0);
+      p1 = exp2_poly(x1);
+    } else {
+      p0 = ex2(x0);
+      p1 = ex2(x1);
+    }
+    s0 += p0;
+    s1 += p1;
+    sv[j] = pack_bf16x2(p0, p1);
   }
-  a = fmax3(a, __uint_as_float(v[30]), __uint_as_float(v[31]));
-  return fmax3(a, b, cc);
 }
-
-__device__ __forceinline__ void mask32(uint32_t (&v)[32], int base, int nv) {
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = base + j < nv ? v[j] : __float_as_uint(-INFINITY);
+// TMEM store of the 8 pairs exp_slice16 left in the even registers.
+__device__ __forceinline__ void tmem_st8_even(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[2]), "r"(r[4]), "r"(r[6]), "r"(r[8]), "r"(r[10]), "r"(r[12]),
+               "r"(r[14])
+               : "memory");
 }
 
 // Tiles per unit and their exclusive prefix sums (one CTA), then the first
@@ -268,7 +239,11 @@ __global__ void __launch_bounds__(1024) attn_plan_kernel(const AttnArgs a) {
     const long long s0 = start[u], s1 = start[u + 1];
     const long long c0 = (s0 * P + T - 1) / T, c1 = (s1 * P + T - 1) / T;
     for (long long c = c0; c < c1 && c < P; ++c) a.first_unit[c] = u;
+    // the merges' view: the CTAs holding the unit's first and last tiles
+    a.unit_ctas[u] = make_int2((int)(((s0 + 1) * P - 1) / T), (int)((s1 * P - 1) / T));
   }
+  for (int c = tid; c < a.n_ctas; c += blockDim.x)
+    a.cta_ran[c] = (long long)c * T / P < (long long)(c + 1) * T / P ? 1 : 0;
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -304,7 +279,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* s_full = v_ready + kVSlots;  // [half]: S_h(i) ready (and P_h(i-1).V done)
   uint64_t* p_full = s_full + 2;         // [half]: P_h(i) written, O_h corrected
   uint64_t* o_full = p_full + 2;         // [half]: the segment's last P.V done
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 2);
+  uint64_t* xbar = o_full + 2;           // [half][quarter]: both column halves' values written
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 8);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -336,9 +312,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&s_full[h], 1);
-      mbar_init(&p_full[h], 128);
+      mbar_init(&p_full[h], 256);
       mbar_init(&o_full[h], 1);
     }
+    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -475,42 +452,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t dQ = sdesc_sw128(smem_u32(sQ) + h * nsub * kQSub, 16, 1024);
       const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
       const uint64_t dV0 = sdesc_sw128(smem_u32(sV), kKVSub, 1024);
-      // S_h = Q_h . K(kt)^T
-      auto scores = [&](int kt) -> bool {
-        const int ks = kt % kKSlots;
-        if (!mbar_wait(&k_full[ks], (uint32_t)(kt / kKSlots) & 1u, a.err, abort_flag,
-                       WHERE_ATTN_MMA))
-          return false;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint64_t dK = dK0 + (uint64_t)((uint32_t)(ks * nsub) * (kKVSub >> 4));
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            if (kk < dh / 16)
-              umma_bf16_ss(tS, dQ + (uint64_t)(((kk >> 2) * kQSub + (kk & 3) * 32) >> 4),
-                           dK + (uint64_t)(((kk >> 2) * kKVSub + (kk & 3) * 32) >> 4), idS,
-                           kk > 0);
-          }
-          umma_commit(&s_full[h]);
-          umma_commit(&k_empty[ks]);
-        }
-        __syncwarp();
-        return true;
-      };
-      int kt = 0, pt = 0, qi = 0;
+      int kt = 0, pt = 0, qi = 0;  // tiles, turns, segments
       bool ok = true;
       while (ok && walk.next(su, sa, sb)) {
         const UnitInfo ui = unit_info(a, su);
         const int n = sb - sa;
+        // S_h = Q_h . K(local tile i)^T; the K slot is free once the MMA has
+        // read it (both halves), Q once the segment's last S has.
+        auto scores = [&](int i) -> bool {
+          const int ks = (kt + i) % kKSlots;
+          if (!mbar_wait(&k_full[ks], (uint32_t)((kt + i) / kKSlots) & 1u, a.err, abort_flag,
+                         WHERE_ATTN_MMA))
+            return false;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint64_t dK = dK0 + (uint64_t)((uint32_t)(ks * nsub) * (kKVSub >> 4));
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              if (kk < dh / 16)
+                umma_bf16_ss(tS, dQ + (uint64_t)(((kk >> 2) * kQSub + (kk & 3) * 32) >> 4),
+                             dK + (uint64_t)(((kk >> 2) * kKVSub + (kk & 3) * 32) >> 4), idS,
+                             kk > 0);
+            }
+            umma_commit(&s_full[h]);
+            umma_commit(&k_empty[ks]);
+            if (i == n - 1) umma_commit(q_empty);
+          }
+          __syncwarp();
+          return true;
+        };
         ok = mbar_wait(q_full, (uint32_t)qi & 1u, a.err, abort_flag, WHERE_ATTN_MMA);
         if (ok) tc_fence_after();
-        if (ok) ok = scores(kt);
-        if (ok && n == 1 && lane == 0) umma_commit(q_empty);
+        if (ok) ok = scores(0);
         for (int i = 0; ok && i < n; ++i, ++pt) {
           // O_h += P_h(i) . V(i), once warp 1 has cleared V(i)'s padding rows
+          const int vs = (kt + i) % kVSlots;
           if (!mbar_wait(&p_full[h], (uint32_t)pt & 1u, a.err, abort_flag, WHERE_ATTN_MMA) ||
-              !mbar_wait(&v_ready[(kt + i) % kVSlots], (uint32_t)((kt + i) / kVSlots) & 1u, a.err,
-                         abort_flag, WHERE_ATTN_MMA)) {
+              !mbar_wait(&v_ready[vs], (uint32_t)((kt + i) / kVSlots) & 1u, a.err, abort_flag,
+                         WHERE_ATTN_MMA)) {
             ok = false;
             break;
           }
@@ -518,23 +497,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int ksteps = (tile_info(sa + i, ui.L, a.S).nvalid + 15) >> 4;
           if (lane == 0) {
             // V as an MN-major operand: 64-wide dh blocks kKVSub apart, 8-key
-            // groups 1 KB apart, 16 keys (2 KB) per MMA; P of keys
-            // 16kk..16kk+15 in columns 8kk..8kk+7.
-            const int vs = (kt + i) % kVSlots;
+            // groups 1 KB apart, 16 keys (2 KB) per MMA.  P of keys 0..63
+            // sits in columns 0..31, of keys 64..127 in columns 64..95.
             const uint64_t dV = dV0 + (uint64_t)((uint32_t)(vs * nsub) * (kKVSub >> 4));
 #pragma unroll
             for (int kk = 0; kk < kAttnBN / 16; ++kk) {
               if (kk < ksteps)
-                umma_bf16_ts(tOh, tS + kk * 8, dV + (uint64_t)(kk * (2048 >> 4)), idO,
-                             (i > 0 || kk > 0) ? 1u : 0u);
+                umma_bf16_ts(tOh, tS + kk * 8 + (kk >= 4 ? 32 : 0),
+                             dV + (uint64_t)(kk * (2048 >> 4)), idO, (i > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(&v_empty[vs]);
           }
           __syncwarp();
-          if (i + 1 < n) {
-            ok = scores(kt + i + 1);
-            if (ok && i + 2 == n && lane == 0) umma_commit(q_empty);
-          }
+          if (i + 1 < n) ok = scores(i + 1);
         }
         if (ok && lane == 0) umma_commit(&o_full[h]);
         __syncwarp();
@@ -544,116 +519,158 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
   } else {
     // ---------------------------------------------------- softmax groups
-    // Half wg is served by warps 4+4*wg .. 7+4*wg; warp w owns the rows of
-    // its TMEM lane quarter q = w % 4, one row per thread, all 128 key
-    // columns of every tile.
-    const int wg = (warp - 4) >> 2;
+    // Half wg is served by warps 4+8*wg .. 11+8*wg.  Warp w owns the rows of
+    // its TMEM lane quarter q = w % 4 and one column half ch of every tile
+    // (S columns ch*64..+63, the O columns ch*dh/2..+dh/2-1), so two warps
+    // per SMSP share a row: they swap their partial row maxima through
+    // shared memory (as bf16, rounded the same way on both sides, so both
+    // use the identical stabiliser) and add their row sums at the end of
+    // each segment.
+    const int wg = (warp - 4) >> 3;
+    const int ch = ((warp - 4) >> 2) & 1;
     const int q = warp & 3;
     const int r = q * 32 + lane;
     if (wg < halves) {
       const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-      const uint32_t tS = tmem + wg * kAttnBN + lane_off;
-      const uint32_t tO = tmem + tO0 + wg * dh + lane_off;
+      const uint32_t tS = tmem + wg * kAttnBN + lane_off + ch * 64;
+      const int dh2 = dh / 2;
+      const uint32_t tO = tmem + tO0 + wg * dh + lane_off + ch * dh2;
+      uint16_t* xch = reinterpret_cast<uint16_t*>(base + SL.xchg) + (wg * 4 + q) * 64;
+      uint64_t* xb = &xbar[wg * 4 + q];
       const float c = a.scale_log2;
-      int pt = 0, qi = 0;
+      int pt = 0, qi = 0, xp = 0;  // turns, segments, exchanges
       bool ok = true;
+      // The row's partial max of this warp's 64 columns -> the row max
+      // (both column halves, rounded to bf16 the same way on both sides).
+      auto exchange = [&](float part, float& mx) -> bool {
+        xch[ch * 32 + lane] = bf16_bits(part);
+        mbar_arrive(xb);
+        if (!mbar_wait(xb, (uint32_t)xp & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) return false;
+        ++xp;
+        mx = fmaxf(bf16_value(xch[lane]), bf16_value(xch[32 + lane]));
+        return true;
+      };
+      // P = exp2(S*c - m) as bf16 pairs over this warp's own S columns: four
+      // 16-column sub-slices, the next one's load in flight while this
+      // one's exponentials run; P of sub-slice k goes to columns [8k, 8k+8),
+      // which sub-slices already read cover.  One pair in eight on the FMA
+      // pipe.
+      auto exps = [&](float m) -> float {
+        float s0 = 0.f, s1 = 0.f;
+        uint32_t s_even[16], s_odd[16];  // sub-slices 0, 2 and 1, 3
+        tmem_ld16(tS, s_even);
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int k = 0; k < 4; k += 2) {
+          tmem_ld16(tS + 16 * (k + 1), s_odd);
+          exp_slice16(s_even, c, m, s0, s1);
+          tmem_st8_even(tS + 8 * k, s_even);
+          tmem_wait_ld();
+          if (k == 0) tmem_ld16(tS + 32, s_even);
+          exp_slice16(s_odd, c, m, s0, s1);
+          tmem_st8_even(tS + 8 * (k + 1), s_odd);
+          if (k == 0) tmem_wait_ld();
+        }
+        return s0 + s1;
+      };
+      // O_h to a new max before P_h(i).V adds to it (s_full also covered
+      // P_h(i-1).V, so O_h is settled).
+      auto rescale_o = [&](float alpha) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < dh2; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(tO + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st16(tO + c0, o);
+        }
+      };
       while (ok && walk.next(su, sa, sb)) {
-        const UnitInfo ui = unit_info(a, su);
+        const int Lu = unit_len(a, (su / a.n_qtiles) / a.Hkv);
         float m = -INFINITY, l = 0.f;
         for (int i = sa; i < sb; ++i, ++pt) {
           // The two halves take turns (0 on tile t, then 1 on tile t, then 0
           // on t+1): the tensor core runs one half's P.V and next S while
-          // the other half's softmax runs.  p_full[other] marks the other
-          // half's turn done.
+          // the other half's softmax runs, instead of both halves contending
+          // for MUFU and then both waiting for their MMAs.  p_full[other]
+          // marks the other half's turn done.
           if (halves == 2 && (wg == 1 || pt > 0) &&
               !mbar_wait(&p_full[wg ^ 1], (uint32_t)(wg == 1 ? pt : pt - 1) & 1u, a.err,
                          abort_flag, WHERE_ATTN_SOFTMAX)) {
             ok = false;
             break;
           }
-          if (!mbar_wait(&s_full[wg], (uint32_t)pt & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
+          if (!mbar_wait(&s_full[wg], (uint32_t)pt & 1u, a.err, abort_flag,
+                         WHERE_ATTN_SOFTMAX)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nv = tile_info(i, ui.L, a.S).nvalid;
-          // The row of S: up to four 32-key chunks (only those holding valid
-          // keys), one TMEM read.  Keys past nv become -inf.
-          uint32_t s0[32], s1[32], s2[32], s3[32];
-          tmem_ld32(tS, s0);
-          if (nv > 32) tmem_ld32(tS + 32, s1);
-          if (nv > 64) tmem_ld32(tS + 64, s2);
-          if (nv > 96) tmem_ld32(tS + 96, s3);
-          tmem_wait_ld();
-          float mt;
-          if (nv >= kAttnBN) {
-            mt = fmaxf(max32(s0, -INFINITY), max32(s1, -INFINITY));
-            mt = fmaxf(mt, fmaxf(max32(s2, -INFINITY), max32(s3, -INFINITY)));
-          } else {
-            mask32(s0, 0, nv);
-            mt = max32(s0, -INFINITY);
-            if (nv > 32) {
-              mask32(s1, 32, nv);
-              mt = max32(s1, mt);
-            }
-            if (nv > 64) {
-              mask32(s2, 64, nv);
-              mt = max32(s2, mt);
-            }
-            if (nv > 96) {
-              mask32(s3, 96, nv);
-              mt = max32(s3, mt);
-            }
-          }
-          const float mxs = mt * c;
-          const bool need = mxs > m + kRescaleThreshold;
-          float alpha = 1.f;
-          if (need) {
-            alpha = ex2(m - mxs);
-            m = mxs;
-          }
-          l *= alpha;
-          // P = exp2(S*c - m) as bf16 pairs over the chunk's own first 16
-          // columns' worth: chunk k's 16 pair columns go to columns 16k..,
-          // all of which were read above.
-          float sa0 = 0.f, sa1 = 0.f;
-          exp_chunk32(s0, c, m, sa0, sa1);
-          tmem_st16_even(tS, s0);
-          if (nv > 32) {
-            exp_chunk32(s1, c, m, sa0, sa1);
-            tmem_st16_even(tS + 16, s1);
-          }
-          if (nv > 64) {
-            exp_chunk32(s2, c, m, sa0, sa1);
-            tmem_st16_even(tS + 32, s2);
-          }
-          if (nv > 96) {
-            exp_chunk32(s3, c, m, sa0, sa1);
-            tmem_st16_even(tS + 48, s3);
-          }
-          l += sa0 + sa1;
-          // O_h to the new max before P_h(i).V adds to it (s_full also
-          // covered P_h(i-1).V, so O_h is settled).  A segment's first P.V
-          // overwrites O, so its first tile needs none.
-          if (i > sa && __any_sync(0xffffffffu, need)) {
+          const int nvt = tile_info(i, Lu, a.S).nvalid;
+          {
+            // Columns past the valid keys (the block's own tile, or the last
+            // tile of a unit) are overwritten with -inf (nothing to the max,
+            // exp2 gives 0 on both exponential paths), then the row max, then
+            // the exponentials.
+            const int nv = nvt - ch * 64;
+            if (nv < 64) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < dh; c0 += 16) {
-              uint32_t o[16];
-              tmem_ld16(tO + c0, o);
+              for (int c0 = max(nv, 0) & ~15; c0 < 64; c0 += 16) {
+                uint32_t v[16];
+                if (c0 < nv) {
+                  tmem_ld16(tS + c0, v);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) v[j] = c0 + j < nv ? v[j] : __float_as_uint(-INFINITY);
+                } else {
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) v[j] = __float_as_uint(-INFINITY);
+                }
+                tmem_st16(tS + c0, v);
+              }
+              tmem_wait_st();
+            }
+            float mc[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mc[k] = -INFINITY;
+            uint32_t sa32[32];
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 32) {
+              tmem_ld32(tS + c0, sa32);
               tmem_wait_ld();
 #pragma unroll
-              for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-              tmem_st16(tO + c0, o);
+              for (int j = 0; j < 32; j += 2)
+                mc[(j >> 1) & 3] =
+                    fmax3(mc[(j >> 1) & 3], __uint_as_float(sa32[j]), __uint_as_float(sa32[j + 1]));
             }
+            float mx;
+            if (!exchange(fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]), mx)) {
+              ok = false;
+              break;
+            }
+            const float mxs = mx * c;
+            const bool need = mxs > m + kRescaleThreshold;
+            float alpha = 1.f;
+            if (need) {
+              alpha = ex2(m - mxs);
+              m = mxs;
+            }
+            l = l * alpha + exps(m);
+            // a segment's first P.V overwrites O, so its first tile needs none
+            if (i > sa && __any_sync(0xffffffffu, need)) rescale_o(alpha);
           }
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(&p_full[wg]);
         }
         if (!ok) break;
-        // The segment's partial: unnormalised O (tile-major [slot][dh/4][256
-        // rows][4], so a warp's float4 store covers 32 consecutive rows, 512
-        // contiguous bytes), the running max (log2 units) and the row sum.
+        // The segment's partial, each column half writing its own: its half
+        // of the unnormalised O row (tile-major [slot][dh/4][256 rows][4],
+        // so a warp's float4 store covers 32 consecutive rows, 512
+        // contiguous bytes), the running max (log2 units, the same in both
+        // halves) and its row sum: [slot][256 rows] x (m, l of column half
+        // 0, l of column half 1, unused).
         if (!mbar_wait(&o_full[wg], (uint32_t)qi & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX)) {
           ok = false;
           break;
@@ -663,21 +680,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const bool valid = r < a.rows_per_half;
         const int r256 = wg * 128 + r;
         float* po = a.part_o + (size_t)slot * dh * 256 + (size_t)r256 * 4;
-        for (int c0 = 0; c0 < dh; c0 += 32) {
+        for (int c0 = 0; c0 < dh2; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tO + c0, o);
           tmem_wait_ld();
           if (valid) {
 #pragma unroll
             for (int v = 0; v < 8; ++v)
-              *reinterpret_cast<float4*>(po + (size_t)(c0 / 4 + v) * 1024) =
+              *reinterpret_cast<float4*>(po + (size_t)((ch * dh2 + c0) / 4 + v) * 1024) =
                   make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
                               __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
           }
         }
-        if (valid)
-          *reinterpret_cast<float2*>(a.part_ml + ((size_t)slot * 256 + r256) * 2) =
-              make_float2(m, l);
+        if (valid) {
+          float* ml = a.part_ml + ((size_t)slot * 256 + r256) * 4;
+          if (ch == 0) {
+            ml[0] = m;
+            ml[1] = l;
+          } else {
+            ml[2] = l;
+          }
+        }
         ++qi;
       }
     }
@@ -721,8 +744,12 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a) {
     for (int k = 0; k < 4; ++k) {
       const bool in = seg_ran(a, sr, c0 + k);
       const size_t slot = (size_t)u + c0 + k;
-      ml[k] = in ? *reinterpret_cast<const float2*>(a.part_ml + (slot * 256 + row256) * 2)
-                 : make_float2(-INFINITY, 0.f);
+      if (in) {
+        const float4 q4 = *reinterpret_cast<const float4*>(a.part_ml + (slot * 256 + row256) * 4);
+        ml[k] = make_float2(q4.x, q4.y + q4.z);
+      } else {
+        ml[k] = make_float2(-INFINITY, 0.f);
+      }
       o[k] = in ? *reinterpret_cast<const float4*>(a.part_o + ((slot * ngrp + grp) * 256 + row256) * 4)
                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }

@@ -91,8 +91,8 @@ cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int
 // ------------------------------------------------------------- attention
 constexpr int kAttnBN = 128;       // keys per tile
 // warp 0 TMA Q/K, warp 1 TMEM owner and TMA V + V padding, warps 2-3 MMA
-// (one per 128-row half), warps 4-7 / 8-11 softmax of half 0 / half 1
-constexpr int kAttnThreads = 384;
+// (one per 128-row half), warps 4-11 / 12-19 softmax of half 0 / half 1
+constexpr int kAttnThreads = 640;
 
 // A unit is (sequence b, KV head g, query tile qt), u = (b*Hkv + g)*n_qtiles
 // + qt.  Its keys form 1 + ceil(L_b / 128) tiles (tile 0: the block's own S
@@ -114,12 +114,15 @@ struct AttnArgs {
   int n_ctas;           // CTAs of the persistent grid
   int* tile_start;      // [units + 1] exclusive prefix sums of tiles per unit (device)
   int* first_unit;      // [n_ctas] the unit holding each CTA's first tile (device)
+  int2* unit_ctas;      // [units] first and last CTA holding a tile of the unit (device)
+  int* cta_ran;         // [n_ctas] 1 if the CTA's range holds a tile (device)
   float scale_log2;     // log2(e) / sqrt(dh)
   uint16_t* out;        // bf16 [B*S, ldo]
   int ldo;
   int kv_keep;          // 1: load K/V with evict-last (small cache re-read every step)
   float* part_o;        // [units + n_ctas - 1][dh/4][256 rows][4] unnormalised partial outputs
-  float* part_ml;       // [units + n_ctas - 1][256][2] (running max in log2 units, sum)
+  float* part_ml;       // [units + n_ctas - 1][256][4]: running max (log2 units), the row
+                        // sums of key columns 0..63 and 64..127 of every tile, unused
   int* err;
 };
 size_t attn_smem_bytes(int dh, int halves);
@@ -130,21 +133,19 @@ cudaError_t launch_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKc, const C
 cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t st);
 
 #ifdef __CUDACC__
-// The CTAs that ran unit u lie in [c_first, c_last]: c(t) = ((t+1)*n_ctas - 1)
-// / T is the CTA whose range holds tile t (the largest c with c*T/n_ctas <=
+// The CTAs that ran unit u lie in [c_first, c_last] (precomputed by the plan
+// kernel: c(t) = ((t+1)*n_ctas - 1) / T is the CTA whose range holds tile
 // t).  With fewer tiles than CTAs some CTAs in between have empty ranges and
 // wrote nothing (seg_ran tells).
 struct SegRange {
   int c_first, c_last;
-  long long T;
 };
 __device__ __forceinline__ SegRange unit_segments(const AttnArgs& a, int u) {
-  const long long T = a.tile_start[a.units], P = a.n_ctas;
-  const long long t0 = a.tile_start[u], t1 = a.tile_start[u + 1] - 1;
-  return SegRange{(int)(((t0 + 1) * P - 1) / T), (int)(((t1 + 1) * P - 1) / T), T};
+  const int2 r = a.unit_ctas[u];
+  return SegRange{r.x, r.y};
 }
 __device__ __forceinline__ bool seg_ran(const AttnArgs& a, const SegRange& r, int c) {
-  return c <= r.c_last && (long long)c * r.T / a.n_ctas < (long long)(c + 1) * r.T / a.n_ctas;
+  return c <= r.c_last && a.cta_ran[c] != 0;
 }
 #endif
 

@@ -344,7 +344,9 @@ __global__ void __launch_bounds__(kAdaThreads)
       for (int k = 0; k < kG; ++k) {
         if (sp0 + i < n_seg[k] && seg_ran(a, sr[k], sr[k].c_first + sp0 + i)) {
           const size_t slot = (size_t)unit[k] + sr[k].c_first + sp0 + i;
-          ml[i][k] = *reinterpret_cast<const float2*>(a.part_ml + (slot * 256 + r256[k]) * 2);
+          const float4 q4 =
+              *reinterpret_cast<const float4*>(a.part_ml + (slot * 256 + r256[k]) * 4);
+          ml[i][k] = make_float2(q4.x, q4.y + q4.z);
           x[i][k] = *reinterpret_cast<const float4*>(
               a.part_o + ((slot * ngrp + grp[k]) * 256 + r256[k]) * 4);
         } else {

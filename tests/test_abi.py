@@ -143,8 +143,8 @@ def test_split_knob(L):
     eight = tt.tt_workspace_bytes(d, tt.TT_WS_ATTN)
     tt.tt_set_attn_splits(0)
     # a partial slot per (unit, CTA) boundary: units + CTAs - 1 slots of 256
-    # rows x (dh + 2) floats
-    slot = 256 * (128 + 2) * 4
+    # rows x (dh + 4) floats
+    slot = 256 * (128 + 4) * 4
     assert eight - one == 7 * slot
 
 
