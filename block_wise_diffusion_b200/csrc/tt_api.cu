@@ -202,7 +202,7 @@ static tt_status check_ptr(const void* p, const char* name, bool need16) {
 
 // ------------------------------------------------------------ geometry
 struct AttnGeom {
-  int G, s_per_half, rows_per_half, halves, n_qtiles, units, n_ctas, slots;
+  int G, s_per_half, rows_per_half, halves, n_qtiles, units, n_ctas, slots, merge_cap, fixup;
   size_t part_o_bytes, part_ml_bytes;
 };
 
@@ -219,6 +219,16 @@ static AttnGeom attn_geom(const tt_dims& d) {
   const int forced = g_forced_splits.load();
   g.n_ctas = forced > 0 ? forced : num_sms();
   g.slots = g.units + g.n_ctas - 1;
+  // With at least half as many units as CTAs a unit spans about three CTAs
+  // at most and the CTA that completes it merges it cheaply (the fix-up);
+  // with fewer, units span many CTAs and one SM merging megabytes of
+  // partials would trail the kernel, so a merge over the whole GPU follows.
+  g.fixup = 2 * g.units >= g.n_ctas ? 1 : 0;
+  // A CTA completes a unit only when the unit's last tile is in its range, and
+  // every unit has a tile: at most its range's tiles, at most ceil(T / CTAs)
+  // with T <= units * (1 + ceil(L_cap / 128)).
+  const long long t_max = (long long)g.units * (1 + (d.L_cap + kAttnBN - 1) / kAttnBN);
+  g.merge_cap = (int)std::min<long long>(g.units, (t_max + g.n_ctas - 1) / g.n_ctas + 1);
   g.part_o_bytes = (size_t)g.slots * 256 * d.dh * sizeof(float);
   g.part_ml_bytes = (size_t)g.slots * 256 * 4 * sizeof(float);
   return g;
@@ -267,8 +277,10 @@ struct Ws {
   float* part_ml = nullptr;
   int* tile_start = nullptr;   // attention plan: tiles per unit, prefix sums
   int* first_unit = nullptr;   // attention plan: first unit of each CTA
-  int2* unit_ctas = nullptr;   // attention plan: first and last CTA of each unit
-  int* cta_ran = nullptr;      // attention plan: CTAs whose range holds a tile
+  int4* unit_ctas = nullptr;   // attention plan: first and last CTA of each unit, CTA count
+  int* unit_done = nullptr;    // attention fix-up: finished segments per unit
+  int* merge_list = nullptr;   // attention fix-up: units each CTA completed
+  uint16_t* attn_out = nullptr;  // loop: the attention output rows
   float4* stats = nullptr;
   float* qkv_partial = nullptr;
   uint16_t* xrows = nullptr;  // loop: one layer's modulated rows for the next layer
@@ -293,8 +305,9 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     const AttnGeom g = attn_geom(d);
     w.tile_start = c.take<int>((size_t)(g.units + 1) * sizeof(int));
     w.first_unit = c.take<int>((size_t)g.n_ctas * sizeof(int));
-    w.unit_ctas = c.take<int2>((size_t)g.units * sizeof(int2));
-    w.cta_ran = c.take<int>((size_t)g.n_ctas * sizeof(int));
+    w.unit_ctas = c.take<int4>((size_t)g.units * sizeof(int4));
+    w.unit_done = c.take<int>((size_t)g.units * sizeof(int));
+    w.merge_list = c.take<int>((size_t)g.n_ctas * g.merge_cap * sizeof(int));
     w.part_o = c.take<float>(g.part_o_bytes);
     w.part_ml = c.take<float>(g.part_ml_bytes);
   }
@@ -310,6 +323,7 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     w.egath = c.take<uint16_t>(rows * d.H * 2);
     w.xrows = c.take<uint16_t>(rows * d.H * 2);
     w.qkv = c.take<uint16_t>(rows * n_qkv * 2);
+    w.attn_out = c.take<uint16_t>(rows * d.H * 2);
     // tile-major partials: ks planes of whole 128 x kQkvBN tiles, for the
     // linear update or the context projection, whichever needs more
     const size_t pb = std::max(splitk_bytes(d, (int)n_qkv, qkv_ksplit(d)),
@@ -376,7 +390,10 @@ static AttnArgs attn_args(const tt_dims& d, const AttnGeom& g, const int32_t* ct
   a.tile_start = w.tile_start;
   a.first_unit = w.first_unit;
   a.unit_ctas = w.unit_ctas;
-  a.cta_ran = w.cta_ran;
+  a.unit_done = w.unit_done;
+  a.fixup = g.fixup;
+  a.merge_list = w.merge_list;
+  a.merge_cap = g.merge_cap;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)d.dh));
   a.out = out;
   a.ldo = d.H;
@@ -400,14 +417,15 @@ static tt_status run_attn_plan(const tt_dims& d, const AttnGeom& g, const int32_
   return TT_OK;
 }
 
-// The attention launch; with `merge` the segment partials are combined into
-// `out` by the merge kernel (the loop fuses that merge into adaLN instead).
+// The attention launch.  With the fix-up the kernel writes the bf16 output
+// to `out`; otherwise, with `merge`, a merge kernel does (the loop fuses that
+// merge into adaLN instead).
 static tt_status run_attn(const tt_dims& d, const AttnGeom& g, const AttnMaps& m,
                           const int32_t* ctx_len, tt_bf16* out, const Ws& w, const int* active,
                           bool merge, cudaStream_t st) {
   const AttnArgs a = attn_args(d, g, ctx_len, out, w, active);
   TT_LAUNCH(TT_K_ATTN, st, launch_attn(m.q, m.kc, m.vc, m.kb, m.vb, a, st));
-  if (merge) TT_LAUNCH(TT_K_MERGE, st, launch_attn_merge(a, st));
+  if (merge && !g.fixup) TT_LAUNCH(TT_K_MERGE, st, launch_attn_merge(a, st));
   return TT_OK;
 }
 
@@ -622,7 +640,8 @@ tt_status tt_adaln_modulate(const tt_dims* d, const tt_bf16* x, const tt_bf16* s
   TT_CHECK(check_ws(*d, TT_WS_ADALN, ws, ws_bytes, &w));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   TT_CUDA(cudaMemsetAsync(w.ctrl, 0, kCtrlBytes, st));
-  TT_LAUNCH(TT_K_ADALN, st, launch_adaln(x, shift_scale, t, y, d->B * d->S, d->S, d->H, st));
+  TT_LAUNCH(TT_K_ADALN, st, launch_adaln(x, shift_scale, t, y, d->B * d->S, d->S, d->H, nullptr,
+                                         nullptr, nullptr, nullptr, st));
   return TT_OK;
 }
 
@@ -730,14 +749,19 @@ static tt_status denoise_block_loop_impl(
       if (ga.ksplit > 1)
         TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
                                                           w.qkv, n_qkv, active, st));
-      TT_CHECK(run_attn(*d, g, maps[l], ctx_len, nullptr, w, active, false, st));
+      TT_CHECK(run_attn(*d, g, maps[l], ctx_len, w.attn_out, w, active, false, st));
       // The last layer keeps the masked rows, compacted, for the vocabulary;
       // earlier layers modulate every row (all positions are keys of the
       // next layer).  A null row list selects the latter.
       uint16_t* y = last ? w.y_c : w.xrows;
       int* rl = last ? w.rowlist : nullptr;
-      const AttnArgs aa = attn_args(*d, g, ctx_len, nullptr, w, active);
-      TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, ss, y, masked, rl, w.ctrl, st));
+      if (g.fixup) {
+        TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, ss, nullptr, y, rows, d->S, d->H,
+                                               masked, rl, w.ctrl, active, st));
+      } else {
+        const AttnArgs aa = attn_args(*d, g, ctx_len, w.attn_out, w, active);
+        TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, ss, y, masked, rl, w.ctrl, st));
+      }
     }
     TT_CHECK(run_vocab_gemm(*d, w, W, logit_scale, w.ctrl + CTRL_M, active, w_keep_tiles, st));
     CommitArgs c = commit_args(*d, w, gamma, logit_scale, tokens, masked);

@@ -15,7 +15,8 @@
 // persistent grid (one CTA per SM), so every SM streams the same number of
 // K/V tiles whatever the batch and the lengths.  A CTA walks its range as
 // segments, one per unit it touches, and writes per segment the unnormalised
-// O and the row maxima and sums; a merge combines a unit's segments.
+// O and the row maxima and sums; the CTA that completes a unit (a per-unit
+// counter) merges the unit's segments into the bf16 output.
 //
 // Inside a CTA the unit's rows form two 128-row halves, each an M=128
 // tcgen05 tile with its own TMEM columns.  Per 128-key tile i and half h:
@@ -55,6 +56,13 @@ constexpr int kKSlots = 3, kVSlots = 2;       // K and V ring depths
 constexpr uint32_t kKVSub = kAttnBN * 128;    // 128 keys x 64 dh bf16 (128-byte rows) = 16 KB
 constexpr uint32_t kQSub = 16384;             // 128 rows x 64 dh bf16
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
+// Context K/V tiles this far ahead of the one being loaded into shared
+// memory are prefetched into L2 (0: none), so that more of the stream is in
+// flight than the rings hold.
+#ifndef TT_ATTN_L2_AHEAD
+#define TT_ATTN_L2_AHEAD 0
+#endif
+constexpr int kL2Ahead = TT_ATTN_L2_AHEAD;
 
 struct AttnSmem {
   uint32_t q, k, v, bars, xchg, total;
@@ -161,6 +169,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+__device__ __forceinline__ float max16(const uint32_t (&v)[16]) {
+  float a = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+  float b = fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
+  a = fmax3(a, __uint_as_float(v[6]), __uint_as_float(v[7]));
+  b = fmax3(b, __uint_as_float(v[8]), __uint_as_float(v[9]));
+  a = fmax3(a, __uint_as_float(v[10]), __uint_as_float(v[11]));
+  b = fmax3(b, __uint_as_float(v[12]), __uint_as_float(v[13]));
+  return fmax3(fmaxf(a, b), __uint_as_float(v[14]), __uint_as_float(v[15]));
+}
+
 // P for 16 score columns as 8 bf16 pairs, written in place: pair j/2 goes to
 // sv[j] (the registers of S it came from are dead by then); the last pair
 // on the FMA pipe.
@@ -239,11 +257,13 @@ __global__ void __launch_bounds__(1024) attn_plan_kernel(const AttnArgs a) {
     const long long s0 = start[u], s1 = start[u + 1];
     const long long c0 = (s0 * P + T - 1) / T, c1 = (s1 * P + T - 1) / T;
     for (long long c = c0; c < c1 && c < P; ++c) a.first_unit[c] = u;
-    // the merges' view: the CTAs holding the unit's first and last tiles
-    a.unit_ctas[u] = make_int2((int)(((s0 + 1) * P - 1) / T), (int)((s1 * P - 1) / T));
+    // the fix-up's view: the CTAs holding the unit's first and last tiles,
+    // and how many CTAs hold a tile of it (with fewer tiles than CTAs every
+    // non-empty CTA holds one tile)
+    const int cf = (int)(((s0 + 1) * P - 1) / T), cl = (int)((s1 * P - 1) / T);
+    a.unit_ctas[u] = make_int4(cf, cl, T >= P ? cl - cf + 1 : (int)(s1 - s0), T >= P ? 1 : 0);
+    a.unit_done[u] = 0;
   }
-  for (int c = tid; c < a.n_ctas; c += blockDim.x)
-    a.cta_ran[c] = (long long)c * T / P < (long long)(c + 1) * T / P ? 1 : 0;
 }
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -258,8 +278,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const long long T = a.tile_start[a.units];
   const int lo = (int)((long long)cta * T / a.n_ctas);
   const int hi = (int)((long long)(cta + 1) * T / a.n_ctas);
-  if (lo >= hi) return;
   const int u0 = a.first_unit[cta];
+  if (lo >= hi) {
+    // An empty range (fewer tiles than CTAs) lies inside the CTA range of at
+    // most one unit, the one holding tile lo, and only when that unit starts
+    // before lo: its slot gets an empty record (no keys, sum 0), so the
+    // merges can take every CTA of a unit's range as present.
+    if (!a.fixup && a.tile_start[u0] < lo)
+      for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        *reinterpret_cast<float4*>(a.part_ml + ((size_t)(u0 + cta) * 256 + i) * 4) =
+            make_float4(-INFINITY, 0.f, 0.f, 0.f);
+    return;
+  }
   const int dh = a.dh, nsub = dh / 64;
   const int halves = a.halves;
 
@@ -280,8 +310,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint64_t* p_full = s_full + 2;         // [half]: P_h(i) written, O_h corrected
   uint64_t* o_full = p_full + 2;         // [half]: the segment's last P.V done
   uint64_t* xbar = o_full + 2;           // [half][quarter]: both column halves' values written
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xbar + 8);
+  uint64_t* seg_done = xbar + 8;         // every softmax thread has written its partial
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(seg_done + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  int* n_merge = abort_flag + 1;         // units this CTA completed (merged at the end)
+  int* merge_list = a.merge_list + (size_t)cta * a.merge_cap;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // TMEM: S/P of half h at column h*128, then O of half h at halves*128 + h*dh.
@@ -316,7 +349,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&o_full[h], 1);
     }
     for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 64);
+    mbar_init(seg_done, halves * 256);
     *abort_flag = 0;
+    *n_merge = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -336,6 +371,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmKc);
       prefetch_tmap(&tmKb);
+      if (kL2Ahead > 0) prefetch_tmap(&tmVc);
       const uint64_t pol_kv = a.kv_keep ? policy_evict_last() : policy_evict_first();
       int kt = 0, qi = 0;
       bool ok = true;
@@ -362,6 +398,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          WHERE_ATTN_PRODUCER)) {
             ok = false;
             break;
+          }
+          if (kL2Ahead > 0 && tl + kL2Ahead < sb) {
+            const TileInfo ta = tile_info(tl + kL2Ahead, ui.L, a.S);
+            for (int xh = 0; xh < nsub; ++xh) {
+              tma_prefetch_l2_2d(&tmKc, xh * 64, row_base + ta.key0);
+              tma_prefetch_l2_2d(&tmVc, xh * 64, row_base + ta.key0);
+            }
           }
           uint8_t* dk = sK + ks * nsub * kKVSub;
           mbar_arrive_expect_tx(&k_full[ks], bytes);
@@ -538,7 +581,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint16_t* xch = reinterpret_cast<uint16_t*>(base + SL.xchg) + (wg * 4 + q) * 64;
       uint64_t* xb = &xbar[wg * 4 + q];
       const float c = a.scale_log2;
-      int pt = 0, qi = 0, xp = 0;  // turns, segments, exchanges
+      int pt = 0, qi = 0, xp = 0, sdp = 0;  // turns, segments, exchanges, fix-ups
       bool ok = true;
       // The row's partial max of this warp's 64 columns -> the row max
       // (both column halves, rounded to bf16 the same way on both sides).
@@ -549,29 +592,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         ++xp;
         mx = fmaxf(bf16_value(xch[lane]), bf16_value(xch[32 + lane]));
         return true;
-      };
-      // P = exp2(S*c - m) as bf16 pairs over this warp's own S columns: four
-      // 16-column sub-slices, the next one's load in flight while this
-      // one's exponentials run; P of sub-slice k goes to columns [8k, 8k+8),
-      // which sub-slices already read cover.  One pair in eight on the FMA
-      // pipe.
-      auto exps = [&](float m) -> float {
-        float s0 = 0.f, s1 = 0.f;
-        uint32_t s_even[16], s_odd[16];  // sub-slices 0, 2 and 1, 3
-        tmem_ld16(tS, s_even);
-        tmem_wait_ld();
-#pragma unroll 1
-        for (int k = 0; k < 4; k += 2) {
-          tmem_ld16(tS + 16 * (k + 1), s_odd);
-          exp_slice16(s_even, c, m, s0, s1);
-          tmem_st8_even(tS + 8 * k, s_even);
-          tmem_wait_ld();
-          if (k == 0) tmem_ld16(tS + 32, s_even);
-          exp_slice16(s_odd, c, m, s0, s1);
-          tmem_st8_even(tS + 8 * (k + 1), s_odd);
-          if (k == 0) tmem_wait_ld();
-        }
-        return s0 + s1;
       };
       // O_h to a new max before P_h(i).V adds to it (s_full also covered
       // P_h(i-1).V, so O_h is settled).
@@ -644,8 +664,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 mc[(j >> 1) & 3] =
                     fmax3(mc[(j >> 1) & 3], __uint_as_float(sa32[j]), __uint_as_float(sa32[j + 1]));
             }
+            uint32_t s_even[16], s_odd[16];
+            tmem_ld16(tS, s_even);  // the first sub-slice is read while the maxima are swapped
             float mx;
             if (!exchange(fmaxf(fmax3(mc[0], mc[1], mc[2]), mc[3]), mx)) {
+              tmem_wait_ld();
               ok = false;
               break;
             }
@@ -656,7 +679,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               alpha = ex2(m - mxs);
               m = mxs;
             }
-            l = l * alpha + exps(m);
+            float e0 = 0.f, e1 = 0.f;
+            tmem_wait_ld();
+#pragma unroll 1
+            for (int k = 0; k < 4; k += 2) {
+              tmem_ld16(tS + 16 * (k + 1), s_odd);
+              exp_slice16(s_even, c, m, e0, e1);
+              tmem_st8_even(tS + 8 * k, s_even);
+              tmem_wait_ld();
+              if (k == 0) tmem_ld16(tS + 32, s_even);
+              exp_slice16(s_odd, c, m, e0, e1);
+              tmem_st8_even(tS + 8 * (k + 1), s_odd);
+              if (k == 0) tmem_wait_ld();
+            }
+            l = l * alpha + (e0 + e1);
             // a segment's first P.V overwrites O, so its first tile needs none
             if (i > sa && __any_sync(0xffffffffu, need)) rescale_o(alpha);
           }
@@ -702,6 +738,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         ++qi;
+        // With the fix-up, the CTA that completes a unit (the last of its
+        // segments to finish, by a per-unit counter) merges it once its
+        // whole range is done.
+        if (!a.fixup) continue;
+        __threadfence();
+        mbar_arrive(seg_done);
+        if (warp == 4 && lane == 0 &&
+            mbar_wait(seg_done, (uint32_t)sdp & 1u, a.err, abort_flag, WHERE_ATTN_SOFTMAX) &&
+            atomicAdd(a.unit_done + su, 1) == a.unit_ctas[su].z - 1) {
+          a.unit_done[su] = 0;  // ready for the next launch
+          merge_list[(*n_merge)++] = su;  // at most merge_cap: a unit's last tile is in range
+        }
+        ++sdp;
       }
     }
   }
@@ -711,6 +760,91 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, tmem_cols);
+  }
+  // Fix-up of the units this CTA completed: all threads, item = (query row,
+  // 16-column chunk) with consecutive threads on consecutive rows (so the
+  // tile-major partial reads are coalesced), o = sum_i 2^(m_i - m*) O_i /
+  // sum_i 2^(m_i - m*) l_i over the unit's segments, two segments' loads in
+  // flight, bf16 output.
+  if (!a.fixup || *n_merge == 0 || *abort_flag) return;
+  __threadfence();
+  // With fewer tiles than CTAs (unit_ctas.w == 0) some CTAs of a unit's range
+  // held no tile and wrote nothing.
+  auto ran = [&](const int4& uc, int c) {
+    return uc.w != 0 || (long long)c * T / a.n_ctas < (long long)(c + 1) * T / a.n_ctas;
+  };
+  const int nrows = halves * 128, items = nrows * (dh / 16);
+  for (int mi = 0; mi < *n_merge; ++mi) {
+    const int u = merge_list[mi];
+    const int4 uc = a.unit_ctas[u];
+    const UnitInfo ui = unit_info(a, u);
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+      const int r256 = it % nrows, c16 = (it / nrows) * 16;
+      const int wg = r256 >> 7, r = r256 & 127;
+      if (r >= a.rows_per_half) continue;
+      float mrun = -INFINITY, den = 0.f;
+      for (int cc = uc.x; cc <= uc.y; ++cc) {
+        if (!ran(uc, cc)) continue;
+        const float4 q4 = __ldcg(
+            reinterpret_cast<const float4*>(a.part_ml + ((size_t)(u + cc) * 256 + r256) * 4));
+        const float li = q4.y + q4.z;
+        if (!(li > 0.f)) continue;
+        if (q4.x > mrun) {
+          den = mrun == -INFINITY ? 0.f : den * ex2(mrun - q4.x);
+          mrun = q4.x;
+        }
+        den += li * ex2(q4.x - mrun);
+      }
+      float acc[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+      for (int cc = uc.x; cc <= uc.y; cc += 2) {
+        float4 o4[2][4];
+        float w[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int c = cc + k;
+          w[k] = 0.f;
+          if (c <= uc.y && ran(uc, c)) {
+            const size_t sl = (size_t)(u + c);
+            const float msl = __ldcg(a.part_ml + (sl * 256 + r256) * 4);
+            w[k] = msl > -INFINITY ? ex2(msl - mrun) : 0.f;
+            const float* pos = a.part_o + sl * dh * 256 + (size_t)r256 * 4;
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              o4[k][v] = __ldcg(reinterpret_cast<const float4*>(pos + (size_t)(c16 / 4 + v) * 1024));
+          } else {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) o4[k][v] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            acc[4 * v] += w[k] * o4[k][v].x;
+            acc[4 * v + 1] += w[k] * o4[k][v].y;
+            acc[4 * v + 2] += w[k] * o4[k][v].z;
+            acc[4 * v + 3] += w[k] * o4[k][v].w;
+          }
+        }
+      }
+      const float inv = 1.f / den;
+      const int s = ui.qt * halves * a.s_per_half + wg * a.s_per_half + r / a.G;
+      const int head = ui.g * a.G + r % a.G;
+      uint16_t* dst = a.out + (size_t)(ui.b * a.S + s) * a.ldo + head * dh + c16;
+      uint4 w0, w1;
+      w0.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      w0.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+      w0.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+      w0.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+      w1.x = pack_bf16x2(acc[8] * inv, acc[9] * inv);
+      w1.y = pack_bf16x2(acc[10] * inv, acc[11] * inv);
+      w1.z = pack_bf16x2(acc[12] * inv, acc[13] * inv);
+      w1.w = pack_bf16x2(acc[14] * inv, acc[15] * inv);
+      reinterpret_cast<uint4*>(dst)[0] = w0;
+      reinterpret_cast<uint4*>(dst)[1] = w1;
+    }
   }
 }
 
@@ -734,15 +868,15 @@ __global__ void __launch_bounds__(256) attn_merge_kernel(const AttnArgs a) {
   if (h >= a.halves || r >= a.rows_per_half) return;
   const int qt = u % a.n_qtiles, pair = u / a.n_qtiles;
   const int b = pair / a.Hkv, g = pair % a.Hkv;
-  const SegRange sr = unit_segments(a, u);
+  const int4 uc = a.unit_ctas[u];
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f, mrun = -INFINITY;
-  for (int c0 = sr.c_first; c0 <= sr.c_last; c0 += 4) {
+  for (int c0 = uc.x; c0 <= uc.y; c0 += 4) {
     float2 ml[4];
     float4 o[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const bool in = seg_ran(a, sr, c0 + k);
+      const bool in = c0 + k <= uc.y;
       const size_t slot = (size_t)u + c0 + k;
       if (in) {
         const float4 q4 = *reinterpret_cast<const float4*>(a.part_ml + (slot * 256 + row256) * 4);

@@ -114,8 +114,14 @@ struct AttnArgs {
   int n_ctas;           // CTAs of the persistent grid
   int* tile_start;      // [units + 1] exclusive prefix sums of tiles per unit (device)
   int* first_unit;      // [n_ctas] the unit holding each CTA's first tile (device)
-  int2* unit_ctas;      // [units] first and last CTA holding a tile of the unit (device)
-  int* cta_ran;         // [n_ctas] 1 if the CTA's range holds a tile (device)
+  int4* unit_ctas;      // [units] first and last CTA of the unit's range, how many CTAs
+                        // hold a tile of it, and 1 if every CTA in the range does (device)
+  int* unit_done;       // [units] segments of the unit finished so far (device; the plan
+                        // kernel zeroes it, the CTA that completes a unit resets it)
+  int fixup;            // 1: the CTA that completes a unit merges it into `out` (units
+                        // span few CTAs); 0: partials only, merged by a separate kernel
+  int* merge_list;      // [n_ctas][merge_cap] units each CTA completed (device)
+  int merge_cap;        // >= the units any CTA can complete: min(units, ceil(T_max / n_ctas) + 1)
   float scale_log2;     // log2(e) / sqrt(dh)
   uint16_t* out;        // bf16 [B*S, ldo]
   int ldo;
@@ -130,24 +136,9 @@ cudaError_t launch_attn_plan(const AttnArgs& a, cudaStream_t st);
 cudaError_t launch_attn(const CUtensorMap& tmQ, const CUtensorMap& tmKc, const CUtensorMap& tmVc,
                         const CUtensorMap& tmKb, const CUtensorMap& tmVb, const AttnArgs& a,
                         cudaStream_t st);
+// Without the fix-up: every unit's segment partials merged into `out`.
 cudaError_t launch_attn_merge(const AttnArgs& a, cudaStream_t st);
 
-#ifdef __CUDACC__
-// The CTAs that ran unit u lie in [c_first, c_last] (precomputed by the plan
-// kernel: c(t) = ((t+1)*n_ctas - 1) / T is the CTA whose range holds tile
-// t).  With fewer tiles than CTAs some CTAs in between have empty ranges and
-// wrote nothing (seg_ran tells).
-struct SegRange {
-  int c_first, c_last;
-};
-__device__ __forceinline__ SegRange unit_segments(const AttnArgs& a, int u) {
-  const int2 r = a.unit_ctas[u];
-  return SegRange{r.x, r.y};
-}
-__device__ __forceinline__ bool seg_ran(const AttnArgs& a, const SegRange& r, int c) {
-  return c <= r.c_last && a.cta_ran[c] != 0;
-}
-#endif
 
 // ------------------------------------------------------ small kernels
 struct PlanArgs {
@@ -161,14 +152,17 @@ struct PlanArgs {
 };
 cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st);
 
-// adaLN of every row, t[b] per sequence.
+// masked == nullptr: every row, t[b] per sequence from `t`.  Otherwise (block
+// loop) t_b = masked count / S computed in the kernel, and with a row list
+// only the masked rows, written compacted (writes rowlist[j] and
+// ctrl[CTRL_M]); with rowlist == nullptr every row at its own index (a
+// denoiser layer before the last).
 cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
-                         uint16_t* y, int rows, int S, int H, cudaStream_t st);
+                         uint16_t* y, int rows, int S, int H, const uint8_t* masked,
+                         int* rowlist, int* ctrl, const int* active, cudaStream_t st);
 
-// Block loop: the attention's segment merge + adaLN.  With a row list, only
-// the masked rows, written compacted (their compact index and t_b computed in
-// the kernel; writes rowlist[j] and ctrl[CTRL_M]); with rowlist == nullptr
-// every row at its own index (a denoiser layer before the last).
+// Block loop without the attention fix-up: the segment merge fused with
+// adaLN, with the same row selection as launch_adaln's loop mode.
 cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, uint16_t* y,
                                const uint8_t* masked, int* rowlist, int* ctrl, cudaStream_t st);
 

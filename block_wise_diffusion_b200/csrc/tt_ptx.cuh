@@ -115,6 +115,12 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       "l"(m), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+// Bring a tensor-map box into L2 only (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(m), "r"(x),
+               "r"(y)
+               : "memory");
+}
 // L2 eviction policies for streamed (read-once) and reused operands.
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;

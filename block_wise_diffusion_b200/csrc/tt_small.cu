@@ -250,14 +250,25 @@ __device__ bool loop_row(const uint8_t* __restrict__ masked, int rows, int S, in
 
 __global__ void __launch_bounds__(kAdaThreads)
     adaln_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ ss,
-                 const float* __restrict__ t, uint16_t* __restrict__ y, int S, int H) {
+                 const float* __restrict__ t, uint16_t* __restrict__ y, int rows, int S, int H,
+                 const uint8_t* __restrict__ masked, int* __restrict__ rowlist, int* ctrl,
+                 const int* active) {
   griddep_launch();
   griddep_wait();
   __shared__ float red[kAdaThreads / 32];
-  const int row = blockIdx.x;
-  const float tb = t[row / S];
+  if (active != nullptr && *active == 0) return;
+  // masked == nullptr: every row, t per sequence from `t`; otherwise the block
+  // loop's rows (the masked ones compacted, or all of them for an earlier
+  // denoiser layer).
+  int j = blockIdx.x, src = blockIdx.x;
+  float tb;
+  if (masked == nullptr) {
+    tb = t[src / S];
+  } else if (!loop_row(masked, rows, S, src, rowlist, ctrl, &j, &tb)) {
+    return;
+  }
   const int nvec = H / 8;
-  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)row * H);
+  const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)src * H);
   float v[kAdaMaxVec][8];
   float s = 0.f;
 #pragma unroll
@@ -275,10 +286,17 @@ __global__ void __launch_bounds__(kAdaThreads)
       for (int e = 0; e < 8; ++e) s += v[k][e];
     }
   }
-  adaln_finish(v, s, H, tb, ss, y + (size_t)row * H, red);
+  adaln_finish(v, s, H, tb, ss, y + (size_t)j * H, red);
 }
 
-// Attention merge fused with adaLN (block loop): one CTA per block row (b, s),
+// The CTAs of a unit's range: [c_first, c_last] (one with an empty range
+// wrote an empty record for the unit).
+struct SegRange {
+  int c_first, c_last;
+};
+
+// Attention merge fused with adaLN (block loop; used when the attention's
+// units span many CTAs, see AttnArgs::fixup): one CTA per block row (b, s),
 // returning at once for a committed row unless every row is wanted.  For
 // each query head the unit's segment partials are combined,
 //   o = sum_i 2^(m_i - m*) O_i / sum_i 2^(m_i - m*) l_i,
@@ -326,7 +344,8 @@ __global__ void __launch_bounds__(kAdaThreads)
     i0[k] = head * a.dh + grp[k] * 4;
     const int g = head / a.G, jh = head % a.G;
     unit[k] = (b * a.Hkv + g) * a.n_qtiles + qt;
-    sr[k] = unit_segments(a, unit[k]);
+    const int4 uc = a.unit_ctas[unit[k]];
+    sr[k] = SegRange{uc.x, uc.y};
     n_seg[k] = gin[k] ? sr[k].c_last - sr[k].c_first + 1 : 0;
     max_seg = max(max_seg, n_seg[k]);
     r256[k] = hh * 128 + sl * a.G + jh;
@@ -342,7 +361,7 @@ __global__ void __launch_bounds__(kAdaThreads)
     for (int i = 0; i < NB; ++i) {
 #pragma unroll
       for (int k = 0; k < kG; ++k) {
-        if (sp0 + i < n_seg[k] && seg_ran(a, sr[k], sr[k].c_first + sp0 + i)) {
+        if (sp0 + i < n_seg[k]) {
           const size_t slot = (size_t)unit[k] + sr[k].c_first + sp0 + i;
           const float4 q4 =
               *reinterpret_cast<const float4*>(a.part_ml + (slot * 256 + r256[k]) * 4);
@@ -691,9 +710,11 @@ cudaError_t launch_plan(const PlanArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_adaln(const uint16_t* x, const uint16_t* shift_scale, const float* t,
-                         uint16_t* y, int rows, int S, int H, cudaStream_t st) {
+                         uint16_t* y, int rows, int S, int H, const uint8_t* masked,
+                         int* rowlist, int* ctrl, const int* active, cudaStream_t st) {
   if (rows <= 0) return cudaSuccess;
-  return launch_k(adaln_kernel, dim3(rows), dim3(kAdaThreads), 0, st, x, shift_scale, t, y, S, H);
+  return launch_k(adaln_kernel, dim3(rows), dim3(kAdaThreads), 0, st, x, shift_scale, t, y, rows,
+                  S, H, masked, rowlist, ctrl, active);
 }
 
 cudaError_t launch_merge_adaln(const AttnArgs& a, const uint16_t* shift_scale, uint16_t* y,

@@ -3,12 +3,14 @@
 The kernels cut all units' key tiles, laid end to end, into one contiguous
 range per CTA of a persistent grid; each CTA walks its range as segments (one
 per unit it touches) and stores each segment's partial at slot u + c; the
-merges find a unit's CTAs by c(t) = ((t+1)*P - 1) // T.  This restates that
-integer arithmetic (attn_plan_kernel, the SegWalk of attn_kernel,
-unit_segments) and checks it against brute force: every tile is run exactly
-once, slots are distinct and inside the partial buffers, every walk starts
-at its first tile's unit and reads no prefix sum past the end, and each
-unit's CTA range is exactly the CTAs that ran a piece of it.
+CTA that completes a unit finds its CTAs by c(t) = ((t+1)*P - 1) // T and
+merges them.  This restates that
+integer arithmetic (attn_plan_kernel and the SegWalk of attn_kernel) and
+checks it against brute force: every tile is run exactly once, slots are
+distinct and inside the partial buffers, every walk starts at its first
+tile's unit and reads no prefix sum past the end, each unit's CTA range is
+exactly the CTAs that ran a piece of it, and the count the fix-up waits for
+is the number of those CTAs.
 """
 import numpy as np
 import pytest
@@ -74,8 +76,31 @@ def check(lengths, n_qtiles, Hkv, L_cap, P):
             slots.add(slot)
             ran[u].add(c)
     assert (seen == 1).all()
+    # an empty range lies in the CTA range [cf, cl] of at most one unit: the
+    # one holding tile lo, when it starts before lo (that CTA writes an empty
+    # record at slot unit + CTA for the merges)
+    for c in range(P):
+        lo, hi = c * T // P, (c + 1) * T // P
+        if lo < hi:
+            continue
+        inside = [u for u in range(units)
+                  if ((start[u] + 1) * P - 1) // T <= c <= (start[u + 1] * P - 1) // T]
+        u0 = first[c]
+        assert inside == ([u0] if start[u0] < lo else []), (c, inside, u0)
+    # the fix-up's per-CTA list of completed units (a unit is completed by the
+    # CTA holding its last tile) never exceeds the capacity the host sizes
+    L_eff = max(L_cap, 0)
+    cap = min(units, -(-units * (1 + -(-L_eff // BN)) // P) + 1)
+    done = [0] * P
+    for u in range(units):
+        done[(start[u + 1] * P - 1) // T] += 1
+    assert max(done) <= cap, (max(done), cap)
     for u in range(units):
         assert ran[u] == unit_segments(start, T, P, u), u
+        # the fix-up's count of the CTAs holding a piece of the unit
+        s0, s1 = start[u], start[u + 1]
+        cf, cl = ((s0 + 1) * P - 1) // T, (s1 * P - 1) // T
+        assert len(ran[u]) == (cl - cf + 1 if T >= P else s1 - s0), u
 
 
 @pytest.mark.parametrize("lengths,n_qtiles,Hkv,L_cap,P", [

@@ -217,7 +217,9 @@ def compare_teacher_forced(inp, g, gamma, logit_scale, bsel=None, steps=None):
     the same trajectory) the kernel's rows are compared with the oracle's
     (relative L2 within oracle.parity.Y_REL_L2) and decisions that the
     oracle itself takes differently on the two sets of rows are excluded and
-    counted.  Returns (compared, excluded) sequence-steps."""
+    counted.  Returns the compared sequence-steps and those excluded as near
+    ties (the decisions explained by the rows' difference are reported in
+    the printed counts)."""
     S = inp["masked"].shape[1]
     g_rows = None
     if steps is not None:
@@ -243,7 +245,7 @@ def compare_teacher_forced(inp, g, gamma, logit_scale, bsel=None, steps=None):
         # summation orders (different query tiles of one sequence) the
         # last bits pick the position, so such counts can be large there.
         assert cnt["y_rel_l2_max"] <= P.Y_REL_L2, cnt
-    return cnt["seq_steps"], cnt["seq_steps_excluded"]
+    return cnt["seq_steps"], cnt["seq_steps_excluded"] - cnt.get("y_explained", 0)
 
 
 def check_invariants(d, inp, g):
