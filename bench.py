@@ -159,13 +159,22 @@ def committed_traffic(kind: str, workload: str):
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
+    """nvidia-smi sampling SM clocks, power and throttle reasons every 200 ms.
+
+    nvidia-smi's start-up (NVML initialisation) competes with kernel launches
+    for the driver for up to a second, so the sampler is started and waited
+    for (first sample seen) before the warm-up; a reader thread stamps each
+    sample with the host clock on arrival, and window(t0, t1) keeps those
+    taken during the timed region (the nearest one on each side when the
+    region is shorter than the sampling period)."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_id: str | None):
         self.proc = None
-        self.out = None
+        self.lines = []
+        self.thread = None
         if gpu_id is None:
             return
         try:
@@ -175,26 +184,49 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return
+        import threading
 
-    def stop(self):
+        def read():
+            for line in self.proc.stdout:
+                self.lines.append((time.time(), line))
+        self.thread = threading.Thread(target=read, daemon=True)
+        self.thread.start()
+
+    def wait_ready(self, timeout_s: float = 10.0):
+        t_end = time.time() + timeout_s
+        while self.proc is not None and not self.lines and time.time() < t_end:
+            time.sleep(0.05)
+
+    def stop(self, t0: float | None = None, t1: float | None = None):
         if self.proc is None:
             return None
         time.sleep(0.25)
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = []
-        for line in out.strip().splitlines():
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        stamped = []
+        for ts, line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) != 7:
                 continue
             try:
-                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+                stamped.append((ts, (float(parts[0]), float(parts[1]), float(parts[2]), parts[3:])))
             except ValueError:
                 continue
+        if t0 is not None and t1 is not None and stamped:
+            inside = [r for ts, r in stamped if t0 <= ts <= t1 + 0.05]
+            if not inside:  # region shorter than the period: the samples around it
+                before = [r for ts, r in stamped if ts < t0][-1:]
+                after = [r for ts, r in stamped if ts > t1][:1]
+                inside = before + after
+            rows = inside
+        else:
+            rows = [r for _, r in stamped]
         if not rows:
             return None
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -459,6 +491,10 @@ def run_ours(args, rank, world, local):
         masked.copy_(masked0)
         flush.zero_()
 
+    # the clock sampler runs from before the warm-up (see ClockSampler)
+    clocks = ClockSampler(gpu_uuid(torch, local))
+    clocks.wait_ready()
+
     # warm-up
     for _ in range(args.warmup):
         reset()
@@ -469,7 +505,7 @@ def run_ours(args, rank, world, local):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    clocks = ClockSampler(gpu_uuid(torch, local))
+    t_wall0 = time.time()
     launches0 = tt.tt_launch_count()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
@@ -481,10 +517,11 @@ def run_ours(args, rank, world, local):
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     gpu_launches = tt.tt_launch_count() - launches0
+    t_wall1 = time.time()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    clk = clocks.stop()
+    clk = clocks.stop(t_wall0, t_wall1)
     ms_local = sum(a.elapsed_time(b) for a, b in ev)
     assert not masked.any().item(), "block not committed"
     ms = reduce_max(ms_local, world, dev)
@@ -567,6 +604,11 @@ def run_ours(args, rank, world, local):
                      roofline_time_frac=round(t_roof / (kms / 1e3), 4))
         if kind == "attn":
             e["exp"] = exp_roof(attn_exp_per_launch(d, inp), kms / n / 1e3, n_sm, clk)
+            # the loop keeps a context cache of at most 48 MiB in L2 across
+            # its steps (evict-last), so the HBM figure then counts bytes that
+            # L2 mostly serves
+            kv_bytes = 2.0 * d.B * d.Hkv * d.L_cap * d.dh * 2
+            e["kv_l2_resident"] = bool(kv_bytes <= 48.0 * (1 << 20))
         kernels[kind] = e
     for kind in ("attn", "gemm_vocab"):
         if kind in kernels:

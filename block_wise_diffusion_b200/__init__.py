@@ -19,7 +19,7 @@ __all__ = [
     "tt_block_denoise_attn", "tt_adaln_modulate", "tt_vocab_confidence_commit",
     "tt_denoise_block_loop", "tt_denoise_block_loop_layers", "tt_decode_blocks",
     "tt_vocab_confidence_commit_noalloc", "tt_loop_last_step",
-    "tt_device_status", "tt_launch_count", "tt_set_attn_splits",
+    "tt_device_status", "tt_launch_count", "tt_set_attn_splits", "tt_set_loop_graphs",
     "tt_status_string", "tt_last_error", "EXPORTS", "tt_profile_enable", "tt_profile_read",
     "tt_selftest_timeout",
     "profile_table", "KERNEL_KINDS",
@@ -36,7 +36,8 @@ STATUS = {0: "TT_OK", 1: "TT_ERR_INVALID_ARG", 2: "TT_ERR_UNSUPPORTED", 3: "TT_E
 # Every symbol the header declares.
 EXPORTS = (
     "tt_status_string", "tt_last_error", "tt_workspace_bytes", "tt_device_status",
-    "tt_launch_count", "tt_set_attn_splits", "tt_block_denoise_attn", "tt_adaln_modulate",
+    "tt_launch_count", "tt_set_attn_splits", "tt_set_loop_graphs", "tt_block_denoise_attn",
+    "tt_adaln_modulate",
     "tt_vocab_confidence_commit", "tt_denoise_block_loop", "tt_profile_enable", "tt_profile_read",
     "tt_vocab_confidence_commit_noalloc", "tt_selftest_timeout", "tt_denoise_block_loop_layers",
     "tt_decode_blocks", "tt_loop_last_step",
@@ -81,6 +82,8 @@ def lib() -> ctypes.CDLL:
         L.tt_launch_count.argtypes = []
         L.tt_set_attn_splits.restype = ctypes.c_int
         L.tt_set_attn_splits.argtypes = [ctypes.c_int32]
+        L.tt_set_loop_graphs.restype = ctypes.c_int
+        L.tt_set_loop_graphs.argtypes = [ctypes.c_int32]
         L.tt_profile_enable.restype = ctypes.c_int
         L.tt_profile_enable.argtypes = [ctypes.c_int32]
         L.tt_profile_read.restype = ctypes.c_int
@@ -185,6 +188,10 @@ def tt_launch_count() -> int:
 
 def tt_set_attn_splits(n: int) -> None:
     _check(lib().tt_set_attn_splits(n), "tt_set_attn_splits")
+
+
+def tt_set_loop_graphs(on: int) -> None:
+    _check(lib().tt_set_loop_graphs(on), "tt_set_loop_graphs")
 
 
 def tt_profile_enable(on: bool) -> None:

@@ -18,9 +18,13 @@ namespace tt {
 
 static thread_local char g_err[512];
 static std::atomic<uint64_t> g_launches{0};
+static thread_local uint64_t t_launches = 0;  // this thread's launches (graph capture bookkeeping)
 static std::atomic<int> g_forced_splits{0};
 
-void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+void count_launch(int n) {
+  g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed);
+  t_launches += (uint64_t)n;
+}
 
 int num_sms() {
   constexpr int kMaxDev = 64;
@@ -38,6 +42,31 @@ int num_sms() {
   }
   cache[dev].store(n, std::memory_order_relaxed);
   return n;
+}
+
+// Identity of the calling thread's current CUDA context (cuCtxGetId: unique
+// for the life of the process, so a context destroyed by a device reset and
+// created again gets a new one).  False when no context is current yet or
+// the driver lacks the call.
+bool current_context_id(unsigned long long* id) {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_cur == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
 }
 
 // ----------------------------------------------------------------- profiler
@@ -407,6 +436,20 @@ static AttnArgs attn_args(const tt_dims& d, const AttnGeom& g, const int32_t* ct
   return a;
 }
 
+// In a loop whose vocabulary GEMM has one row tile (B*S <= 128 rows) the
+// GEMM streams W from HBM while the kernels before it leave HBM mostly idle
+// when the context sits in L2.  The attention then prefetches into L2 the
+// first kVocabPrefetchBytes of every W row of the GEMM's first wave (CTA c
+// of the GEMM starts on the W tile c), a balanced head start of 34 MB at
+// V = 131072, H = 4096.
+#ifndef TT_VOCAB_PF_BYTES
+#define TT_VOCAB_PF_BYTES 1024
+#endif
+constexpr int kVocabPrefetchBytes = TT_VOCAB_PF_BYTES;
+static bool vocab_prefetch(const tt_dims& d, const AttnArgs& a) {
+  return a.kv_keep && d.B * d.S <= kGemmBM && (double)d.V * d.H * 2 >= 64.0 * (1 << 20);
+}
+
 // The attention's tile plan (prefix sums of tiles per unit from the device
 // context lengths, first unit of each CTA): once per call, since ctx_len does
 // not change within one.
@@ -420,10 +463,18 @@ static tt_status run_attn_plan(const tt_dims& d, const AttnGeom& g, const int32_
 // The attention launch.  With the fix-up the kernel writes the bf16 output
 // to `out`; otherwise, with `merge`, a merge kernel does (the loop fuses that
 // merge into adaLN instead).
+// `pf_w` (optional): the W the next vocabulary GEMM streams; see vocab_prefetch.
 static tt_status run_attn(const tt_dims& d, const AttnGeom& g, const AttnMaps& m,
                           const int32_t* ctx_len, tt_bf16* out, const Ws& w, const int* active,
-                          bool merge, cudaStream_t st) {
-  const AttnArgs a = attn_args(d, g, ctx_len, out, w, active);
+                          bool merge, cudaStream_t st, const tt_bf16* pf_w = nullptr) {
+  AttnArgs a = attn_args(d, g, ctx_len, out, w, active);
+  if (pf_w != nullptr && kVocabPrefetchBytes > 0) {
+    a.pf_base = reinterpret_cast<const uint8_t*>(pf_w);
+    a.pf_ld = (long long)d.H * 2;
+    a.pf_rows = d.V;
+    a.pf_tile = kVocabBN;
+    a.pf_bytes = std::min(kVocabPrefetchBytes, d.H * 2);
+  }
   TT_LAUNCH(TT_K_ATTN, st, launch_attn(m.q, m.kc, m.vc, m.kb, m.vb, a, st));
   if (merge && !g.fixup) TT_LAUNCH(TT_K_MERGE, st, launch_attn_merge(a, st));
   return TT_OK;
@@ -515,6 +566,117 @@ tt_status run_vocab_commit(const tt_dims& d, void* scratch, const tt_bf16* y, co
   return TT_OK;
 }
 
+// ------------------------------------------------------------ loop graphs
+// The block loop enqueues five or six kernels per step.  A host thread that
+// is slow to issue them (a busy host) leaves the GPU idle between them, so
+// each distinct argument set is captured once into a CUDA graph and replayed:
+// one launch per call, the same kernels with the same arguments (programmatic
+// launch edges included), so results are bitwise those of direct launches.
+// Captured on a library stream of the calling device, replayed on the
+// caller's; keyed by every argument, the attention's CTA count, the device
+// and its context identity; at most kMaxLoopGraphs kept, least recently used
+// dropped first.  Off while the profiler is on (it brackets each launch).
+struct LoopKey {
+  tt_dims d;
+  int n_layers, max_steps, n_ctas, dev;
+  unsigned long long ctx;
+  const void* p[14];
+  size_t ws_bytes;
+  uint32_t gamma_bits, scale_bits;
+};
+struct LoopGraph {
+  LoopKey key;
+  cudaGraphExec_t exec;
+  uint64_t launches, last_use;
+  int users;
+};
+constexpr size_t kMaxLoopGraphs = 32;
+constexpr int kMaxGraphDevices = 64;
+static std::mutex g_graph_mu;
+static std::vector<LoopGraph> g_graphs;
+static uint64_t g_graph_clock = 0;
+static std::atomic<bool> g_graphs_on{true};
+struct CapStream {
+  unsigned long long ctx;
+  cudaStream_t s;
+};
+static CapStream g_cap[kMaxGraphDevices];
+
+static bool key_eq(const LoopKey& a, const LoopKey& b) { return std::memcmp(&a, &b, sizeof a) == 0; }
+
+// The cached graph for `k`, marked in use (release with graph_release), or
+// nullptr.
+static LoopGraph* graph_acquire(const LoopKey& k) {
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  for (LoopGraph& e : g_graphs)
+    if (key_eq(e.key, k)) {
+      e.last_use = ++g_graph_clock;
+      ++e.users;
+      return &e;
+    }
+  return nullptr;
+}
+static void graph_release(LoopGraph* e) {
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  --e->users;
+}
+// Adds a graph (in use by the caller), replacing the least recently used
+// idle entry when full.  Every replay of a replaced graph has completed: each
+// loop call waits for its stream before it returns.
+static LoopGraph* graph_insert(const LoopKey& k, cudaGraphExec_t exec, uint64_t launches) {
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  // capacity fixed before the first entry: entries never move while in use
+  if (g_graphs.capacity() < kMaxLoopGraphs) g_graphs.reserve(kMaxLoopGraphs);
+  if (g_graphs.size() < kMaxLoopGraphs) {
+    g_graphs.push_back(LoopGraph{k, exec, launches, ++g_graph_clock, 1});
+    return &g_graphs.back();
+  }
+  LoopGraph* victim = nullptr;
+  for (LoopGraph& e : g_graphs)
+    if (e.users == 0 && (victim == nullptr || e.last_use < victim->last_use)) victim = &e;
+  if (victim == nullptr) return nullptr;  // all in use: the caller runs it uncached
+  cudaGraphExecDestroy(victim->exec);
+  *victim = LoopGraph{k, exec, launches, ++g_graph_clock, 1};
+  return victim;
+}
+static cudaStream_t capture_stream(int dev, unsigned long long ctx) {
+  std::lock_guard<std::mutex> lk(g_graph_mu);
+  CapStream& c = g_cap[dev];
+  if (c.s == nullptr || c.ctx != ctx) {
+    cudaStream_t s = nullptr;
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    c = CapStream{ctx, s};
+  }
+  return c.s;
+}
+
+// Captures enqueue(cs) into an executable graph; false (and nothing cached)
+// when capture or instantiation fails.
+template <class F>
+static bool capture_loop(F&& enqueue, cudaStream_t cs, cudaGraphExec_t* exec, uint64_t* launches) {
+  const uint64_t t0 = t_launches;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeRelaxed) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const tt_status s = enqueue(cs);
+  cudaGraph_t graph = nullptr;
+  const cudaError_t e = cudaStreamEndCapture(cs, &graph);
+  // the captured launches did not run: take them off the counters
+  const uint64_t n = t_launches - t0;
+  g_launches.fetch_sub(n, std::memory_order_relaxed);
+  t_launches = t0;
+  bool ok = s == TT_OK && e == cudaSuccess && graph != nullptr &&
+            cudaGraphInstantiate(exec, graph, 0) == cudaSuccess;
+  if (graph != nullptr) cudaGraphDestroy(graph);
+  if (!ok) cudaGetLastError();
+  *launches = n;
+  return ok;
+}
+
 }  // namespace tt
 
 using namespace tt;
@@ -562,9 +724,15 @@ tt_status tt_profile_read(int32_t kind, double* total_ms, int64_t* launches) {
   return TT_OK;
 }
 
+tt_status tt_set_loop_graphs(int32_t on) {
+  if (on != 0 && on != 1) return fail(TT_ERR_INVALID_ARG, "on=%d not 0 or 1", on);
+  g_graphs_on.store(on != 0);
+  return TT_OK;
+}
+
 tt_status tt_set_attn_splits(int32_t n_splits) {
-  if (n_splits < 0 || n_splits > 64)
-    return fail(TT_ERR_INVALID_ARG, "n_splits=%d not in [0, 64]", n_splits);
+  if (n_splits < 0 || n_splits > 1024)
+    return fail(TT_ERR_INVALID_ARG, "n_splits=%d not in [0, 1024]", n_splits);
   g_forced_splits.store(n_splits);
   return TT_OK;
 }
@@ -666,7 +834,8 @@ static tt_status denoise_block_loop_impl(
     const int32_t* ctx_len, const tt_bf16* emb, const tt_bf16* e_mask, const tt_bf16* u_t,
     const tt_bf16* shift_scale, const tt_bf16* W, float gamma, float logit_scale,
     int32_t max_steps, int32_t* tokens, uint8_t* masked, int32_t* steps_taken,
-    int32_t* commit_step, int32_t* steps_run, void* ws, size_t ws_bytes, void* stream) {
+    int32_t* commit_step, int32_t* steps_run, void* ws, size_t ws_bytes, void* stream,
+    bool allow_graph = true) {
   TT_CHECK(check_dims(d));
   TT_CHECK(check_ptr(k_ctx, "k_ctx", true));
   TT_CHECK(check_ptr(v_ctx, "v_ctx", true));
@@ -696,87 +865,145 @@ static tt_status denoise_block_loop_impl(
   const AttnGeom g = attn_geom(*d);
   const size_t ctx_elems = (size_t)d->B * d->Hkv * d->L_cap * d->dh;
 
-  // Layer 0 reads the gathered embeddings, later layers the previous
-  // layer's modulated rows (every position of the block).
-  CUtensorMap tmE, tmX;
-  if (!make_tmap_2d(&tmE, w.egath, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM) ||
-      !make_tmap_2d(&tmX, w.xrows, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM))
-    return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
-  std::vector<CUtensorMap> tmU(n_layers);
-  std::vector<AttnMaps> maps(n_layers);
-  for (int l = 0; l < n_layers; ++l) {
-    if (!make_tmap_2d(&tmU[l], u_t + (size_t)l * n_qkv * d->H, d->H, n_qkv, (uint64_t)d->H * 2,
-                      kGemmBK, kQkvBN))
-      return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
-    TT_CHECK(build_attn_maps(*d, g, w.qkv, n_qkv, w.qkv + d->H, w.qkv + d->H + d->Hkv * d->dh,
-                             n_qkv, k_ctx + (size_t)l * ctx_elems, v_ctx + (size_t)l * ctx_elems,
-                             &maps[l]));
+  // Replay of a captured graph of this exact call (see LoopKey).
+  LoopKey key;
+  std::memset(&key, 0, sizeof key);
+  int dev = 0;
+  bool use_graph = allow_graph && g_graphs_on.load() && !g_prof_on.load();
+  if (use_graph) {
+    use_graph = cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxGraphDevices &&
+                current_context_id(&key.ctx);
+    if (!use_graph) cudaGetLastError();
   }
-
-  TT_CUDA(cudaMemsetAsync(w.ctrl, 0, w.ctrl_clear, st));
-  TT_LAUNCH(TT_K_INIT, st, launch_loop_init(d->B, d->S, steps_taken, commit_step, w.ctrl, st));
-  TT_CHECK(run_attn_plan(*d, g, ctx_len, w, st));
-  // a step runs while masked positions remain (commit decrements the count)
-  const int* active = w.ctrl + CTRL_REMAINING;
-  GemmArgs ga{};
-  ga.M_alloc = rows;
-  ga.active = active;
-  ga.N = n_qkv;
-  ga.K = d->H;
-  ga.C = w.qkv;
-  ga.ldc = n_qkv;
-  ga.err = w.ctrl;
-  ga.ksplit = qkv_ksplit(*d);
-  ga.partial = w.qkv_partial;
-  ga.b_keep = 1;  // U is re-read by every step
-  const int qkv_tiles =
-      ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kQkvBN - 1) / kQkvBN) * ga.ksplit;
-  // W streams with evict-first; pinning part of it in L2 across steps was
-  // measured slower (the vocab GEMM lost ~10 us per step), so none is kept.
-  const int w_keep_tiles = 0;
-  // Step 0's plan and the embedding of every position; afterwards the commit
-  // kernel re-embeds what it commits and its last CTA plans the next step.
-  PlanArgs p{d->B, d->S, masked, w.rowlist, w.tvec, w.ctrl, 0};
-  TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
-  TT_LAUNCH(TT_K_EMBED, st, launch_embed(tokens, masked, emb, e_mask, w.egath, rows, d->H, d->V,
-                                         active, w.ctrl, st));
-  for (int step = 0; step < max_steps; ++step) {
+  if (use_graph) {
+    key.d = *d;
+    key.n_layers = n_layers;
+    key.max_steps = max_steps;
+    key.n_ctas = g.n_ctas;
+    key.dev = dev;
+    const void* ptrs[14] = {k_ctx, v_ctx, ctx_len, emb,     e_mask,      u_t,         shift_scale,
+                            W,     tokens, masked, steps_taken, commit_step, ws,          nullptr};
+    std::memcpy(key.p, ptrs, sizeof ptrs);
+    key.ws_bytes = ws_bytes;
+    std::memcpy(&key.gamma_bits, &gamma, sizeof gamma);
+    std::memcpy(&key.scale_bits, &logit_scale, sizeof logit_scale);
+  }
+  LoopGraph* cached = use_graph ? graph_acquire(key) : nullptr;
+  cudaGraphExec_t uncached = nullptr;  // captured, but the cache is full of graphs in use
+  uint64_t uncached_n = 0;
+  if (cached == nullptr) {
+    // Layer 0 reads the gathered embeddings, later layers the previous
+    // layer's modulated rows (every position of the block).
+    CUtensorMap tmE, tmX;
+    if (!make_tmap_2d(&tmE, w.egath, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM) ||
+        !make_tmap_2d(&tmX, w.xrows, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM))
+      return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
+    std::vector<CUtensorMap> tmU(n_layers);
+    std::vector<AttnMaps> maps(n_layers);
     for (int l = 0; l < n_layers; ++l) {
-      const bool last = l == n_layers - 1;
-      const tt_bf16* ss = shift_scale + (size_t)l * 2 * d->H;
-      TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(l == 0 ? tmE : tmX, tmU[l], ga,
-                                                    std::min(qkv_tiles, num_sms()), st));
-      if (ga.ksplit > 1)
-        TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
-                                                          w.qkv, n_qkv, active, st));
-      TT_CHECK(run_attn(*d, g, maps[l], ctx_len, w.attn_out, w, active, false, st));
-      // The last layer keeps the masked rows, compacted, for the vocabulary;
-      // earlier layers modulate every row (all positions are keys of the
-      // next layer).  A null row list selects the latter.
-      uint16_t* y = last ? w.y_c : w.xrows;
-      int* rl = last ? w.rowlist : nullptr;
-      if (g.fixup) {
-        TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, ss, nullptr, y, rows, d->S, d->H,
-                                               masked, rl, w.ctrl, active, st));
-      } else {
-        const AttnArgs aa = attn_args(*d, g, ctx_len, w.attn_out, w, active);
-        TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, ss, y, masked, rl, w.ctrl, st));
-      }
+      if (!make_tmap_2d(&tmU[l], u_t + (size_t)l * n_qkv * d->H, d->H, n_qkv, (uint64_t)d->H * 2,
+                        kGemmBK, kQkvBN))
+        return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
+      TT_CHECK(build_attn_maps(*d, g, w.qkv, n_qkv, w.qkv + d->H, w.qkv + d->H + d->Hkv * d->dh,
+                               n_qkv, k_ctx + (size_t)l * ctx_elems, v_ctx + (size_t)l * ctx_elems,
+                               &maps[l]));
     }
-    TT_CHECK(run_vocab_gemm(*d, w, W, logit_scale, w.ctrl + CTRL_M, active, w_keep_tiles, st));
-    CommitArgs c = commit_args(*d, w, gamma, logit_scale, tokens, masked);
-    c.commit_step = commit_step;
-    c.steps_taken = steps_taken;
-    c.step = step;
-    c.active = active;
-    c.emb = emb;
-    c.egath = w.egath;
-    c.H = d->H;
-    c.plan_next = 1;
-    TT_LAUNCH(TT_K_COMMIT, st, launch_commit(c, st));
+
+    auto enqueue = [&](cudaStream_t st) -> tt_status {
+      TT_CUDA(cudaMemsetAsync(w.ctrl, 0, w.ctrl_clear, st));
+      TT_LAUNCH(TT_K_INIT, st, launch_loop_init(d->B, d->S, steps_taken, commit_step, w.ctrl, st));
+      TT_CHECK(run_attn_plan(*d, g, ctx_len, w, st));
+      // a step runs while masked positions remain (commit decrements the count)
+      const int* active = w.ctrl + CTRL_REMAINING;
+      GemmArgs ga{};
+      ga.M_alloc = rows;
+      ga.active = active;
+      ga.N = n_qkv;
+      ga.K = d->H;
+      ga.C = w.qkv;
+      ga.ldc = n_qkv;
+      ga.err = w.ctrl;
+      ga.ksplit = qkv_ksplit(*d);
+      ga.partial = w.qkv_partial;
+      ga.b_keep = 1;  // U is re-read by every step
+      const int qkv_tiles =
+          ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kQkvBN - 1) / kQkvBN) * ga.ksplit;
+      // W streams with evict-first; pinning part of it in L2 across steps was
+      // measured slower (the vocab GEMM lost ~10 us per step), so none is kept.
+      const int w_keep_tiles = 0;
+      const bool pf_w = vocab_prefetch(*d, attn_args(*d, g, ctx_len, w.attn_out, w, active));
+      // Step 0's plan and the embedding of every position; afterwards the commit
+      // kernel re-embeds what it commits and its last CTA plans the next step.
+      PlanArgs p{d->B, d->S, masked, w.rowlist, w.tvec, w.ctrl, 0};
+      TT_LAUNCH(TT_K_PLAN, st, launch_plan(p, st));
+      TT_LAUNCH(TT_K_EMBED, st, launch_embed(tokens, masked, emb, e_mask, w.egath, rows, d->H, d->V,
+                                             active, w.ctrl, st));
+      for (int step = 0; step < max_steps; ++step) {
+        for (int l = 0; l < n_layers; ++l) {
+          const bool last = l == n_layers - 1;
+          const tt_bf16* ss = shift_scale + (size_t)l * 2 * d->H;
+          TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(l == 0 ? tmE : tmX, tmU[l], ga,
+                                                        std::min(qkv_tiles, num_sms()), st));
+          if (ga.ksplit > 1)
+            TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
+                                                              w.qkv, n_qkv, active, st));
+          TT_CHECK(run_attn(*d, g, maps[l], ctx_len, w.attn_out, w, active, false, st,
+                            last && pf_w ? W : nullptr));
+          // The last layer keeps the masked rows, compacted, for the vocabulary;
+          // earlier layers modulate every row (all positions are keys of the
+          // next layer).  A null row list selects the latter.
+          uint16_t* y = last ? w.y_c : w.xrows;
+          int* rl = last ? w.rowlist : nullptr;
+          if (g.fixup) {
+            TT_LAUNCH(TT_K_ADALN, st, launch_adaln(w.attn_out, ss, nullptr, y, rows, d->S, d->H,
+                                                   masked, rl, w.ctrl, active, st));
+          } else {
+            const AttnArgs aa = attn_args(*d, g, ctx_len, w.attn_out, w, active);
+            TT_LAUNCH(TT_K_ADALN, st, launch_merge_adaln(aa, ss, y, masked, rl, w.ctrl, st));
+          }
+        }
+        TT_CHECK(run_vocab_gemm(*d, w, W, logit_scale, w.ctrl + CTRL_M, active, w_keep_tiles, st));
+        CommitArgs c = commit_args(*d, w, gamma, logit_scale, tokens, masked);
+        c.commit_step = commit_step;
+        c.steps_taken = steps_taken;
+        c.step = step;
+        c.active = active;
+        c.emb = emb;
+        c.egath = w.egath;
+        c.H = d->H;
+        c.plan_next = 1;
+        TT_LAUNCH(TT_K_COMMIT, st, launch_commit(c, st));
+      }
+      return TT_OK;
+    };
+    cudaGraphExec_t exec = nullptr;
+    uint64_t n = 0;
+    cudaStream_t cs = use_graph ? capture_stream(dev, key.ctx) : nullptr;
+    if (cs != nullptr && capture_loop(enqueue, cs, &exec, &n)) {
+      cached = graph_insert(key, exec, n);
+      if (cached == nullptr) {
+        uncached = exec;
+        uncached_n = n;
+      }
+    } else {
+      TT_CHECK(enqueue(st));
+    }
+  }
+  cudaGraphExec_t run = cached != nullptr ? cached->exec : uncached;
+  if (run != nullptr) {
+    const cudaError_t e = cudaGraphLaunch(run, st);
+    count_launch((int)(cached != nullptr ? cached->launches : uncached_n));
+    if (e != cudaSuccess) {
+      if (cached != nullptr) graph_release(cached);
+      if (uncached != nullptr) cudaGraphExecDestroy(uncached);
+      return fail(TT_ERR_CUDA, "cudaGraphLaunch failed: %s", cudaGetErrorString(e));
+    }
   }
   int h[8];
-  TT_CHECK(read_ctrl(w, st, h));
+  const tt_status rs = read_ctrl(w, st, h);
+  if (cached != nullptr) graph_release(cached);
+  if (uncached != nullptr) cudaGraphExecDestroy(uncached);
+  TT_CHECK(rs);
   if (g_prof_on.load()) prof_harvest();
   if (steps_run != nullptr) *steps_run = h[CTRL_STEPS_RUN];
   if (h[CTRL_ERR] != 0)
@@ -887,7 +1114,8 @@ tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx, t
     TT_CHECK(denoise_block_loop_impl(d, 1, k_ctx, v_ctx, ctx_len, emb, e_mask, u_t, shift_scale,
                                      W, gamma, logit_scale, d->S, tok, w.blk_masked,
                                      steps_taken + (size_t)j * d->B,
-                                     commit_step + (size_t)j * rows, &n, ws, ws_bytes, stream));
+                                     commit_step + (size_t)j * rows, &n, ws, ws_bytes, stream,
+                                     /*allow_graph=*/false));
     total_steps += n;
     // The committed block joins the context: its rows of the workspace's
     // embeddings are Emb[token] (the commit re-embeds what it commits), so

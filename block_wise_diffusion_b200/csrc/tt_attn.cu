@@ -169,16 +169,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
-__device__ __forceinline__ float max16(const uint32_t (&v)[16]) {
-  float a = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
-  float b = fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
-  a = fmax3(a, __uint_as_float(v[6]), __uint_as_float(v[7]));
-  b = fmax3(b, __uint_as_float(v[8]), __uint_as_float(v[9]));
-  a = fmax3(a, __uint_as_float(v[10]), __uint_as_float(v[11]));
-  b = fmax3(b, __uint_as_float(v[12]), __uint_as_float(v[13]));
-  return fmax3(fmaxf(a, b), __uint_as_float(v[14]), __uint_as_float(v[15]));
-}
-
 // P for 16 score columns as 8 bf16 pairs, written in place: pair j/2 goes to
 // sv[j] (the registers of S it came from are dead by then); the last pair
 // on the FMA pipe.
@@ -275,6 +265,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   if (a.active != nullptr && *a.active == 0) return;
   const int cta = blockIdx.x;
+  // HBM is mostly idle while this kernel runs on an L2-resident context:
+  // warm L2 with the head of the W rows the vocabulary GEMM's CTA `cta`
+  // streams first.  Issued by the softmax warps (threads 128..), which
+  // wait for the first S anyway, not by the producers.
+  if (a.pf_bytes > 0 && threadIdx.x >= 128) {
+    const int r1 = min(a.pf_rows, (cta + 1) * a.pf_tile);
+    for (int r = cta * a.pf_tile + (int)threadIdx.x - 128; r < r1; r += (int)blockDim.x - 128)
+      prefetch_l2_bulk(a.pf_base + (long long)r * a.pf_ld, (uint32_t)a.pf_bytes);
+  }
   const long long T = a.tile_start[a.units];
   const int lo = (int)((long long)cta * T / a.n_ctas);
   const int hi = (int)((long long)(cta + 1) * T / a.n_ctas);

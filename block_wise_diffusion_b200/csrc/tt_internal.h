@@ -15,6 +15,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per bounded wait
 // e.g. when workspace sizes are computed on a host without a GPU.
 constexpr int kDefaultSMs = 148;
 int num_sms();
+// Identity of the calling thread's current CUDA context (cuCtxGetId); false
+// when no context is current or the driver lacks the call.
+bool current_context_id(unsigned long long* id);
 
 // Control block: the first 256 bytes of every workspace.
 enum CtrlWord {
@@ -130,6 +133,12 @@ struct AttnArgs {
   float* part_ml;       // [units + n_ctas - 1][256][4]: running max (log2 units), the row
                         // sums of key columns 0..63 and 64..127 of every tile, unused
   int* err;
+  // Optional L2 prefetch of the next vocabulary GEMM's first W tiles (pf_bytes
+  // = 0: none): CTA c prefetches the first pf_bytes of each of rows
+  // [c * pf_tile, (c + 1) * pf_tile) of W (pf_rows rows, pf_ld bytes apart).
+  const uint8_t* pf_base;
+  long long pf_ld;
+  int pf_rows, pf_tile, pf_bytes;
 };
 size_t attn_smem_bytes(int dh, int halves);
 cudaError_t launch_attn_plan(const AttnArgs& a, cudaStream_t st);

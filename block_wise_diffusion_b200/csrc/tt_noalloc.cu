@@ -11,8 +11,6 @@
 // GPU that loads it until the process exits.  The work itself is the kernel
 // sequence of tt_vocab_confidence_commit (run_vocab_commit), carved from the
 // array instead of a caller's workspace.
-#include <cudaTypedefs.h>
-
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -27,31 +25,6 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB per device
 // The scratch.  In host code this name is only a stand-in for the device
 // array: its device address must come from cudaGetSymbolAddress.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-
-// Identity of the calling thread's current CUDA context (cuCtxGetId: unique
-// for the life of the process, so a context destroyed by a device reset and
-// created again gets a new one).  False when no context is current yet or
-// the driver lacks the call.
-bool current_context_id(unsigned long long* id) {
-  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
-  static PFN_cuCtxGetId_v12000 get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
-    p = nullptr;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
-  });
-  if (get_cur == nullptr || get_id == nullptr) return false;
-  CUcontext ctx = nullptr;
-  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
-  return get_id(ctx, id) == CUDA_SUCCESS;
-}
 
 constexpr int kMaxDevices = 128;
 struct AddrSlot {

@@ -98,11 +98,19 @@ TT_API tt_status tt_selftest_timeout(void* ws, int32_t limit_us, void* stream);
 /* Number of kernels this library has launched in this process so far. */
 TT_API uint64_t tt_launch_count(void);
 
-/* Number of CTAs the attention's key tiles are divided over (0 = one per SM,
- * the default; otherwise at most 64): all units' tiles, laid end to end, are
- * cut into that many equal contiguous ranges.  Process-wide; results are
- * independent of it up to float rounding. */
+/* Number of CTAs the attention's key tiles are divided over (0 = the
+ * library's choice, the default; otherwise at most 1024, CTAs beyond the
+ * SM count running in later waves): all units' tiles, laid end to end, are
+ * cut into that many equal contiguous ranges.  Process-wide, read when a
+ * workspace is sized and when a call runs, so set it before sizing the
+ * workspace; results are independent of it up to float rounding. */
 TT_API tt_status tt_set_attn_splits(int32_t n_splits);
+
+/* 1 (the default): tt_denoise_block_loop and tt_denoise_block_loop_layers
+ * replay a captured CUDA graph per argument set; 0: they launch every kernel
+ * directly (as they also do while the profiler is on).  Process-wide.  Any
+ * other value is TT_ERR_INVALID_ARG. */
+TT_API tt_status tt_set_loop_graphs(int32_t on);
 
 /* Kernel kinds of the per-kernel profiler. */
 enum {
@@ -224,6 +232,12 @@ TT_API tt_status tt_vocab_confidence_commit(const tt_dims* d, const tt_bf16* y, 
  *   ws           workspace of at least tt_workspace_bytes(d, TT_WS_LOOP) bytes
  * Blocking: returns after the stream has finished the loop (one host
  * synchronisation at the end, none per step).
+ * Launch: the first call with a given set of arguments (every pointer and
+ * size, gamma, logit_scale, max_steps, the attention's CTA count) captures
+ * its kernel sequence into a CUDA graph on a library stream; later calls with
+ * the same set replay it on `stream` as one launch (results bitwise those of
+ * direct launches).  Up to 32 sets are kept per process; see
+ * tt_set_loop_graphs.
  */
 TT_API tt_status tt_denoise_block_loop(const tt_dims* d, const tt_bf16* k_ctx, const tt_bf16* v_ctx,
                                 const int32_t* ctx_len, const tt_bf16* emb,

@@ -95,8 +95,10 @@ int main(void) {
   }
 
   /* the attention split knob is process-wide and bounded */
-  CHECK(tt_set_attn_splits(65) == TT_ERR_INVALID_ARG);
+  CHECK(tt_set_attn_splits(1025) == TT_ERR_INVALID_ARG);
   CHECK(tt_set_attn_splits(0) == TT_OK);
+  CHECK(tt_set_loop_graphs(2) == TT_ERR_INVALID_ARG);
+  CHECK(tt_set_loop_graphs(1) == TT_OK);
 
   /* none of the refused calls launched anything */
   CHECK(tt_launch_count() == 0);

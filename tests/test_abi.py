@@ -133,9 +133,16 @@ def test_commit_and_loop_argument_checks(L):
     assert n_rows.value == -3                               # nothing written on refusal
 
 
+def test_loop_graph_knob(L):
+    with pytest.raises(tt.TTError):
+        tt.tt_set_loop_graphs(2)
+    tt.tt_set_loop_graphs(0)
+    tt.tt_set_loop_graphs(1)
+
+
 def test_split_knob(L):
     with pytest.raises(tt.TTError):
-        tt.tt_set_attn_splits(65)
+        tt.tt_set_attn_splits(1025)
     d = _d(B=1, L_cap=65536)
     tt.tt_set_attn_splits(1)
     one = tt.tt_workspace_bytes(d, tt.TT_WS_ATTN)

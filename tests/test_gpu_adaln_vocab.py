@@ -130,6 +130,18 @@ def test_vocab_commit_ragged_vocab_and_partial_mask():
     assert n_der <= 1, n_der                      # at most one of the 4 masked sequences
 
 
+@pytest.mark.parametrize("V", [2, 3])
+def test_vocab_commit_smallest_vocabularies(V):
+    """The bottom of the accepted envelope: a vocabulary of 2 or 3 tokens, one
+    224-wide tile almost all past V."""
+    d = tt_inputs.Dims(B=4, S=16, Hq=4, Hkv=1, dh=64, V=V, L_cap=0)
+    got, ref, m, tok = _vocab_case(d, 24, 3.0, 0.6)
+    n_spec, n_der = _check_commit(got, ref, m, tok, 0.6)
+    print(f"V={V}: spec-excluded {n_spec}, test-excluded sequences {n_der}")
+    assert n_der <= 1, n_der
+    assert np.all((got["tok"][m.astype(bool)] >= 0) & (got["tok"][m.astype(bool)] < V))
+
+
 def test_vocab_planted_argmax_ties_pick_lowest_id():
     d = tt_inputs.workload("tiny", B=2)
     inp = tt_inputs.generate(d, seed=23, names=["w"])

@@ -74,6 +74,14 @@ CASES = [
                                    ctx=("fixed", 150)), np.array([150]), True),
     ("gqa128-H8192", tt_inputs.Dims(B=2, S=32, Hq=128, Hkv=1, dh=64, V=512, L_cap=200,
                                     ctx=("fixed", 200)), np.array([200, 3]), True),
+    # the rest of the envelope's edges: one query head per KV head (G = 1), a
+    # batch of 200 sequences, a context longer than 65536 keys
+    ("g1", tt_inputs.Dims(B=2, S=16, Hq=4, Hkv=4, dh=64, V=512, L_cap=300,
+                          ctx=("fixed", 300)), np.array([300, 17]), True),
+    ("batch200", tt_inputs.Dims(B=200, S=16, Hq=4, Hkv=1, dh=64, V=512, L_cap=130,
+                                ctx=("uniform", 0, 130)), None, False),
+    ("L70000", tt_inputs.Dims(B=1, S=16, Hq=4, Hkv=1, dh=64, V=512, L_cap=70000,
+                              ctx=("fixed", 70000)), None, False),
 ]
 
 

@@ -327,6 +327,47 @@ def test_loop_widest_hidden_and_group(logit_scale):
     assert n_cmp > 0 and n_ex <= 2, (n_cmp, n_ex)
 
 
+@pytest.mark.parametrize("wl,logit_scale", [("tiny", 12.0), ("mid", 1.0)])
+def test_loop_graph_replay_equals_direct_launches(wl, logit_scale):
+    """The loop replays one captured CUDA graph per argument set: the first
+    call captures and replays, later calls with the same buffers replay.  All
+    give bitwise the state of direct launches, and each call counts the same
+    kernels."""
+    d = tt_inputs.workload(wl, precommit=("uniform", 0.0, 0.75)) if wl == "tiny" else \
+        tt_inputs.workload(wl, B=2, L_cap=512, ctx=("fixed", 512))
+    inp = tt_inputs.generate(d, seed=46)
+    D = tt.dims(d)
+    dv = {k: G.dev_bf16(inp[k]) for k in LOOP_INPUTS}
+    cl = G.dev(inp["ctx_len"])
+    tok0, msk0 = G.dev(inp["tokens"]), G.dev(inp["masked"])
+    tokens, masked = tok0.clone(), msk0.clone()
+    steps_taken = torch.empty((d.B,), dtype=torch.int32, device="cuda")
+    commit_step = torch.empty((d.B, d.S), dtype=torch.int32, device="cuda")
+    ws = G.workspace(D, tt.TT_WS_LOOP)
+
+    def call():
+        tokens.copy_(tok0)
+        masked.copy_(msk0)
+        n0 = tt.tt_launch_count()
+        n = tt.tt_denoise_block_loop(D, dv["k_ctx"], dv["v_ctx"], cl, dv["emb"], dv["e_mask"],
+                                     dv["u_t"], dv["shift_scale"], dv["w"], 0.8, logit_scale, d.S,
+                                     tokens, masked, steps_taken, commit_step, ws)
+        return (n, tt.tt_launch_count() - n0, tokens.cpu().numpy(), masked.cpu().numpy(),
+                steps_taken.cpu().numpy(), commit_step.cpu().numpy())
+
+    tt.tt_set_loop_graphs(0)
+    try:
+        direct = call()
+    finally:
+        tt.tt_set_loop_graphs(1)
+    first, second, third = call(), call(), call()
+    for got in (first, second, third):
+        assert got[0] == direct[0] and got[1] == direct[1], (got[:2], direct[:2])
+        for a, b in zip(got[2:], direct[2:]):
+            np.testing.assert_array_equal(a, b)
+    assert not direct[3].any()
+
+
 def test_loop_canonical_scale_commits_in_position_order():
     d = tt_inputs.workload("tiny", B=2)
     inp = tt_inputs.generate(d, seed=32)
