@@ -400,7 +400,7 @@ static tt_status build_attn_maps(const tt_dims& d, const AttnGeom& g, const tt_b
 
 static AttnArgs attn_args(const tt_dims& d, const AttnGeom& g, const int32_t* ctx_len,
                           tt_bf16* out, const Ws& w, const int* active) {
-  AttnArgs a;
+  AttnArgs a{};  // every field not set below (the optional prefetch) is zero
   a.B = d.B;
   a.S = d.S;
   a.Hq = d.Hq;
