@@ -355,6 +355,11 @@ def test_loop_graph_replay_equals_direct_launches(wl, logit_scale):
         return (n, tt.tt_launch_count() - n0, tokens.cpu().numpy(), masked.cpu().numpy(),
                 steps_taken.cpu().numpy(), commit_step.cpu().numpy())
 
+    def same(got, ref):
+        assert got[0] == ref[0] and got[1] == ref[1], (got[:2], ref[:2])
+        for a, b in zip(got[2:], ref[2:]):
+            np.testing.assert_array_equal(a, b)
+
     tt.tt_set_loop_graphs(0)
     try:
         direct = call()
@@ -362,10 +367,29 @@ def test_loop_graph_replay_equals_direct_launches(wl, logit_scale):
         tt.tt_set_loop_graphs(1)
     first, second, third = call(), call(), call()
     for got in (first, second, third):
-        assert got[0] == direct[0] and got[1] == direct[1], (got[:2], direct[:2])
-        for a, b in zip(got[2:], direct[2:]):
-            np.testing.assert_array_equal(a, b)
+        same(got, direct)
     assert not direct[3].any()
+    # the same buffers with another logit scale, or another attention CTA
+    # count, are other argument sets: no stale graph may be replayed
+    logit_scale, saved = logit_scale * 3.0, logit_scale
+    tt.tt_set_loop_graphs(0)
+    try:
+        direct2 = call()
+    finally:
+        tt.tt_set_loop_graphs(1)
+    same(call(), direct2)
+    logit_scale = saved
+    tt.tt_set_attn_splits(37)
+    try:
+        tt.tt_set_loop_graphs(0)
+        try:
+            direct3 = call()
+        finally:
+            tt.tt_set_loop_graphs(1)
+        same(call(), direct3)
+    finally:
+        tt.tt_set_attn_splits(0)
+    same(call(), direct)
 
 
 def test_loop_canonical_scale_commits_in_position_order():
