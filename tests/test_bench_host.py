@@ -115,3 +115,23 @@ def test_both_roofs_reports_each_view():
     ms = [1024 - 64 * k for k in range(16)]
     v = bench.both_roofs("gemm_vocab", d, inp, ms, 16, 450e-6, PEAKS)
     assert v["tensor"]["flops_per_launch"] == sum(2.0 * m * d.V * d.H for m in ms) / 16
+
+
+def test_clock_sampler_keeps_the_samples_of_the_timed_region():
+    """The sampler starts before the warm-up; only samples stamped inside the
+    timed region count (the nearest one on each side when it is shorter than
+    the sampling period), and throttle reasons are read from those."""
+    s = bench.ClockSampler(None)   # no nvidia-smi: fill in stamped lines by hand
+    line = "{mhz}, 1965, {w}, Not Active, Not Active, Not Active, {cap}\n"
+    s.lines = [(10.0, line.format(mhz=1965, w=300, cap="Not Active")),   # warm-up
+               (10.2, line.format(mhz=1500, w=990, cap="Active")),       # timed
+               (10.4, line.format(mhz=1520, w=995, cap="Active")),       # timed
+               (10.6, line.format(mhz=1965, w=150, cap="Not Active"))]   # after
+    s.proc = type("P", (), {"terminate": lambda self: None, "wait": lambda self, timeout=None: 0,
+                            "kill": lambda self: None})()
+    got = s.stop(10.1, 10.45)
+    assert got["samples"] == 2 and got["sm_mhz"] == 1510.0
+    assert got["reasons"] == ["sw_power_cap"] and got["sm_max_mhz"] == 1965.0
+    # a region between two samples: the samples on either side
+    got = s.stop(10.25, 10.3)
+    assert got["samples"] == 2 and got["sm_mhz"] == 1510.0
