@@ -267,7 +267,8 @@ static AttnGeom attn_geom(const tt_dims& d) {
 // the SMs when the block has few rows; a power of two dividing H/64.
 static int ksplit_for(const tt_dims& d, int n_out) {
   const int rows = d.B * d.S;
-  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_out + kQkvBN - 1) / kQkvBN);
+  const int bn = qkv_bn(rows);
+  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_out + bn - 1) / bn);
   const int kb = d.H / kGemmBK;
   const int sms = num_sms();
   int k = 1;
@@ -279,8 +280,9 @@ static int qkv_ksplit(const tt_dims& d) { return ksplit_for(d, d.H + 2 * d.Hkv *
 static int ctx_ksplit(const tt_dims& d) { return ksplit_for(d, 2 * d.Hkv * d.dh); }
 static size_t splitk_bytes(const tt_dims& d, int n_out, int ks) {
   const size_t rows = (size_t)d.B * d.S;
-  const size_t tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_out + kQkvBN - 1) / kQkvBN);
-  return ks > 1 ? (size_t)ks * tiles * kGemmBM * kQkvBN * sizeof(float) : 0;
+  const size_t bn = (size_t)qkv_bn((int)rows);
+  const size_t tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_out + bn - 1) / bn);
+  return ks > 1 ? (size_t)ks * tiles * kGemmBM * bn * sizeof(float) : 0;
 }
 
 struct Carver {
@@ -353,7 +355,7 @@ static Ws carve(const tt_dims& d, int which, void* ws) {
     w.xrows = c.take<uint16_t>(rows * d.H * 2);
     w.qkv = c.take<uint16_t>(rows * n_qkv * 2);
     w.attn_out = c.take<uint16_t>(rows * d.H * 2);
-    // tile-major partials: ks planes of whole 128 x kQkvBN tiles, for the
+    // tile-major partials: ks planes of whole 128 x qkv_bn(rows) tiles, for the
     // linear update or the context projection, whichever needs more
     const size_t pb = std::max(splitk_bytes(d, (int)n_qkv, qkv_ksplit(d)),
                                splitk_bytes(d, 2 * d.Hkv * d.dh, ctx_ksplit(d)));
@@ -902,7 +904,7 @@ static tt_status denoise_block_loop_impl(
     std::vector<AttnMaps> maps(n_layers);
     for (int l = 0; l < n_layers; ++l) {
       if (!make_tmap_2d(&tmU[l], u_t + (size_t)l * n_qkv * d->H, d->H, n_qkv, (uint64_t)d->H * 2,
-                        kGemmBK, kQkvBN))
+                        kGemmBK, qkv_bn(rows)))
         return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the linear update");
       TT_CHECK(build_attn_maps(*d, g, w.qkv, n_qkv, w.qkv + d->H, w.qkv + d->H + d->Hkv * d->dh,
                                n_qkv, k_ctx + (size_t)l * ctx_elems, v_ctx + (size_t)l * ctx_elems,
@@ -927,7 +929,8 @@ static tt_status denoise_block_loop_impl(
       ga.partial = w.qkv_partial;
       ga.b_keep = 1;  // U is re-read by every step
       const int qkv_tiles =
-          ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + kQkvBN - 1) / kQkvBN) * ga.ksplit;
+          ((rows + kGemmBM - 1) / kGemmBM) * ((n_qkv + qkv_bn(rows) - 1) / qkv_bn(rows)) *
+          ga.ksplit;
       // W streams with evict-first; pinning part of it in L2 across steps was
       // measured slower (the vocab GEMM lost ~10 us per step), so none is kept.
       const int w_keep_tiles = 0;
@@ -943,10 +946,12 @@ static tt_status denoise_block_loop_impl(
           const bool last = l == n_layers - 1;
           const tt_bf16* ss = shift_scale + (size_t)l * 2 * d->H;
           TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(l == 0 ? tmE : tmX, tmU[l], ga,
-                                                        std::min(qkv_tiles, num_sms()), st));
+                                                        std::min(qkv_tiles, num_sms()),
+                                                        qkv_bn(rows), st));
           if (ga.ksplit > 1)
             TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_qkv,
-                                                              w.qkv, n_qkv, active, st));
+                                                              w.qkv, n_qkv, active, qkv_bn(rows),
+                                                              st));
           TT_CHECK(run_attn(*d, g, maps[l], ctx_len, w.attn_out, w, active, false, st,
                             last && pf_w ? W : nullptr));
           // The last layer keeps the masked rows, compacted, for the vocabulary;
@@ -1092,7 +1097,7 @@ tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx, t
   const int n_kv = 2 * d->Hkv * d->dh;
   CUtensorMap tmE, tmC;
   if (!make_tmap_2d(&tmE, w.egath, d->H, rows, (uint64_t)d->H * 2, kGemmBK, kGemmBM) ||
-      !make_tmap_2d(&tmC, u_ctx, d->H, n_kv, (uint64_t)d->H * 2, kGemmBK, kQkvBN))
+      !make_tmap_2d(&tmC, u_ctx, d->H, n_kv, (uint64_t)d->H * 2, kGemmBK, qkv_bn(rows)))
     return fail(TT_ERR_CUDA, "cuTensorMapEncodeTiled failed for the context projection");
   GemmArgs ga{};
   ga.M_alloc = rows;
@@ -1103,7 +1108,8 @@ tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx, t
   ga.err = w.ctrl;
   ga.ksplit = ctx_ksplit(*d);
   ga.partial = w.qkv_partial;
-  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_kv + kQkvBN - 1) / kQkvBN) * ga.ksplit;
+  const int bn = qkv_bn(rows);
+  const int tiles = ((rows + kGemmBM - 1) / kGemmBM) * ((n_kv + bn - 1) / bn) * ga.ksplit;
   int total_steps = 0;
   for (int j = 0; j < n_blocks; ++j) {
     int32_t* tok = tokens + (size_t)j * rows;
@@ -1120,10 +1126,11 @@ tt_status tt_decode_blocks(const tt_dims* d, int32_t n_blocks, tt_bf16* k_ctx, t
     // The committed block joins the context: its rows of the workspace's
     // embeddings are Emb[token] (the commit re-embeds what it commits), so
     // [k | v] = Emb[token] . U_ctx^T, appended at each sequence's end.
-    TT_LAUNCH(TT_K_GEMM_QKV, st, launch_gemm_bf16(tmE, tmC, ga, std::min(tiles, num_sms()), st));
+    TT_LAUNCH(TT_K_GEMM_QKV, st,
+              launch_gemm_bf16(tmE, tmC, ga, std::min(tiles, num_sms()), bn, st));
     if (ga.ksplit > 1)
       TT_LAUNCH(TT_K_REDUCE, st, launch_splitk_reduce(w.qkv_partial, ga.ksplit, rows, n_kv,
-                                                        w.qkv, n_kv, nullptr, st));
+                                                        w.qkv, n_kv, nullptr, bn, st));
     TT_LAUNCH(TT_K_APPEND, st, launch_append_kv(w.qkv, n_kv, k_ctx, v_ctx, ctx_len, d->B, d->S,
                                                 d->Hkv, d->dh, d->L_cap, w.ctrl, st));
     // the next block's loop clears the control block: check this append now

@@ -326,16 +326,25 @@ cudaError_t launch_gemm_vocab(const CUtensorMap& tmA, const CUtensorMap& tmB, co
   return launch_gemm<0, kVocabBN, kVocabStages>(tmA, tmB, a, grid, st);
 }
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                             int grid, cudaStream_t st) {
+                             int grid, int bn, cudaStream_t st) {
+  if (bn == kQkvBNSmall)
+    return launch_gemm<1, kQkvBNSmall, kQkvStagesSmall>(tmA, tmB, a, grid, st);
   return launch_gemm<1, kQkvBN, kQkvStages>(tmA, tmB, a, grid, st);
 }
 
-cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int N, uint16_t* C,
+template <int BN>
+static cudaError_t launch_reduce(const float* partial, int ksplit, int rows, int N, uint16_t* C,
                                  int ldc, const int* active, cudaStream_t st) {
-  const long long tiles = (long long)((rows + kGemmBM - 1) / kGemmBM) * ((N + kQkvBN - 1) / kQkvBN);
-  const long long threads = tiles * (kQkvBN / 8) * kGemmBM;
-  return launch_k(splitk_reduce_kernel<kQkvBN>, dim3((unsigned)((threads + 255) / 256)), dim3(256),
-                  0, st, partial, ksplit, rows, N, C, ldc, active);
+  const long long tiles = (long long)((rows + kGemmBM - 1) / kGemmBM) * ((N + BN - 1) / BN);
+  const long long threads = tiles * (BN / 8) * kGemmBM;
+  return launch_k(splitk_reduce_kernel<BN>, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0,
+                  st, partial, ksplit, rows, N, C, ldc, active);
+}
+cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int N, uint16_t* C,
+                                 int ldc, const int* active, int bn, cudaStream_t st) {
+  if (bn == kQkvBNSmall)
+    return launch_reduce<kQkvBNSmall>(partial, ksplit, rows, N, C, ldc, active, st);
+  return launch_reduce<kQkvBN>(partial, ksplit, rows, N, C, ldc, active, st);
 }
 
 }  // namespace tt

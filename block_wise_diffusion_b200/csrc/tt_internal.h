@@ -51,10 +51,14 @@ enum WhereTag {
 // vocabulary GEMM uses N tiles of 224 columns (131072 columns -> 586 tiles,
 // 3.96 per SM, so the last round is nearly full) with a 5-deep ring; the
 // linear update uses 256-column tiles (4608 columns x 1024 rows -> 144
-// tiles, one wave) with a 4-deep ring.
+// tiles, one wave) with a 4-deep ring when the block has several row tiles,
+// and 128-column tiles with a 6-deep ring when it has one (the K split that
+// fills the SMs is then half as deep, and so are its fp32 partials).
 constexpr int kGemmBM = 128, kGemmBK = 64;
 constexpr int kVocabBN = 224, kVocabStages = 5;
 constexpr int kQkvBN = 256, kQkvStages = 4;
+constexpr int kQkvBNSmall = 128, kQkvStagesSmall = 6;
+inline int qkv_bn(int rows) { return rows <= kGemmBM ? kQkvBNSmall : kQkvBN; }
 constexpr int kGemmThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue
 constexpr size_t gemm_smem_bytes(int bn, int stages) {
   return (size_t)stages * (kGemmBM + bn) * kGemmBK * 2 + 1024 + 256;
@@ -85,11 +89,13 @@ struct GemmArgs {
 
 cudaError_t launch_gemm_vocab(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
                               int grid, cudaStream_t st);
+// bn: kQkvBN or kQkvBNSmall (the B tensor map's box height)
 cudaError_t launch_gemm_bf16(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a,
-                             int grid, cudaStream_t st);
-// C[r, :] = bf16(sum_k partial[k][r][:]) for r < rows (N multiple of 8).
+                             int grid, int bn, cudaStream_t st);
+// C[r, :] = bf16(sum_k partial[k][r][:]) for r < rows (N multiple of 8), the
+// partials tile-major in tiles of bn columns.
 cudaError_t launch_splitk_reduce(const float* partial, int ksplit, int rows, int N, uint16_t* C,
-                                 int ldc, const int* active, cudaStream_t st);
+                                 int ldc, const int* active, int bn, cudaStream_t st);
 
 // ------------------------------------------------------------- attention
 constexpr int kAttnBN = 128;       // keys per tile
